@@ -1,0 +1,221 @@
+"""ctypes wrapper over the fp64 C oracle (``pkv_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY (tests, smoke check, CPU-baseline leg of the
+benchmark).  Inputs are CPU arrays: 16-bit caches and queries are passed as
+their raw bit patterns (numpy ``uint16``, or a CPU torch ``float16`` /
+``bfloat16`` tensor which is reinterpreted without conversion).  Outputs of
+the attention functions are numpy ``float64``.
+
+Every function follows the C oracle's definition; see the comments there for
+the passages of the pages each one restates.
+"""
+import ctypes as C
+
+import numpy as np
+
+from . import build_oracle
+
+F16, BF16 = 0, 1
+_DTYPES = {"f16": F16, "float16": F16, "fp16": F16, "bf16": BF16, "bfloat16": BF16}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = build_oracle.build()
+        L = C.CDLL(path)
+        p = C.c_void_p
+        i = C.c_int
+        i64 = C.c_int64
+        d = C.c_double
+        L.pkv_oracle_bf16_to_f64.argtypes = [C.c_uint16]
+        L.pkv_oracle_bf16_to_f64.restype = d
+        L.pkv_oracle_f16_to_f64.argtypes = [C.c_uint16]
+        L.pkv_oracle_f16_to_f64.restype = d
+        L.pkv_oracle_decode_attention.argtypes = [p, p, p, p, p, i, p, i, i, i, i, i, i, i64, d, i, i]
+        L.pkv_oracle_decode_partials.argtypes = [p, p, p, p, p, p, p, i, p, i, i, i, i, i, i, i64, d, i, i, i]
+        L.pkv_oracle_merge_partials.argtypes = [p, p, p, p, p, i, i, i, i, i]
+        L.pkv_oracle_write_slots.argtypes = [p, p, p, p, p, i, i, i, i, i, i64]
+        L.pkv_oracle_copy_blocks.argtypes = [p, p, p, i, i, i, i, i, i64]
+        L.pkv_oracle_block_bytes.argtypes = [i, i, i, i, i]
+        L.pkv_oracle_block_bytes.restype = i64
+        L.pkv_oracle_max_threads.argtypes = []
+        for name in ("pkv_oracle_decode_attention", "pkv_oracle_decode_partials",
+                     "pkv_oracle_merge_partials", "pkv_oracle_write_slots",
+                     "pkv_oracle_copy_blocks", "pkv_oracle_max_threads"):
+            getattr(L, name).restype = i
+        _lib = L
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _dtype_code(dtype):
+    if isinstance(dtype, int):
+        return dtype
+    name = str(dtype).replace("torch.", "")
+    return _DTYPES[name]
+
+
+def bits(x):
+    """Raw 16-bit patterns of ``x`` as a C-contiguous numpy uint16 array."""
+    if isinstance(x, np.ndarray):
+        if x.dtype == np.uint16:
+            return np.ascontiguousarray(x)
+        if x.dtype == np.float16:
+            return np.ascontiguousarray(x).view(np.uint16)
+        raise TypeError("expected uint16 bits or float16, got %s" % x.dtype)
+    # torch tensor (kept duck-typed so this module does not need torch)
+    t = x.detach().cpu().contiguous()
+    import torch
+
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _ptr(a):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _i32(a):
+    a = np.ascontiguousarray(np.asarray(a), dtype=np.int32)
+    return a
+
+
+def _i64(a):
+    return np.ascontiguousarray(np.asarray(a), dtype=np.int64)
+
+
+def _num_blocks(size, block_stride, block_elems):
+    """Blocks that fit in a flat buffer of ``size`` elements whose blocks of
+    ``block_elems`` elements start ``block_stride`` elements apart."""
+    if size < block_elems:
+        return 0
+    return (size - block_elems) // block_stride + 1
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise OracleError("%s: oracle rejected the input (status %d)" % (what, rc))
+
+
+def bf16_to_f64(b):
+    return lib().pkv_oracle_bf16_to_f64(int(b))
+
+
+def f16_to_f64(b):
+    return lib().pkv_oracle_f16_to_f64(int(b))
+
+
+def decode_attention(query, key_cache, value_cache, block_tables, context_lens,
+                     scale, dtype, num_kv_heads, block_size, block_stride=None,
+                     num_threads=0):
+    """Paged decode attention in fp64.
+
+    query ``[S, Hq, D]``; caches hold ``NB`` blocks of ``[bs, Hkv, D]`` at
+    ``block_stride`` elements apart (default: contiguous blocks);
+    block_tables ``int32 [S, MB]``; context_lens ``int32 [S]``.
+    Returns ``float64 [S, Hq, D]``.
+    """
+    q = bits(query)
+    kc = bits(key_cache)
+    vc = bits(value_cache)
+    S, Hq, D = q.shape
+    tables = _i32(block_tables)
+    lens = _i32(context_lens)
+    MB = tables.shape[1] if tables.ndim == 2 else 0
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    rc = lib().pkv_oracle_decode_attention(
+        _ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables), MB, _ptr(lens), S,
+        Hq, num_kv_heads, D, NB, block_size, block_stride, float(scale),
+        _dtype_code(dtype), int(num_threads))
+    _check(rc, "decode_attention")
+    return out
+
+
+def decode_partials(query, key_cache, value_cache, block_tables, context_lens,
+                    scale, dtype, num_kv_heads, block_size, partition_size,
+                    num_partitions, block_stride=None):
+    """Per-partition (m, l, o) in fp64: token ranges [pP, min((p+1)P, L))."""
+    q = bits(query)
+    kc = bits(key_cache)
+    vc = bits(value_cache)
+    S, Hq, D = q.shape
+    tables = _i32(block_tables)
+    lens = _i32(context_lens)
+    MB = tables.shape[1]
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    NP = int(num_partitions)
+    m = np.zeros((S, Hq, NP), dtype=np.float64)
+    l = np.zeros((S, Hq, NP), dtype=np.float64)
+    o = np.zeros((S, Hq, NP, D), dtype=np.float64)
+    rc = lib().pkv_oracle_decode_partials(
+        _ptr(m), _ptr(l), _ptr(o), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables), MB,
+        _ptr(lens), S, Hq, num_kv_heads, D, NB, block_size, block_stride,
+        float(scale), _dtype_code(dtype), int(partition_size), NP)
+    _check(rc, "decode_partials")
+    return m, l, o
+
+
+def merge_partials(m, l, o, context_lens, partition_size):
+    m = np.ascontiguousarray(m, dtype=np.float64)
+    l = np.ascontiguousarray(l, dtype=np.float64)
+    o = np.ascontiguousarray(o, dtype=np.float64)
+    lens = _i32(context_lens)
+    S, Hq, NP, D = o.shape
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    rc = lib().pkv_oracle_merge_partials(_ptr(out), _ptr(m), _ptr(l), _ptr(o),
+                                         _ptr(lens), S, Hq, D, int(partition_size), NP)
+    _check(rc, "merge_partials")
+    return out
+
+
+def write_slots(key_cache, value_cache, key, value, slot_mapping, block_size,
+                num_kv_heads, block_stride=None):
+    """Returns new (key_cache, value_cache) bit arrays with the tokens written."""
+    kc = bits(key_cache).copy()
+    vc = bits(value_cache).copy()
+    k = bits(key)
+    v = bits(value)
+    slots = _i64(slot_mapping)
+    T = slots.shape[0]
+    D = k.shape[-1]
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    rc = lib().pkv_oracle_write_slots(_ptr(kc), _ptr(vc), _ptr(k), _ptr(v), _ptr(slots),
+                                      T, NB, block_size, num_kv_heads, D, block_stride)
+    _check(rc, "write_slots")
+    return kc, vc
+
+
+def copy_blocks(key_cache, value_cache, block_pairs, block_size, num_kv_heads,
+                head_dim, block_stride=None):
+    """Returns new (key_cache, value_cache) bit arrays after the copies."""
+    kc = bits(key_cache).copy()
+    vc = bits(value_cache).copy()
+    pairs = _i32(block_pairs).reshape(-1, 2)
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * head_dim
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * head_dim)
+    rc = lib().pkv_oracle_copy_blocks(_ptr(kc), _ptr(vc), _ptr(pairs), pairs.shape[0],
+                                      NB, block_size, num_kv_heads, head_dim, block_stride)
+    _check(rc, "copy_blocks")
+    return kc, vc
+
+
+def block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):
+    return int(lib().pkv_oracle_block_bytes(block_size, num_kv_heads, head_dim,
+                                            num_layers, dtype_bytes))
+
+
+def max_threads():
+    return int(lib().pkv_oracle_max_threads())
