@@ -1,0 +1,520 @@
+#!/usr/bin/env python
+"""Benchmark of one decode step of the paged KV cache hot path.
+
+A step, for every sequence of the batch: the host pool reserves the new
+token's slot (copy-on-write pairs where a block is shared), the new token's
+K/V rows are written into the cache (pkv_write_slots), and paged decode
+attention runs over the whole context through the Block Tables
+(pkv_decode_attention: one pass, or split-K partitions plus a merge).  The
+workload is the 7B-shaped decode batch: 256 sequences, 32 query = 32 KV
+heads, head_dim 128, block size 16, context lengths U[128, 2048], bf16,
+blocks scattered over a pool of 1.1x the blocks needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pkv|reference]
+
+`value` is effective GB/s of algorithmic bytes (every context token's K and V
+read once, plus queries, outputs, table rows, the slot write and any
+workspace traffic) over device time, with all inputs resident in HBM.  `e2e`
+is the same metric through the public step API from pinned host buffers,
+host allocator and copies included.  Under torchrun each rank runs its own
+batch (weak scaling, no collective on the data path) and the time is the
+maximum over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "paged decode attention effective KV GB/s (% of HBM peak); decode tok/s"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
+    ap.add_argument("--workload", default="7b_s256_h32_d128_bs16_bf16")
+    ap.add_argument("--partition-size", type=int, default=-1,
+                    help="tokens per split-K partition (0: one pass; -1: the workload's)")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="profiling only: run the workload's first N sequences")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# byte accounting (algorithmic bytes, not DRAM traffic)
+# ---------------------------------------------------------------------------
+def decode_bytes(spec, lens, partition_size):
+    """Bytes paged decode attention must move for one step: each context
+    token's K and V once, queries, outputs, the table entries it follows,
+    the context lengths, and with split-K the fp32 partials written and read
+    back by the merge."""
+    dtb = 2
+    S, Hq, Hkv, D, bs = (spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
+                         spec.block_size)
+    kv = sum(lens) * Hkv * D * 2 * dtb
+    qo = 2 * S * Hq * D * dtb
+    table = sum(-(-L // bs) for L in lens) * 4 + S * 4
+    ws = 0
+    maxlen = max(lens)
+    if partition_size and partition_size < maxlen:
+        nparts = sum(-(-L // partition_size) if L > partition_size else 0 for L in lens)
+        ws = nparts * Hq * (D + 2) * 4 * 2
+    return kv + qo + table + ws
+
+
+def write_bytes(spec, num_tokens):
+    """Slot write: new K and V rows read and written, plus the slots."""
+    return num_tokens * spec.num_kv_heads * spec.head_dim * 2 * 2 * 2 + num_tokens * 8
+
+
+def copy_bytes(spec, num_pairs):
+    return num_pairs * spec.block_size * spec.num_kv_heads * spec.head_dim * 2 * 2 * 2
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.index = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except OSError:
+            return None
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def profiled_traffic(source_digest):
+    """DRAM bytes per launch of the decode kernel from the committed ncu
+    summary, or None when that summary is missing or was taken on other
+    kernel source."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            text = f.read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        line = line.strip().strip("`").strip("-").strip()
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256") != source_digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+def kernel_source_digest():
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in ("decode_attention.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_337_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline, not a target)
+# ---------------------------------------------------------------------------
+def oracle_sample_problem(spec, lens, seed):
+    """A compact copy of the workload's first sequences for the CPU oracle:
+    the same lengths and shapes, scattered over a small pool."""
+    import numpy as np
+
+    g = torch.Generator().manual_seed(seed)
+    bs = spec.block_size
+    need = sum(-(-L // bs) for L in lens)
+    nb = need + 1
+    perm = torch.randperm(nb, generator=g).tolist()
+    mb = max(-(-L // bs) for L in lens)
+    tables = np.full((len(lens), mb), -1, np.int32)
+    i = 0
+    for s, L in enumerate(lens):
+        for j in range(-(-L // bs)):
+            tables[s, j] = perm[i]
+            i += 1
+    dt = spec.torch_dtype
+    shape = (nb, bs, spec.num_kv_heads, spec.head_dim)
+    kc = torch.randn(shape, generator=g).to(dt)
+    vc = torch.randn(shape, generator=g).to(dt)
+    q = torch.randn(len(lens), spec.num_q_heads, spec.head_dim, generator=g).to(dt)
+    return q, kc, vc, tables, np.asarray(lens, np.int32)
+
+
+def time_oracle(spec, lens, target_s):
+    """Times the fp64 oracle (all host cores) on the first n sequences, n
+    grown until one call takes about target_s seconds.  Returns (GB/s,
+    seconds, n, cores)."""
+    from oracle import reference as ref
+
+    n = 1
+    while True:
+        q, kc, vc, tables, l = oracle_sample_problem(spec, lens[:n], 7)
+        t0 = time.perf_counter()
+        ref.decode_attention(q, kc, vc, tables, l, spec.scale, spec.dtype, spec.num_kv_heads,
+                             spec.block_size, num_threads=0)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or n >= len(lens):
+            byts = decode_bytes(spec, list(lens[:n]), 0)
+            return byts / dt / 1e9, dt, n, ref.max_threads()
+        n = min(len(lens), max(n + 1, int(n * target_s / max(dt, 1e-3))))
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the oracle as it stands, on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, spec, world, rank):
+    if rank != 0:
+        return
+    from paged_kv_cache_337_b200 import workloads as W
+
+    gen = torch.Generator("cpu").manual_seed(spec.seed)
+    lens = W.draw_lens(spec, gen).tolist()
+    per_step = max(0.2, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    gbs, dt, n, cores = time_oracle(spec, lens, per_step)
+    q, kc, vc, tables, l = oracle_sample_problem(spec, lens[:n], 11)
+    from oracle import reference as ref
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        ref.decode_attention(q, kc, vc, tables, l, spec.scale, spec.dtype, spec.num_kv_heads,
+                             spec.block_size, num_threads=0)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    byts = decode_bytes(spec, lens[:n], 0)
+    value = byts * len(times) / sum(times) / 1e9
+    sample = "first %d of %d sequences (all %d query heads), one decode step each" % (
+        n, spec.num_seqs, spec.num_q_heads)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name, "oracle": "fp64 C oracle, OpenMP over (seq, head)",
+                   "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the product arm
+# ---------------------------------------------------------------------------
+def run_pkv(args, spec, world, rank, local):
+    from paged_kv_cache_337_b200 import _abi
+    from paged_kv_cache_337_b200 import workloads as W
+    from paged_kv_cache_337_b200.cache import PagedKVCache
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _abi.lib()
+    P = spec.partition_size if args.partition_size < 0 else args.partition_size
+
+    # seeded shapes on the CPU; cache values drawn on the device (per rank)
+    gen = torch.Generator("cpu").manual_seed(spec.seed)
+    lens0 = W.draw_lens(spec, gen).tolist()
+    nb = W.pool_size(spec, lens0)
+    order = torch.randperm(nb, generator=gen, dtype=torch.int64).to(torch.int32)
+    S, Hq, Hkv, D, bs = (spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
+                         spec.block_size)
+    n_states = 16  # decode steps whose metadata is prepared (one block's worth)
+    e2e_steps = 0 if args.no_e2e else min(args.steps, 48)
+    mb = spec.max_blocks_per_seq + -(-(n_states + e2e_steps + 2) // bs)
+    cache = PagedKVCache(nb, bs, Hq, Hkv, D, spec.torch_dtype, dev, mb, P,
+                         free_order=order.tolist(), scale=spec.scale)
+    W.fill_device_cache_(cache.key_cache, spec.seed * 10 + 2 * rank)
+    W.fill_device_cache_(cache.value_cache, spec.seed * 10 + 2 * rank + 1)
+    ids = list(range(S))
+    for s in ids:
+        cache.add_sequence(s, lens0[s] - 1)
+
+    stream = torch.cuda.Stream(dev)
+    dgen = torch.Generator(dev).manual_seed(spec.seed + 100 * rank)
+    dt = spec.torch_dtype
+
+    # prepare n_states consecutive steps: the host pool really appends one
+    # token per sequence each time; the step replays them cyclically
+    states = []
+    for j in range(n_states):
+        prep = cache.prepare_step(ids)
+        st = prep["st"]
+        npairs = prep["num_pairs"]
+        lens = st["h_lens"].tolist()
+        states.append(dict(
+            slots=st["h_slots"].to(dev), pairs=st["h_pairs"][:npairs].to(dev),
+            tables=st["h_tables"].to(dev), lens=st["h_lens"].to(dev), max_len=max(lens),
+            q=torch.randn((S, Hq, D), generator=dgen, device=dev).to(dt),
+            k=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
+            v=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
+            bytes_decode=decode_bytes(spec, lens, P),
+            bytes_step=decode_bytes(spec, lens, P) + write_bytes(spec, S) +
+            copy_bytes(spec, npairs), npairs=npairs, lens_sum=sum(lens)))
+    max_len_all = max(s["max_len"] for s in states)
+    ws_bytes = _abi.pkv_decode_workspace_bytes(S, Hq, max_len_all, P, D)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
+    out = torch.empty((S, Hq, D), dtype=dt, device=dev)
+    err = cache.dev_error
+    kc, vc = cache.key_cache, cache.value_cache
+
+    def step(state, ev=None):
+        if state["npairs"]:
+            _abi.pkv_copy_blocks(kc, vc, state["pairs"], dev_error=err, stream=stream)
+        _abi.pkv_write_slots(state["k"], state["v"], kc, vc, state["slots"], dev_error=err,
+                             stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        _abi.pkv_decode_attention(out, state["q"], kc, vc, state["tables"], state["lens"],
+                                  state["max_len"], spec.scale, P, ws, dev_error=err,
+                                  stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        return (1 if state["npairs"] else 0) + 1 + (2 if ws is not None else 1)
+
+    for i in range(args.warmup):
+        step(states[i % n_states])
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    bytes_step = bytes_decode = 0
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(K):
+        stt = states[(args.warmup + i) % n_states]
+        launches += step(stt, evs[i])
+        bytes_step += stt["bytes_step"]
+        bytes_decode += stt["bytes_decode"]
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clock_info = clocks.stop() if clocks else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    decode_ms = sum(a.elapsed_time(b) for a, b in evs)
+    cache.check_errors()
+
+    t_max = max_over_ranks(elapsed_ms, world, dev)
+    total_bytes = sum_over_ranks(bytes_step, world, dev)
+    value = total_bytes / (t_max * 1e-3) / 1e9
+    ms_per_step = t_max / K
+    decode_gbs = bytes_decode / (decode_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    tok_s = world * S * K / (t_max * 1e-3)
+
+    # ---- end to end through the public step API from pinned host memory ----
+    e2e = None
+    if e2e_steps:
+        hq = [torch.randn((S, Hq, D)).to(dt).pin_memory() for _ in range(2)]
+        hk = [torch.randn((S, Hkv, D)).to(dt).pin_memory() for _ in range(2)]
+        hv = [torch.randn((S, Hkv, D)).to(dt).pin_memory() for _ in range(2)]
+        hout = torch.empty((S, Hq, D), dtype=dt).pin_memory()
+        dq = torch.empty((S, Hq, D), dtype=dt, device=dev)
+        dk = torch.empty((S, Hkv, D), dtype=dt, device=dev)
+        dv = torch.empty((S, Hkv, D), dtype=dt, device=dev)
+        e2e_bytes = 0
+        h2d = d2h = 0
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for i in range(e2e_steps):
+                dq.copy_(hq[i % 2], non_blocking=True)
+                dk.copy_(hk[i % 2], non_blocking=True)
+                dv.copy_(hv[i % 2], non_blocking=True)
+                prep = cache.prepare_step(ids)
+                cache.upload_step(prep, stream)
+                cache.launch_step(prep, dq, dk, dv, out, stream=stream)
+                hout.copy_(out, non_blocking=True)
+                stream.synchronize()
+                lens = prep["st"]["h_lens"].tolist()
+                e2e_bytes += (decode_bytes(spec, lens, P) + write_bytes(spec, S) +
+                              copy_bytes(spec, prep["num_pairs"]))
+                h2d = (dq.numel() + dk.numel() + dv.numel()) * 2 + S * (8 + 4) + \
+                    prep["st"]["h_tables"].numel() * 4 + prep["num_pairs"] * 8
+                d2h = hout.numel() * 2
+        e2e_s = time.perf_counter() - t0
+        barrier(world)
+        e2e_s = max_over_ranks(e2e_s, world, dev)
+        e2e_total = sum_over_ranks(e2e_bytes, world, dev)
+        e2e = {"value": round(e2e_total / e2e_s / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": e2e_steps, "ms_per_step": round(1e3 * e2e_s / e2e_steps, 4)}
+        cache.check_errors()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, secs, n, cores = time_oracle(spec, lens0, 10.0)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": "first %d of %d sequences (all %d query heads), one decode step, "
+                         "%.1f s" % (n, S, Hq, secs)}
+
+    if rank == 0:
+        traffic = profiled_traffic(kernel_source_digest())
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if dt == torch.bfloat16 else "f16", "data": "synthetic",
+            "config": {
+                "workload": spec.name, "num_seqs": S, "num_q_heads": Hq, "num_kv_heads": Hkv,
+                "head_dim": D, "block_size": bs, "context_lens": "U[%d,%d]" % (spec.len_lo,
+                                                                             spec.len_hi),
+                "pool_blocks": nb, "partition_size": P,
+                "step": "host slot append + slot write + paged decode attention"
+                        " (+ copy-on-write copies, split-K merge)",
+                "l2": "inputs larger than L2 (%.2f GB of K/V read per step)" % (
+                    states[0]["lens_sum"] * Hkv * D * 4 / 1e9),
+                "states": "%d consecutive decode steps prepared by the host pool, replayed "
+                          "cyclically" % n_states},
+            "pct_hbm_peak": round(100 * value / (world * peak), 2),
+            "decode_tok_s": round(tok_s, 1),
+            "roofline": {"bound": "hbm", "achieved": round(decode_gbs, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(decode_gbs / peak, 4),
+                         "traffic": traffic, "kernel": "paged_decode_kernel",
+                         "peak_source": peak_kind},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    from paged_kv_cache_337_b200 import workloads as W
+
+    spec = W.SPECS[args.workload]
+    if args.num_seqs:
+        import dataclasses
+
+        spec = dataclasses.replace(spec, num_seqs=args.num_seqs,
+                                   name="%s_first%d" % (spec.name, args.num_seqs))
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, spec, world, rank)
+        else:
+            run_pkv(args, spec, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

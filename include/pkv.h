@@ -1,0 +1,273 @@
+/*
+ * pkv.h — C ABI of the B200 paged KV cache library (libpkv.so).
+ *
+ * The library implements the data-parallel hot path of PagedAttention as the
+ * pages describe it:
+ *   - a physical block pool with per-sequence Block Tables, refcounts and
+ *     copy-on-write ("Paged KV" wiki page, sections 实现原理 / 初始化阶段 and
+ *     运行阶段; "PagedAttention 动态内存分页" page, sections 块粒度与块表,
+ *     写时复制与内存共享, 动态块分配与回收);
+ *   - the slot-mapped write of each new token's K/V (运行阶段);
+ *   - decode attention that reads K/V block by block through the Block Table
+ *     ("Paged KV" wiki page, section Attention Kernel 的适配);
+ *   - the copy of a shared block before a sequence writes into it.
+ *
+ * Conventions shared by every entry point
+ *   - Every function returns a pkv_status (0 on success) and never throws.
+ *     pkv_last_error() gives a message for the calling thread's last failure.
+ *   - Device memory is owned by the caller: the library allocates none, and
+ *     every pointer it is given stays the caller's.  Kernels run
+ *     asynchronously on the caller's stream; a host-side argument error is
+ *     reported before anything is launched.
+ *   - Cache layout: K and V are separate caches, each a sequence of physical
+ *     blocks of shape [block_size, num_kv_heads, head_dim] (contiguous inside
+ *     a block), block b starting block_stride ELEMENTS after block 0.  A plain
+ *     [num_blocks, block_size, num_kv_heads, head_dim] tensor has
+ *     block_stride = block_size * num_kv_heads * head_dim; a combined or
+ *     multi-layer tensor passes a larger stride (a multiple of 8 elements).
+ *   - A slot is physical_block * block_size + offset.
+ *   - dev_error, where taken, is NULL or a device int32[2] that the caller
+ *     zeroes; a kernel that meets bad metadata records the first problem as
+ *     {code, index} (PKV_DEVERR_*), skips that piece of work and carries on.
+ *     No kernel traps.
+ *   - Supported: fp16 and bf16 storage; head_dim 64 or 128 for attention
+ *     (any multiple of 8 for the write and the copy); block_size a multiple
+ *     of 16 up to 256 for attention (any positive size for the write and the
+ *     copy); num_q_heads / num_kv_heads from 1 to 16.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID = -1,     /* bad argument: shape, pointer, alignment, id */
+    PKV_ERR_UNSUPPORTED = -2, /* valid but not built: dtype, head_dim, ... */
+    PKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+    PKV_ERR_OOM = -4,         /* the block pool has too few free blocks */
+    PKV_ERR_WORKSPACE = -5    /* workspace missing or too small */
+} pkv_status;
+
+typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Codes a kernel writes into dev_error[0]; dev_error[1] gets the index. */
+#define PKV_DEVERR_NONE 0
+#define PKV_DEVERR_CONTEXT_LEN 1 /* index: seq; len < 0, > max_context_len or > table */
+#define PKV_DEVERR_BLOCK_ID 2    /* index: seq; a table entry outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT 3        /* index: token; slot >= num_blocks * block_size */
+#define PKV_DEVERR_PAIR 4        /* index: pair; a block id outside [0, num_blocks) */
+#define PKV_DEVERR_TIMEOUT 5     /* index: 0; a bounded wait on a copy ran out */
+
+/* ---------------------------------------------------------------------- */
+/* Slot write                                                              */
+/* ---------------------------------------------------------------------- */
+/*
+ * Writes the K and V rows of num_tokens new tokens into their slots
+ * ("Paged KV" wiki page, 实现原理 / 运行阶段: each decoded token goes to the
+ * next slot of the sequence's current block; prefill fills blocks in order).
+ *
+ *   key, value     device, [num_tokens, num_kv_heads, head_dim], contiguous
+ *   key_cache,     device caches in the layout above (num_blocks blocks)
+ *   value_cache
+ *   slot_mapping   device int64 [num_tokens]; token t goes to block
+ *                  slot / block_size, offset slot % block_size; a negative
+ *                  slot writes nothing.  Slots must be distinct (else which
+ *                  token lands is unspecified).  A slot >= num_blocks *
+ *                  block_size is skipped and reported (PKV_DEVERR_SLOT).
+ *   All pointers 16-byte aligned; num_kv_heads * head_dim a multiple of 8.
+ */
+PKV_API int pkv_write_slots(const void* key, const void* value, void* key_cache,
+                    void* value_cache, const int64_t* slot_mapping,
+                    int num_tokens, int num_blocks, int block_size,
+                    int num_kv_heads, int head_dim, int64_t block_stride,
+                    pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Copy-on-write block copy                                                */
+/* ---------------------------------------------------------------------- */
+/*
+ * For every pair (src, dst), block dst of both caches becomes a copy of
+ * block src: all block_size slots of all heads ("PagedAttention 动态内存
+ * 分页" page, 写时复制与内存共享: a block shared by several sequences is copied
+ * when one of them needs to write into it).
+ *
+ *   block_pairs  device int32 [num_pairs, 2] = (src, dst).  Pairs run
+ *                concurrently: destinations must be distinct and no
+ *                destination may be another pair's source.  A pair naming a
+ *                block outside [0, num_blocks) is skipped and reported
+ *                (PKV_DEVERR_PAIR).
+ *   Cache pointers 16-byte aligned, block_stride a multiple of 8 elements.
+ */
+PKV_API int pkv_copy_blocks(void* key_cache, void* value_cache,
+                    const int32_t* block_pairs, int num_pairs, int num_blocks,
+                    int block_size, int num_kv_heads, int head_dim,
+                    int64_t block_stride, pkv_dtype dtype, int32_t* dev_error,
+                    cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Paged decode attention                                                  */
+/* ---------------------------------------------------------------------- */
+/*
+ * Bytes of workspace pkv_decode_attention needs for these sizes (0 when every
+ * sequence fits one partition, i.e. partition_size == 0 or
+ * partition_size >= max_context_len).  The workspace holds, per (seq, query
+ * head, partition), the fp32 running maximum, sum and unnormalised output.
+ */
+PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads,
+                                  int max_context_len, int partition_size,
+                                  int head_dim);
+
+/*
+ * One decode step of attention for num_seqs sequences, one query token each
+ * ("Paged KV" wiki page, Attention Kernel 的适配: besides the usual inputs the
+ * kernel takes the Block Table and block_size and reads K/V block by block
+ * through that indirection).  For sequence s and query head h, with
+ * kv = h / (num_q_heads / num_kv_heads) and L = context_lens[s]:
+ *     out[s, h] = sum_t softmax_t(scale * <query[s, h], K_t>) V_t,  t < L,
+ * where token t is slot t % block_size of physical block
+ * block_tables[s, t / block_size].  L counts every cached token, the one
+ * written this step included.  L == 0 gives zeros.
+ *
+ *   out, query       device [num_seqs, num_q_heads, head_dim], dtype
+ *   key_cache,       device caches (layout above); 16-byte aligned
+ *   value_cache
+ *   block_tables     device int32 [num_seqs, max_blocks_per_seq]; only the
+ *                    first ceil(L / block_size) entries of a row are read
+ *   context_lens     device int32 [num_seqs]
+ *   max_context_len  host copy of max(context_lens) (or any bound on it):
+ *                    it sizes the grid; a longer sequence is reported
+ *                    (PKV_DEVERR_CONTEXT_LEN) and gets zeros
+ *   scale            multiplies the dot product before the softmax
+ *   partition_size   0: one pass per sequence.  Otherwise a multiple of 16:
+ *                    each sequence is split into partitions of that many
+ *                    tokens that run in parallel, and a second kernel merges
+ *                    their fp32 partial results (split-K for long contexts).
+ *   workspace        device scratch of pkv_decode_workspace_bytes() bytes,
+ *                    16-byte aligned (may be NULL when that is 0); its
+ *                    contents on entry and exit are unspecified
+ * Returns PKV_ERR_UNSUPPORTED for a head_dim, block_size or group size that
+ * is not built, PKV_ERR_WORKSPACE when the workspace is too small.
+ */
+PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_cache,
+                         const void* value_cache, const int32_t* block_tables,
+                         int max_blocks_per_seq, const int32_t* context_lens,
+                         int num_seqs, int max_context_len, int num_q_heads,
+                         int num_kv_heads, int head_dim, int num_blocks,
+                         int block_size, int64_t block_stride, float scale,
+                         int partition_size, void* workspace,
+                         size_t workspace_bytes, pkv_dtype dtype,
+                         int32_t* dev_error, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Host block pool (allocator)                                             */
+/* ---------------------------------------------------------------------- */
+/*
+ * One global pool of num_blocks physical blocks, from which sequences take
+ * blocks on demand and to which they return them ("一文读懂vLLM的…
+ * PagedAttention" page, 运行模式的根本转变; "Paged KV" wiki page, 初始化阶段
+ * and 运行阶段; "PagedAttention 动态内存分页" page, 块粒度与块表, 写时复制与内存
+ * 共享, 动态块分配与回收).  Policy where the pages are silent: the free pool is a
+ * LIFO stack; a fresh pool hands out free_order[0], free_order[1], ... (or
+ * 0, 1, ... when free_order is NULL); freed blocks are pushed in table order;
+ * an operation that runs out of blocks returns PKV_ERR_OOM and changes
+ * nothing.  Not thread-safe: the caller serialises calls on one pool.
+ * All pointers here are host pointers.
+ */
+typedef struct pkv_pool pkv_pool;
+
+/* free_order: NULL or a permutation of 0..num_blocks-1 (host int32). */
+PKV_API int pkv_pool_create(int num_blocks, int block_size, const int32_t* free_order,
+                    pkv_pool** out);
+PKV_API void pkv_pool_destroy(pkv_pool* pool);
+
+/* Prefill: a new sequence of num_tokens tokens takes ceil(num_tokens /
+ * block_size) blocks in pool order.  PKV_ERR_INVALID if seq_id exists. */
+PKV_API int pkv_seq_add(pkv_pool* pool, int64_t seq_id, int num_tokens);
+
+/* The child shares every block of the parent (refcount + 1 each). */
+PKV_API int pkv_seq_fork(pkv_pool* pool, int64_t parent, int64_t child);
+
+/* Reserves the slot of one new token of seq_id.  When the current block is
+ * full a new block is appended to the table.  When the current block is
+ * shared (refcount > 1) it is replaced by a fresh block, *cow_src / *cow_dst
+ * receive the pair to copy with pkv_copy_blocks before the write, and the
+ * old block loses one reference; otherwise both are set to -1. */
+PKV_API int pkv_seq_append(pkv_pool* pool, int64_t seq_id, int64_t* slot,
+                   int32_t* cow_src, int32_t* cow_dst);
+
+/* pkv_seq_append for n sequences in order.  slots[i] receives the slot of
+ * seq_ids[i]; the copy pairs are packed into cow_pairs (capacity n pairs,
+ * int32 [n, 2]) and counted in *num_cow.  Stops at the first failure, with
+ * *num_done (may be NULL) appends completed. */
+PKV_API int pkv_seq_append_batch(pkv_pool* pool, int n, const int64_t* seq_ids,
+                         int64_t* slots, int32_t* cow_pairs, int* num_cow,
+                         int* num_done);
+
+/* Drops the sequence's reference to each of its blocks; blocks that reach
+ * refcount 0 return to the pool. */
+PKV_API int pkv_seq_free(pkv_pool* pool, int64_t seq_id);
+
+PKV_API int pkv_seq_num_tokens(const pkv_pool* pool, int64_t seq_id, int* num_tokens);
+
+/* Slots of tokens [first_token, first_token + num_tokens) of the sequence, in
+ * order, into out (host int64): slot = table[t / block_size] * block_size +
+ * t % block_size.  The range must lie inside the sequence.  Used to write a
+ * prompt's K/V after pkv_seq_add ("Paged KV" wiki page, 运行阶段: prefill
+ * fills the blocks it took, in order). */
+PKV_API int pkv_seq_slot_mapping(const pkv_pool* pool, int64_t seq_id, int first_token,
+                                 int num_tokens, int64_t* out);
+
+/* Copies the sequence's Block Table (physical ids in logical order) into
+ * out[0..cap); *n receives its length (PKV_ERR_INVALID if cap < length). */
+PKV_API int pkv_seq_block_table(const pkv_pool* pool, int64_t seq_id, int32_t* out,
+                        int cap, int* n);
+
+/* Fills a dense [n, max_blocks_per_seq] table for seq_ids (rows padded with
+ * `fill`) and, if context_lens is not NULL, their token counts. */
+PKV_API int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t* seq_ids,
+                          int32_t* out, int max_blocks_per_seq, int32_t fill,
+                          int32_t* context_lens);
+
+PKV_API int pkv_pool_num_free(const pkv_pool* pool);
+PKV_API int pkv_pool_num_blocks(const pkv_pool* pool);
+PKV_API int pkv_pool_block_size(const pkv_pool* pool);
+
+/* The free stack from bottom to top (the next block taken is the last). */
+PKV_API int pkv_pool_free_list(const pkv_pool* pool, int32_t* out, int cap, int* n);
+
+/* Refcount of a block (number of tables holding it), or a negative status. */
+PKV_API int pkv_block_refcount(const pkv_pool* pool, int block);
+
+/* ---------------------------------------------------------------------- */
+/* Sizing and diagnostics                                                  */
+/* ---------------------------------------------------------------------- */
+/* Bytes of one physical block over all layers ("Paged KV" wiki page,
+ * 初始化阶段): block_size * num_kv_heads * head_dim * 2 (K and V) *
+ * num_layers * dtype_bytes.  Negative on bad arguments. */
+PKV_API int64_t pkv_block_bytes(int block_size, int num_kv_heads, int head_dim,
+                        int num_layers, int dtype_bytes);
+
+PKV_API const char* pkv_status_string(int status);
+/* Message of the calling thread's last failed call ("" if none). */
+PKV_API const char* pkv_last_error(void);
+/* Library version as major * 10000 + minor * 100 + patch. */
+PKV_API int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PKV_H */

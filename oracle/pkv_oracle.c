@@ -168,7 +168,7 @@ int pkv_oracle_decode_attention(double* out, const uint16_t* query,
     const int G = Hq / Hkv;
     int bad = 0;
 #ifdef _OPENMP
-    if (num_threads > 0) omp_set_num_threads(num_threads);
+    omp_set_num_threads(num_threads > 0 ? num_threads : omp_get_num_procs());
 #else
     (void)num_threads;
 #endif

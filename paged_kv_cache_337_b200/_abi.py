@@ -1,0 +1,351 @@
+"""ctypes binding of ``libpkv.so`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+work of its own beyond reading shapes, strides and pointers off torch tensors:
+the computation runs in the library's CUDA kernels and C++ allocator.  There
+is no fallback: if the library is missing, every call raises.
+"""
+import ctypes as C
+import os
+
+import torch
+
+from . import build as _build
+
+PKV_OK = 0
+PKV_ERR_INVALID = -1
+PKV_ERR_UNSUPPORTED = -2
+PKV_ERR_CUDA = -3
+PKV_ERR_OOM = -4
+PKV_ERR_WORKSPACE = -5
+
+PKV_F16 = 0
+PKV_BF16 = 1
+
+PKV_DEVERR_NONE = 0
+PKV_DEVERR_CONTEXT_LEN = 1
+PKV_DEVERR_BLOCK_ID = 2
+PKV_DEVERR_SLOT = 3
+PKV_DEVERR_PAIR = 4
+PKV_DEVERR_TIMEOUT = 5
+
+_DTYPE = {torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+
+# name -> (restype, argtypes)
+_p, _i, _i64, _sz, _f = C.c_void_p, C.c_int, C.c_int64, C.c_size_t, C.c_float
+SIGNATURES = {
+    "pkv_write_slots": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p, _p]),
+    "pkv_copy_blocks": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p, _p]),
+    "pkv_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "pkv_decode_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
+                                  _i64, _f, _i, _p, _sz, _i, _p, _p]),
+    "pkv_pool_create": (_i, [_i, _i, _p, C.POINTER(_p)]),
+    "pkv_pool_destroy": (None, [_p]),
+    "pkv_seq_add": (_i, [_p, _i64, _i]),
+    "pkv_seq_fork": (_i, [_p, _i64, _i64]),
+    "pkv_seq_append": (_i, [_p, _i64, _p, _p, _p]),
+    "pkv_seq_append_batch": (_i, [_p, _i, _p, _p, _p, _p, _p]),
+    "pkv_seq_free": (_i, [_p, _i64]),
+    "pkv_seq_num_tokens": (_i, [_p, _i64, _p]),
+    "pkv_seq_block_table": (_i, [_p, _i64, _p, _i, _p]),
+    "pkv_seq_slot_mapping": (_i, [_p, _i64, _i, _i, _p]),
+    "pkv_pool_block_tables": (_i, [_p, _i, _p, _p, _i, C.c_int32, _p]),
+    "pkv_pool_num_free": (_i, [_p]),
+    "pkv_pool_num_blocks": (_i, [_p]),
+    "pkv_pool_block_size": (_i, [_p]),
+    "pkv_pool_free_list": (_i, [_p, _p, _i, _p]),
+    "pkv_block_refcount": (_i, [_p, _i]),
+    "pkv_block_bytes": (_i64, [_i, _i, _i, _i, _i]),
+    "pkv_status_string": (C.c_char_p, [_i]),
+    "pkv_last_error": (C.c_char_p, []),
+    "pkv_version": (_i, []),
+}
+
+_lib = None
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(what)
+
+
+def library_path():
+    return _build.LIB
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                "libpkv.so is not built (%s); run `python -m paged_kv_cache_337_b200.build`" % path)
+        L = C.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status, name):
+    if status != PKV_OK:
+        msg = lib().pkv_last_error().decode(errors="replace")
+        raise PkvError(status, "%s: %s (%s)" % (name, lib().pkv_status_string(status).decode(), msg))
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _cache_geometry(cache):
+    """(num_blocks, block_size, num_kv_heads, head_dim, block_stride) of a
+    [NB, bs, Hkv, D] cache view whose last three dims are contiguous."""
+    if cache.dim() != 4:
+        raise ValueError("cache must be [num_blocks, block_size, num_kv_heads, head_dim]")
+    nb, bs, hkv, d = cache.shape
+    st = cache.stride()
+    if st[3] != 1 or st[2] != d or st[1] != hkv * d:
+        raise ValueError("a cache block must be contiguous")
+    stride0 = st[0] if nb > 1 else bs * hkv * d
+    return nb, bs, hkv, d, stride0
+
+
+def _dtype(t):
+    try:
+        return _DTYPE[t.dtype]
+    except KeyError:
+        raise PkvError(PKV_ERR_UNSUPPORTED, "unsupported dtype %s" % t.dtype) from None
+
+
+def _on_device(name, *tensors):
+    """Kernel arguments must live on one CUDA device (a host pointer handed
+    to a kernel would fault)."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s: every tensor argument must be a CUDA tensor" % name)
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("%s: tensors on different devices" % name)
+    return dev
+
+
+def _need(t, dtype, name, device=None):
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+# ---------------------------------------------------------------------------
+# kernels
+# ---------------------------------------------------------------------------
+def pkv_write_slots(key, value, key_cache, value_cache, slot_mapping, dev_error=None,
+                    stream=None):
+    """Write token rows key/value [T, Hkv, D] into their slots (int64 [T])."""
+    _on_device("pkv_write_slots", key, value, key_cache, value_cache, slot_mapping, dev_error)
+    nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
+        raise ValueError("key_cache and value_cache differ in geometry")
+    _need(slot_mapping, torch.int64, "slot_mapping")
+    _need(key, key_cache.dtype, "key")
+    _need(value, key_cache.dtype, "value")
+    T = slot_mapping.numel()
+    if key.shape != (T, hkv, d) or value.shape != (T, hkv, d):
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim]")
+    st = lib().pkv_write_slots(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
+                               _ptr(slot_mapping), T, nb, bs, hkv, d, bstride,
+                               _dtype(key_cache), _ptr(dev_error),
+                               _stream(stream, key_cache.device))
+    _check(st, "pkv_write_slots")
+
+
+def pkv_copy_blocks(key_cache, value_cache, block_pairs, dev_error=None, stream=None):
+    """Copy whole blocks for each (src, dst) row of int32 block_pairs [n, 2]."""
+    _on_device("pkv_copy_blocks", key_cache, value_cache, block_pairs, dev_error)
+    nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
+        raise ValueError("key_cache and value_cache differ in geometry")
+    _need(block_pairs, torch.int32, "block_pairs")
+    n = block_pairs.numel() // 2
+    st = lib().pkv_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(block_pairs), n, nb,
+                               bs, hkv, d, bstride, _dtype(key_cache), _ptr(dev_error),
+                               _stream(stream, key_cache.device))
+    _check(st, "pkv_copy_blocks")
+
+
+def pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len, partition_size,
+                               head_dim):
+    return int(lib().pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len,
+                                                partition_size, head_dim))
+
+
+def pkv_decode_attention(out, query, key_cache, value_cache, block_tables, context_lens,
+                         max_context_len, scale, partition_size=0, workspace=None,
+                         dev_error=None, stream=None):
+    """Paged decode attention: out/query [S, Hq, D]; block_tables int32
+    [S, MB]; context_lens int32 [S]; workspace a uint8 device tensor of at
+    least pkv_decode_workspace_bytes(...) bytes when partitions are used."""
+    _on_device("pkv_decode_attention", out, query, key_cache, value_cache, block_tables,
+               context_lens, workspace, dev_error)
+    nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
+        raise ValueError("key_cache and value_cache differ in geometry")
+    S, hq, dq = query.shape
+    if dq != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs, num_q_heads, head_dim]")
+    _need(query, key_cache.dtype, "query")
+    _need(out, key_cache.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and context_lens [num_seqs]")
+    if dev_error is not None:
+        _need(dev_error, torch.int32, "dev_error")
+    mb = block_tables.shape[1]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().pkv_decode_attention(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), mb,
+        _ptr(context_lens), S, int(max_context_len), hq, hkv, d, nb, bs, bstride,
+        float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
+        _ptr(dev_error), _stream(stream, query.device))
+    _check(st, "pkv_decode_attention")
+
+
+def pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):
+    v = int(lib().pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes))
+    if v < 0:
+        _check(v, "pkv_block_bytes")
+    return v
+
+
+# ---------------------------------------------------------------------------
+# host block pool
+# ---------------------------------------------------------------------------
+class BlockPool:
+    """The library's host block pool (pkv_pool_* / pkv_seq_*)."""
+
+    def __init__(self, num_blocks, block_size, free_order=None):
+        handle = C.c_void_p()
+        order = None
+        if free_order is not None:
+            order = torch.as_tensor(free_order, dtype=torch.int32).contiguous()
+            if order.numel() != num_blocks:
+                raise ValueError("free_order must have num_blocks entries")
+        st = lib().pkv_pool_create(num_blocks, block_size, _ptr(order) if order is not None
+                                   else C.c_void_p(0), C.byref(handle))
+        _check(st, "pkv_pool_create")
+        self._h = handle
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().pkv_pool_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add(self, seq_id, num_tokens):
+        _check(lib().pkv_seq_add(self._h, seq_id, num_tokens), "pkv_seq_add")
+
+    def fork(self, parent, child):
+        _check(lib().pkv_seq_fork(self._h, parent, child), "pkv_seq_fork")
+
+    def append(self, seq_id):
+        """Returns (slot, cow_src, cow_dst)."""
+        slot = C.c_int64()
+        src = C.c_int32()
+        dst = C.c_int32()
+        _check(lib().pkv_seq_append(self._h, seq_id, C.byref(slot), C.byref(src),
+                                    C.byref(dst)), "pkv_seq_append")
+        return slot.value, src.value, dst.value
+
+    def append_batch(self, seq_ids, slots_out=None, pairs_out=None):
+        """Append one token to each sequence in order.  Returns (slots int64
+        [n], cow_pairs int32 [n_cow, 2]) as CPU tensors (views of the given
+        output buffers, which may be pinned)."""
+        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+        n = ids.numel()
+        slots = slots_out if slots_out is not None else torch.empty(n, dtype=torch.int64)
+        pairs = pairs_out if pairs_out is not None else torch.empty((n, 2), dtype=torch.int32)
+        ncow = C.c_int()
+        done = C.c_int()
+        st = lib().pkv_seq_append_batch(self._h, n, _ptr(ids), _ptr(slots), _ptr(pairs),
+                                        C.byref(ncow), C.byref(done))
+        _check(st, "pkv_seq_append_batch")
+        return slots[:n], pairs[:ncow.value]
+
+    def free(self, seq_id):
+        _check(lib().pkv_seq_free(self._h, seq_id), "pkv_seq_free")
+
+    def num_tokens(self, seq_id):
+        n = C.c_int()
+        _check(lib().pkv_seq_num_tokens(self._h, seq_id, C.byref(n)), "pkv_seq_num_tokens")
+        return n.value
+
+    def slot_mapping(self, seq_id, first_token, num_tokens, out=None):
+        """int64 [num_tokens] slots of the sequence's tokens from first_token."""
+        slots = out if out is not None else torch.empty(num_tokens, dtype=torch.int64)
+        _check(lib().pkv_seq_slot_mapping(self._h, seq_id, first_token, num_tokens,
+                                          _ptr(slots)), "pkv_seq_slot_mapping")
+        return slots[:num_tokens]
+
+    def block_table(self, seq_id):
+        n = C.c_int()
+        cap = self.num_blocks
+        buf = (C.c_int32 * max(cap, 1))()
+        _check(lib().pkv_seq_block_table(self._h, seq_id, buf, cap, C.byref(n)),
+               "pkv_seq_block_table")
+        return list(buf[:n.value])
+
+    def block_tables(self, seq_ids, max_blocks_per_seq, fill=-1, out=None, lens_out=None):
+        """Dense int32 [n, max_blocks_per_seq] tables and int32 [n] lengths."""
+        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+        n = ids.numel()
+        tables = out if out is not None else torch.empty((n, max_blocks_per_seq),
+                                                         dtype=torch.int32)
+        lens = lens_out if lens_out is not None else torch.empty(n, dtype=torch.int32)
+        st = lib().pkv_pool_block_tables(self._h, n, _ptr(ids), _ptr(tables),
+                                         max_blocks_per_seq, fill, _ptr(lens))
+        _check(st, "pkv_pool_block_tables")
+        return tables, lens
+
+    def num_free(self):
+        v = lib().pkv_pool_num_free(self._h)
+        if v < 0:
+            _check(v, "pkv_pool_num_free")
+        return v
+
+    def free_list(self):
+        n = C.c_int()
+        buf = (C.c_int32 * max(self.num_blocks, 1))()
+        _check(lib().pkv_pool_free_list(self._h, buf, self.num_blocks, C.byref(n)),
+               "pkv_pool_free_list")
+        return list(buf[:n.value])
+
+    def refcount(self, block):
+        v = lib().pkv_block_refcount(self._h, block)
+        if v < 0:
+            _check(v, "pkv_block_refcount")
+        return v
+
+    def refcounts(self):
+        return [self.refcount(b) for b in range(self.num_blocks)]

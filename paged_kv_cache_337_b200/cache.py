@@ -1,0 +1,154 @@
+"""Decode-step driver over the C ABI: one paged KV cache (one layer) with its
+block pool, and the per-step sequence of calls the pages describe.
+
+A decode step for a batch of sequences ("Paged KV" wiki page, 实现原理 /
+运行阶段; "PagedAttention 动态内存分页" page, 写时复制与内存共享):
+
+1. the host pool reserves each sequence's next slot, taking a new block when
+   the current one is full and copying a shared current block first
+   (``pkv_seq_append_batch``);
+2. the copy-on-write pairs are applied on the GPU (``pkv_copy_blocks``);
+3. the new tokens' K/V are written into their slots (``pkv_write_slots``);
+4. decode attention runs over every sequence's blocks through its Block
+   Table (``pkv_decode_attention``; split-K with a merge for long contexts).
+
+Steps 2-4 are launched on one stream; the metadata of step 1 travels to the
+device through pinned host staging buffers.  All arithmetic is in the
+library; this module only moves arguments.
+"""
+import torch
+
+from . import _abi
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks, block_size, num_q_heads, num_kv_heads, head_dim, dtype,
+                 device, max_blocks_per_seq, partition_size=0, free_order=None,
+                 key_cache=None, value_cache=None, scale=None):
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        self.num_q_heads = num_q_heads
+        self.num_kv_heads = num_kv_heads
+        self.head_dim = head_dim
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.max_blocks_per_seq = max_blocks_per_seq
+        self.partition_size = partition_size
+        self.scale = scale if scale is not None else 1.0 / (head_dim ** 0.5)
+        shape = (num_blocks, block_size, num_kv_heads, head_dim)
+        self.key_cache = key_cache if key_cache is not None else torch.empty(
+            shape, dtype=dtype, device=self.device)
+        self.value_cache = value_cache if value_cache is not None else torch.empty(
+            shape, dtype=dtype, device=self.device)
+        self.pool = _abi.BlockPool(num_blocks, block_size, free_order)
+        self.dev_error = torch.zeros(2, dtype=torch.int32, device=self.device)
+        self._workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self._staging = {}
+
+    # -- sequence management (host) ---------------------------------------
+    def add_sequence(self, seq_id, num_tokens, key=None, value=None, stream=None):
+        """Prefill allocation of num_tokens tokens; with key/value
+        ([num_tokens, Hkv, D] device tensors) their rows are written into the
+        blocks taken, in order."""
+        self.pool.add(seq_id, num_tokens)
+        if key is not None and num_tokens > 0:
+            slots = self.pool.slot_mapping(seq_id, 0, num_tokens).to(self.device)
+            _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, slots,
+                                 dev_error=self.dev_error, stream=stream)
+
+    def fork(self, parent, child):
+        self.pool.fork(parent, child)
+
+    def free(self, seq_id):
+        self.pool.free(seq_id)
+
+    # -- one decode step --------------------------------------------------
+    def _stage(self, n):
+        """Pinned host staging and device buffers for a batch of n sequences."""
+        st = self._staging.get(n)
+        if st is None:
+            pin = torch.cuda.is_available()
+            mb = self.max_blocks_per_seq
+            st = dict(
+                ids=torch.empty(n, dtype=torch.int64),
+                h_slots=torch.empty(n, dtype=torch.int64, pin_memory=pin),
+                h_pairs=torch.empty((n, 2), dtype=torch.int32, pin_memory=pin),
+                h_tables=torch.empty((n, mb), dtype=torch.int32, pin_memory=pin),
+                h_lens=torch.empty(n, dtype=torch.int32, pin_memory=pin),
+                d_slots=torch.empty(n, dtype=torch.int64, device=self.device),
+                d_pairs=torch.empty((n, 2), dtype=torch.int32, device=self.device),
+                d_tables=torch.empty((n, mb), dtype=torch.int32, device=self.device),
+                d_lens=torch.empty(n, dtype=torch.int32, device=self.device),
+            )
+            self._staging[n] = st
+        return st
+
+    def prepare_step(self, seq_ids):
+        """Host part of a decode step: reserve one slot per sequence and
+        gather tables and lengths into pinned buffers.  Returns a dict of
+        host tensors and the step's maximum context length."""
+        st = self._stage(len(seq_ids))
+        if st.get("uploaded") is not None:
+            st["uploaded"].synchronize()  # the previous copies out of these buffers are done
+        st["ids"].copy_(torch.as_tensor(seq_ids, dtype=torch.int64))
+        slots, pairs = self.pool.append_batch(st["ids"], st["h_slots"], st["h_pairs"])
+        tables, lens = self.pool.block_tables(st["ids"], self.max_blocks_per_seq, -1,
+                                              st["h_tables"], st["h_lens"])
+        return dict(st=st, num_pairs=pairs.shape[0], max_len=int(lens.max()) if len(lens) else 0)
+
+    def upload_step(self, prep, stream=None):
+        """Host-to-device copies of a prepared step's metadata."""
+        st = prep["st"]
+        n = prep["num_pairs"]
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            st["d_slots"].copy_(st["h_slots"], non_blocking=True)
+            if n:
+                st["d_pairs"][:n].copy_(st["h_pairs"][:n], non_blocking=True)
+            st["d_tables"].copy_(st["h_tables"], non_blocking=True)
+            st["d_lens"].copy_(st["h_lens"], non_blocking=True)
+            if st.get("uploaded") is None:
+                st["uploaded"] = torch.cuda.Event()
+            st["uploaded"].record(s)
+
+    def workspace(self, num_seqs, max_len):
+        need = _abi.pkv_decode_workspace_bytes(num_seqs, self.num_q_heads, max_len,
+                                               self.partition_size, self.head_dim)
+        if self._workspace.numel() < need:
+            self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._workspace if need else None
+
+    def launch_step(self, prep, query, key, value, out, max_len=None, stream=None):
+        """Device part of a decode step (copy, write, attention) with the
+        prepared metadata already uploaded."""
+        st = prep["st"]
+        n = prep["num_pairs"]
+        max_len = prep["max_len"] if max_len is None else max_len
+        if n:
+            _abi.pkv_copy_blocks(self.key_cache, self.value_cache, st["d_pairs"][:n],
+                                 dev_error=self.dev_error, stream=stream)
+        _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, st["d_slots"],
+                             dev_error=self.dev_error, stream=stream)
+        _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache,
+                                  st["d_tables"], st["d_lens"], max_len,
+                                  self.scale, self.partition_size,
+                                  self.workspace(len(st["ids"]), max_len),
+                                  dev_error=self.dev_error, stream=stream)
+        return out
+
+    def decode_step(self, seq_ids, query, key, value, out=None, stream=None):
+        """One full decode step for seq_ids (query [S, Hq, D], key/value
+        [S, Hkv, D] on the device).  Returns out [S, Hq, D]."""
+        prep = self.prepare_step(seq_ids)
+        self.upload_step(prep, stream)
+        if out is None:
+            out = torch.empty_like(query)
+        return self.launch_step(prep, query, key, value, out, stream=stream)
+
+    def check_errors(self):
+        """Raises if a kernel recorded bad metadata since the last check."""
+        err = self.dev_error.tolist()
+        if err[0] != _abi.PKV_DEVERR_NONE:
+            self.dev_error.zero_()
+            raise _abi.PkvError(_abi.PKV_ERR_INVALID,
+                                "device error code %d at index %d" % (err[0], err[1]))

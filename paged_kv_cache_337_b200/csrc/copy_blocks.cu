@@ -1,0 +1,84 @@
+// copy_blocks.cu — copy-on-write block copy ("PagedAttention 动态内存分页"
+// page, 写时复制与内存共享: a block shared by several sequences is copied when
+// one of them needs to write into it).
+//
+// A block of one cache is bs * Hkv * D contiguous elements, so each (src,
+// dst) pair is two contiguous copies (K and V).  Each CTA moves one chunk of
+// one pair with 16-byte vectors and several loads in flight per thread; the
+// grid covers pairs x chunks.  Bound: HBM (read + write of whole blocks).
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kVecsPerThread = 4;
+constexpr int kChunkVecs = kThreads * kVecsPerThread;  // 16 KiB per CTA
+
+__global__ void __launch_bounds__(kThreads)
+copy_blocks_kernel(uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
+                   const int32_t* __restrict__ block_pairs, int num_pairs, int num_blocks,
+                   int64_t block_vecs, int64_t block_stride_vecs, int chunks_per_cache,
+                   int32_t* __restrict__ dev_error) {
+    const int64_t item = blockIdx.x;
+    const int per_pair = 2 * chunks_per_cache;
+    const int pair = (int)(item / per_pair);
+    const int r = (int)(item - (int64_t)pair * per_pair);
+    const bool is_v = r >= chunks_per_cache;
+    const int chunk = is_v ? r - chunks_per_cache : r;
+    const int32_t src = __ldg(block_pairs + 2 * pair);
+    const int32_t dst = __ldg(block_pairs + 2 * pair + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (r == 0 && threadIdx.x == 0) report_error(dev_error, PKV_DEVERR_PAIR, pair);
+        return;
+    }
+    uint4* cache = is_v ? value_cache : key_cache;
+    const uint4* s = cache + (int64_t)src * block_stride_vecs;
+    uint4* d = cache + (int64_t)dst * block_stride_vecs;
+    const int64_t base = (int64_t)chunk * kChunkVecs + threadIdx.x;
+    uint4 buf[kVecsPerThread];
+#pragma unroll
+    for (int j = 0; j < kVecsPerThread; ++j) {
+        const int64_t v = base + (int64_t)j * kThreads;
+        if (v < block_vecs) buf[j] = __ldg(s + v);
+    }
+#pragma unroll
+    for (int j = 0; j < kVecsPerThread; ++j) {
+        const int64_t v = base + (int64_t)j * kThreads;
+        if (v < block_vecs) d[v] = buf[j];
+    }
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int pkv_copy_blocks(void* key_cache, void* value_cache, const int32_t* block_pairs,
+                               int num_pairs, int num_blocks, int block_size, int num_kv_heads,
+                               int head_dim, int64_t block_stride, pkv_dtype dtype,
+                               int32_t* dev_error, cudaStream_t stream) {
+    using namespace pkv;
+    PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
+                "pkv_copy_blocks: dtype %d", (int)dtype);
+    PKV_REQUIRE(num_pairs >= 0 && num_blocks >= 0 && block_size > 0 && num_kv_heads > 0 &&
+                    head_dim > 0,
+                PKV_ERR_INVALID, "pkv_copy_blocks: bad sizes");
+    const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    PKV_REQUIRE(block_elems % 8 == 0, PKV_ERR_INVALID,
+                "pkv_copy_blocks: block_size * num_kv_heads * head_dim must be a multiple of 8");
+    PKV_REQUIRE(block_stride >= block_elems && block_stride % 8 == 0, PKV_ERR_INVALID,
+                "pkv_copy_blocks: block_stride %lld", (long long)block_stride);
+    if (num_pairs == 0) return PKV_OK;
+    PKV_REQUIRE(key_cache && value_cache && block_pairs, PKV_ERR_INVALID,
+                "pkv_copy_blocks: NULL pointer");
+    PKV_REQUIRE(aligned16(key_cache) && aligned16(value_cache), PKV_ERR_INVALID,
+                "pkv_copy_blocks: caches must be 16-byte aligned");
+    DeviceGuard guard(stream, key_cache);
+    const int64_t block_vecs = block_elems / 8;
+    const int64_t chunks = (block_vecs + kChunkVecs - 1) / kChunkVecs;
+    const int64_t grid = (int64_t)num_pairs * 2 * chunks;
+    PKV_REQUIRE(grid < (1ll << 31), PKV_ERR_INVALID, "pkv_copy_blocks: too many pairs");
+    copy_blocks_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(
+        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), block_pairs,
+        num_pairs, num_blocks, block_vecs, block_stride / 8, (int)chunks, dev_error);
+    return launch_status("pkv_copy_blocks");
+}

@@ -1,0 +1,801 @@
+// decode_attention.cu — single-token decode attention over the paged KV cache
+// ("Paged KV" wiki page, Attention Kernel 的适配: the kernel takes the Block
+// Table and block_size and reads K/V block by block through the table; the
+// result is ordinary softmax attention over the sequence's tokens in logical
+// order, since PagedAttention changes the storage, not the algorithm —
+// "一文读懂vLLM的…PagedAttention" page, opening section).
+//
+// Work decomposition
+//   One CTA per (sequence, KV head, partition).  A partition is a run of
+//   partition_size tokens (the whole context in single-pass mode).  The G
+//   query heads that share the KV head are packed into the CTA, so each K/V
+//   byte is read from HBM once per step.  Each of the CTA's warps owns every
+//   NW-th 16-token tile of the partition and runs its own TMA pipeline:
+//   lane 0 resolves the tile's physical block from the partition's slice of
+//   the Block Table (staged in shared memory once per CTA) and issues 4-D
+//   tiled TMA loads of the K and V tiles into a STAGES-deep ring of
+//   128B-swizzled shared-memory buffers, completing on per-stage mbarriers.
+//   Softmax is online (running max and sum in fp32, base-2 exponentials with
+//   scale * log2(e) folded into the scores).  The warps' partial results are
+//   merged through shared memory at the end; with several partitions the CTA
+//   writes fp32 (max, sum, unnormalised output) to the workspace and a merge
+//   kernel combines them.
+//
+// Arithmetic paths
+//   G == 1 (no grouping): a GEMV; FFMA with warp shuffles.  Lane l owns
+//   head_dim / 32 dimensions; the 16 partial dot products of a tile are
+//   reduce-scattered across the warp (16 shuffles) so lane l ends with token
+//   l / 2's score.
+//   G >= 2: the G query heads form a real dense contraction.  S^T = K Q^T is
+//   an m16n8k16 tensor-core product with the 16 tokens as M and up to 8
+//   heads as N (K tiles through ldmatrix, Q^T fragments in registers);
+//   O^T += V^T P^T takes V^T tiles through ldmatrix.trans and P^T from the
+//   score fragments by movmatrix, with head_dim as M.
+//
+// Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
+// PKV_DEVERR_TIMEOUT, waits (bounded) for its loads in flight and skips its
+// output.  Table entries outside [0, num_blocks) are reported; the TMA unit
+// fills such a tile with zeros, so no access leaves the cache.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kTile = 16;                          // tokens per tile
+constexpr int kBoxD = 64;                          // head_dim per TMA box (128 B)
+constexpr int kSubTileBytes = kTile * kBoxD * 2;   // one swizzled box: 2 KiB
+constexpr int kWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct Geom {
+    static constexpr int kBoxes = D / kBoxD;             // boxes per K (or V) tile
+    static constexpr int kKBytes = kBoxes * kSubTileBytes;
+    static constexpr int kStageBytes = 2 * kKBytes;      // K + V of one tile
+    static constexpr int kStages = D == 128 ? 3 : 4;
+};
+
+struct DecodeParams {
+    void* out;
+    const void* query;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float* ws_m;
+    float* ws_l;
+    float* ws_o;
+    int32_t* dev_error;
+    int num_seqs;
+    int max_blocks_per_seq;
+    int max_context_len;
+    int num_q_heads;
+    int group;  // query heads per KV head
+    int num_blocks;
+    int block_size;
+    int partition_size;  // tokens per partition
+    int num_partitions;  // grid.z and the workspace's partition extent
+    float scale_log2;    // scale * log2(e)
+};
+
+// Byte offset of 16-byte chunk `chunk` (0 .. D/8-1) of row `r` inside a tile
+// written by TMA with 128-byte swizzling: each 64-element box is 16 rows of
+// 128 bytes whose chunks are XOR-permuted by the row index.
+__device__ __forceinline__ uint32_t swz(int r, int chunk) {
+    return (chunk >> 3) * kSubTileBytes + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    const uint32_t a = smem_addr(p);
+    return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// Context length of sequence s as the kernels use it: a value outside
+// [0, max_context_len] or beyond the table row is treated as 0 (reported by
+// the attention kernel).
+__device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool* bad) {
+    int L = __ldg(p.context_lens + s);
+    *bad = L < 0 || L > p.max_context_len ||
+           (int64_t)L > (int64_t)p.max_blocks_per_seq * p.block_size;
+    return *bad ? 0 : L;
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp arithmetic, G == 1: FFMA + shuffles
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+struct GemvWarp {
+    static constexpr int DV = D / 32;  // dims per lane
+    static constexpr int GP = 1;       // heads held (padded)
+    float q[DV], o[DV], m, l;
+
+    __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
+        const T* qrow = static_cast<const T*>(p.query) + ((int64_t)s * p.num_q_heads + kvh) * D;
+        load(reinterpret_cast<const uint8_t*>(qrow + lane * DV), q);
+#pragma unroll
+        for (int j = 0; j < DV; ++j) o[j] = 0.f;
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    __device__ __forceinline__ static void load(const uint8_t* src, float (&v)[DV]) {
+        if constexpr (DV == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(src);
+            const float2 a = Storage<T>::to_float2(w.x), b = Storage<T>::to_float2(w.y);
+            v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+        } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+            const float2 a = Storage<T>::to_float2(w);
+            v[0] = a.x; v[1] = a.y;
+        }
+    }
+
+    // lane's DV elements of row r of a swizzled tile
+    __device__ __forceinline__ static const uint8_t* at(const uint8_t* tile, int r, int lane) {
+        const int d0 = lane * DV;
+        return tile + swz(r, d0 >> 3) + (d0 & 7) * 2;
+    }
+
+    __device__ __forceinline__ void tile(const uint8_t* kt, const uint8_t* vt, int valid,
+                                         float scale_log2, int lane) {
+        float part[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float k[DV];
+            load(at(kt, r, lane), k);
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
+            part[r] = acc;
+        }
+        // reduce-scatter the 16 partial sums over the 32 lanes: after the
+        // rounds with masks 16, 8, 4, 2 and a final pairwise add, lane l
+        // holds the full dot product of token l / 2
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool up = lane & 16;
+            const float send = up ? part[i] : part[i + 8];
+            const float keep = up ? part[i + 8] : part[i];
+            part[i] = keep + __shfl_xor_sync(kFull, send, 16);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool up = lane & 8;
+            const float send = up ? part[i] : part[i + 4];
+            const float keep = up ? part[i + 4] : part[i];
+            part[i] = keep + __shfl_xor_sync(kFull, send, 8);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const bool up = lane & 4;
+            const float send = up ? part[i] : part[i + 2];
+            const float keep = up ? part[i + 2] : part[i];
+            part[i] = keep + __shfl_xor_sync(kFull, send, 4);
+        }
+        {
+            const bool up = lane & 2;
+            const float send = up ? part[0] : part[1];
+            const float keep = up ? part[1] : part[0];
+            part[0] = keep + __shfl_xor_sync(kFull, send, 2);
+        }
+        const float dot = part[0] + __shfl_xor_sync(kFull, part[0], 1);
+        const int r = lane >> 1;
+        const float sc = r < valid ? dot * scale_log2 : -INFINITY;
+        float mx = sc;
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+        const float m_new = fmaxf(m, mx);
+        const float alpha = exp2f(m - m_new);
+        const float pr = exp2f(sc - m_new);
+        l = l * alpha + ((lane & 1) ? 0.f : pr);  // each token is held by 2 lanes
+        m = m_new;
+#pragma unroll
+        for (int j = 0; j < DV; ++j) o[j] *= alpha;
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            const float pb = __shfl_sync(kFull, pr, rr * 2);
+            float v[DV];
+            load(at(vt, rr, lane), v);
+#pragma unroll
+            for (int j = 0; j < DV; ++j) o[j] = fmaf(pb, v[j], o[j]);
+        }
+    }
+
+    // warp-level totals: m is already uniform; l is summed over the lanes
+    __device__ __forceinline__ void finish() {
+#pragma unroll
+        for (int x = 1; x < 32; x <<= 1) l += __shfl_xor_sync(kFull, l, x);
+    }
+
+    __device__ __forceinline__ void store_ml(float* sm_m, float* sm_l, int warp, int lane,
+                                             int G) {
+        if (lane == 0) {
+            sm_m[warp * GP] = m;
+            sm_l[warp * GP] = l;
+        }
+    }
+
+    // scaled output into sm_o[warp][head][d]
+    __device__ __forceinline__ void store_o(float* sm_o, const float* M, int warp, int lane,
+                                            int G) {
+        const float f = M[0] == -INFINITY ? 0.f : exp2f(m - M[0]);
+#pragma unroll
+        for (int j = 0; j < DV; ++j) sm_o[warp * D + lane * DV + j] = o[j] * f;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Per-warp arithmetic, G >= 2: mma.sync m16n8k16 on the head group
+// ---------------------------------------------------------------------------
+template <typename T, int D, int NT>
+struct MmaWarp {
+    static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
+    static constexpr int GP = NT * 8;  // heads held (padded)
+    uint32_t qf[KS][NT][2];            // Q^T B-fragments
+    float acc[KS][NT][4];              // O^T[d][head]
+    float m[NT][2], l[NT][2];          // per lane: heads nt*8 + (lane&3)*2 + {0,1}
+
+    __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
+        const int G = p.group;
+        const T* qbase = static_cast<const T*>(p.query) +
+                         ((int64_t)s * p.num_q_heads + (int64_t)kvh * G) * D;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = nt * 8 + (lane >> 2);
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                if (h < G) {
+                    const T* qrow = qbase + (int64_t)h * D + kk * 16 + (lane & 3) * 2;
+                    qf[kk][nt][0] = *reinterpret_cast<const uint32_t*>(qrow);
+                    qf[kk][nt][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+                } else {
+                    qf[kk][nt][0] = 0u;
+                    qf[kk][nt][1] = 0u;
+                }
+            }
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
+        }
+    }
+
+    __device__ __forceinline__ void tile(const uint8_t* kt, const uint8_t* vt, int valid,
+                                         float scale_log2, int lane) {
+        const uint32_t kbase = smem_addr(kt), vbase = smem_addr(vt);
+        const int j = lane >> 3;
+        // S^T[token][head] = K Q^T over head_dim
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            uint32_t a[4];
+            const int row = (lane & 7) + (j & 1) * 8;
+            ldmatrix_x4(a, kbase + swz(row, kk * 2 + (j >> 1)));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                Mma<T>::m16n8k16(sacc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+        }
+        // online softmax per head; the lane holds tokens r0, r0 + 8
+        const int r0 = lane >> 2;
+        const bool v0 = r0 < valid, v1 = r0 + 8 < valid;
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float s0 = v0 ? sacc[nt][0] * scale_log2 : -INFINITY;
+            const float s1 = v0 ? sacc[nt][1] * scale_log2 : -INFINITY;
+            const float s2 = v1 ? sacc[nt][2] * scale_log2 : -INFINITY;
+            const float s3 = v1 ? sacc[nt][3] * scale_log2 : -INFINITY;
+            float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, x));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, x));
+            }
+            const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+            const float a0 = exp2f(m[nt][0] - mn0), a1 = exp2f(m[nt][1] - mn1);
+            const float p0 = exp2f(s0 - mn0), p1 = exp2f(s1 - mn1);
+            const float p2 = exp2f(s2 - mn0), p3 = exp2f(s3 - mn1);
+            l[nt][0] = l[nt][0] * a0 + (p0 + p2);
+            l[nt][1] = l[nt][1] * a1 + (p1 + p3);
+            m[nt][0] = mn0;
+            m[nt][1] = mn1;
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                acc[mt][nt][0] *= a0;
+                acc[mt][nt][1] *= a1;
+                acc[mt][nt][2] *= a0;
+                acc[mt][nt][3] *= a1;
+            }
+            // P[token][head] as 16-bit fragments, transposed to P^T B-fragments
+            pb[nt][0] = movmatrix_trans(Storage<T>::from_float2(p0, p1));
+            pb[nt][1] = movmatrix_trans(Storage<T>::from_float2(p2, p3));
+        }
+        // O^T[d][head] += V^T P^T over the 16 tokens
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            uint32_t a[4];
+            const int row = (lane & 7) + (j >> 1) * 8;
+            ldmatrix_x4_trans(a, vbase + swz(row, mt * 2 + (j & 1)));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Mma<T>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
+        }
+    }
+
+    __device__ __forceinline__ void finish() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                l[nt][0] += __shfl_xor_sync(kFull, l[nt][0], x);
+                l[nt][1] += __shfl_xor_sync(kFull, l[nt][1], x);
+            }
+    }
+
+    __device__ __forceinline__ void store_ml(float* sm_m, float* sm_l, int warp, int lane,
+                                             int G) {
+        if (lane < 4) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int h = nt * 8 + lane * 2 + i;
+                    sm_m[warp * GP + h] = m[nt][i];
+                    sm_l[warp * GP + h] = l[nt][i];
+                }
+        }
+    }
+
+    __device__ __forceinline__ void store_o(float* sm_o, const float* M, int warp, int lane,
+                                            int G) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int h = nt * 8 + (lane & 3) * 2 + (i & 1);
+                if (h >= G) continue;
+                const float f = M[h] == -INFINITY ? 0.f : exp2f(m[nt][i & 1] - M[h]);
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    const int d = mt * 16 + (lane >> 2) + (i >> 1) * 8;
+                    sm_o[(warp * G + h) * D + d] = acc[mt][nt][i] * f;
+                }
+            }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// The attention kernel (single pass or one partition of split-K)
+// ---------------------------------------------------------------------------
+template <typename T, int D, typename Warp>
+__global__ void __launch_bounds__(kWarps * 32)
+paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+    using Gm = Geom<D>;
+    constexpr int STAGES = Gm::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* stages = smem;  // [warp][stage][K tile | V tile]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * STAGES * Gm::kStageBytes);
+    int32_t* table = reinterpret_cast<int32_t*>(bars + kWarps * STAGES);
+
+    const int s = blockIdx.x, kvh = blockIdx.y, part = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.group, bs = p.block_size, P = p.partition_size;
+
+    bool bad_len;
+    const int L = checked_len(p, s, &bad_len);
+    if (bad_len && part == 0 && kvh == 0 && threadIdx.x == 0)
+        report_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN, s);
+    const int np = L > 0 ? (L + P - 1) / P : 1;
+    if (part >= np) return;
+    const int t_begin = part * P;
+    const int t_end = min(L, t_begin + P);
+    const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+    const int lb0 = t_begin / bs;
+    const int nlb = t_end > t_begin ? (t_end - 1) / bs - lb0 + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+    // this partition's slice of the Block Table, one load per logical block
+    const int32_t* trow = p.block_tables + (int64_t)s * p.max_blocks_per_seq + lb0;
+    for (int i = threadIdx.x; i < nlb; i += kWarps * 32) {
+        const int32_t b = __ldg(trow + i);
+        if (b < 0 || b >= p.num_blocks) report_error(p.dev_error, PKV_DEVERR_BLOCK_ID, s);
+        table[i] = b;
+    }
+    uint64_t* my_bars = bars + warp * STAGES;
+    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // TMA of tile `tile` (K and V, all boxes) into stage `st`; lane 0 only
+    auto issue = [&](int st, int tile) {
+        const int t0 = t_begin + tile * kTile;
+        const int phys = table[t0 / bs - lb0];
+        const int off = t0 % bs;
+        uint8_t* kdst = my_stages + st * Gm::kStageBytes;
+        uint8_t* vdst = kdst + Gm::kKBytes;
+        mbar_arrive_expect_tx(&my_bars[st], Gm::kStageBytes);
+#pragma unroll
+        for (int b = 0; b < Gm::kBoxes; ++b)
+            tma_load_4d(kdst + b * kSubTileBytes, &kmap, &my_bars[st], b * kBoxD, kvh, off, phys);
+#pragma unroll
+        for (int b = 0; b < Gm::kBoxes; ++b)
+            tma_load_4d(vdst + b * kSubTileBytes, &vmap, &my_bars[st], b * kBoxD, kvh, off, phys);
+    };
+
+    const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < STAGES; ++st)
+            if (st < my_tiles) issue(st, warp + st * kWarps);
+    }
+    __syncwarp();
+
+    Warp w;
+    w.init(p, s, kvh, lane);
+    int it = 0;
+    bool failed = false;
+    for (; it < my_tiles; ++it) {
+        const int st = it % STAGES;
+        const int tile = warp + it * kWarps;
+        if (!mbar_wait_bounded(&my_bars[st], (it / STAGES) & 1)) {
+            failed = true;
+            break;
+        }
+        uint8_t* kt = my_stages + st * Gm::kStageBytes;
+        uint8_t* vt = kt + Gm::kKBytes;
+        const int valid = min(kTile, t_end - (t_begin + tile * kTile));
+        if (valid < kTile) {
+            // rows past the context may hold anything (NaN included): zero
+            // the V rows so that their zero weights contribute exactly 0
+            const int nchunks = (kTile - valid) * Gm::kBoxes * 8;
+            for (int c = lane; c < nchunks; c += 32) {
+                const int r = valid + c / (Gm::kBoxes * 8);
+                const int ch = c % (Gm::kBoxes * 8);
+                *reinterpret_cast<uint4*>(vt + swz(r, ch)) = make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+        }
+        w.tile(kt, vt, valid, p.scale_log2, lane);
+        fence_proxy_async();  // our reads of this stage before TMA rewrites it
+        __syncwarp();
+        const int next = it + STAGES;
+        if (lane == 0 && next < my_tiles) issue(st, warp + next * kWarps);
+    }
+    if (failed) {
+        // drain this warp's loads still in flight before giving up
+        for (int k = it; k < my_tiles && k < it + STAGES; ++k)
+            mbar_wait_bounded(&my_bars[k % STAGES], (k / STAGES) & 1);
+    }
+    if (__syncthreads_or(failed)) {
+        if (threadIdx.x == 0) report_error(p.dev_error, PKV_DEVERR_TIMEOUT, 0);
+        return;
+    }
+
+    // ---- merge the warps' partial softmax states through shared memory ----
+    w.finish();
+    constexpr int GP = Warp::GP;
+    float* sm_m = reinterpret_cast<float*>(stages);  // [warp][GP]
+    float* sm_l = sm_m + kWarps * GP;                // [warp][GP]
+    float* sm_M = sm_l + kWarps * GP;                // [GP]
+    float* sm_o = sm_M + GP;                         // [warp][G][D]
+    w.store_ml(sm_m, sm_l, warp, lane, G);
+    __syncthreads();
+    if (threadIdx.x < G) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) M = fmaxf(M, sm_m[k * GP + threadIdx.x]);
+        sm_M[threadIdx.x] = M;
+    }
+    __syncthreads();
+    w.store_o(sm_o, sm_M, warp, lane, G);
+    __syncthreads();
+
+    const int Hq = p.num_q_heads;
+    for (int idx = threadIdx.x; idx < G * D; idx += kWarps * 32) {
+        const int h = idx / D, d = idx - h * D;
+        const float M = sm_M[h];
+        float Lsum = 0.f, O = 0.f;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) {
+            const float mk = sm_m[k * GP + h];
+            Lsum += M == -INFINITY ? 0.f : sm_l[k * GP + h] * exp2f(mk - M);
+            O += sm_o[(k * G + h) * D + d];
+        }
+        const int64_t qh = (int64_t)s * Hq + (int64_t)kvh * G + h;
+        if (np == 1) {
+            static_cast<T*>(p.out)[qh * D + d] = Storage<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+        } else {
+            const int64_t wi = qh * p.num_partitions + part;
+            p.ws_o[wi * D + d] = O;
+            if (d == 0) {
+                p.ws_m[wi] = M;
+                p.ws_l[wi] = Lsum;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of split-K partials: with M = max_p m_p and w_p = 2^(m_p - M),
+// out = sum_p w_p o_p / sum_p w_p l_p  (m in base-2 units of scaled scores).
+// One warp per (sequence, query head); sequences that fit one partition were
+// finished by the attention kernel.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
+    constexpr int DV = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Hq = p.num_q_heads;
+    const int64_t qh = (int64_t)blockIdx.x * 4 + warp;
+    if (qh >= (int64_t)p.num_seqs * Hq) return;
+    const int s = (int)(qh / Hq);
+    bool bad;
+    const int L = checked_len(p, s, &bad);
+    const int P = p.partition_size;
+    const int np = L > 0 ? (L + P - 1) / P : 1;
+    if (np <= 1) return;
+    const float* m = p.ws_m + qh * p.num_partitions;
+    const float* l = p.ws_l + qh * p.num_partitions;
+    const float* o = p.ws_o + qh * p.num_partitions * D;
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, x));
+    float Lsum = 0.f;
+    for (int i = lane; i < np; i += 32) Lsum += l[i] * exp2f(m[i] - M);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) Lsum += __shfl_xor_sync(kFull, Lsum, x);
+    float acc[DV];
+#pragma unroll
+    for (int j = 0; j < DV; ++j) acc[j] = 0.f;
+    for (int i = 0; i < np; ++i) {
+        const float wgt = exp2f(m[i] - M);
+        const float* oi = o + (int64_t)i * D + lane * DV;
+        if constexpr (DV == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(oi);
+            acc[0] = fmaf(wgt, v.x, acc[0]);
+            acc[1] = fmaf(wgt, v.y, acc[1]);
+            acc[2] = fmaf(wgt, v.z, acc[2]);
+            acc[3] = fmaf(wgt, v.w, acc[3]);
+        } else {
+            const float2 v = *reinterpret_cast<const float2*>(oi);
+            acc[0] = fmaf(wgt, v.x, acc[0]);
+            acc[1] = fmaf(wgt, v.y, acc[1]);
+        }
+    }
+    const float inv = 1.f / Lsum;
+    T* out = static_cast<T*>(p.out) + qh * D + lane * DV;
+#pragma unroll
+    for (int j = 0; j < DV; j += 2) {
+        const uint32_t w = Storage<T>::from_float2(acc[j] * inv, acc[j + 1] * inv);
+        *reinterpret_cast<uint32_t*>(out + j) = w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 4-D view of one cache: (head_dim, kv head, slot in block, physical block),
+// boxes of 64 x 1 x 16 x 1 elements with 128-byte swizzling.
+int encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dtype, int head_dim,
+                     int num_kv_heads, int block_size, int num_blocks, int64_t block_stride) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
+                                (cuuint64_t)block_size, (cuuint64_t)num_blocks};
+    const cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2,
+                                   (cuuint64_t)num_kv_heads * head_dim * 2,
+                                   (cuuint64_t)block_stride * 2};
+    const cuuint32_t box[4] = {kBoxD, 1, kTile, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapDataType ty = dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(map, ty, 4, const_cast<void*>(cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
+}
+
+struct WorkspaceLayout {
+    size_t m_off, l_off, o_off, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t NP, int64_t D) {
+    WorkspaceLayout w;
+    const size_t ml = align256((size_t)(S * Hq * NP) * sizeof(float));
+    w.m_off = 0;
+    w.l_off = ml;
+    w.o_off = 2 * ml;
+    w.total = 2 * ml + align256((size_t)(S * Hq * NP * D) * sizeof(float));
+    return w;
+}
+
+// partition length actually used, and the number of partitions of the grid
+void plan_partitions(int max_context_len, int partition_size, int* P, int* NP) {
+    if (partition_size <= 0 || partition_size >= max_context_len) {
+        int ctx = max_context_len > 0 ? max_context_len : 1;
+        *P = (ctx + kTile - 1) / kTile * kTile;
+        *NP = 1;
+    } else {
+        *P = partition_size;
+        *NP = (max_context_len + partition_size - 1) / partition_size;
+    }
+}
+
+template <typename T, int D, typename Warp>
+int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                  int num_kv_heads, cudaStream_t stream) {
+    using Gm = Geom<D>;
+    const int table_cap = (p.partition_size + p.block_size - 1) / p.block_size + 1;
+    const size_t smem = 1024 + (size_t)kWarps * Gm::kStages * Gm::kStageBytes +
+                        (size_t)kWarps * Gm::kStages * sizeof(uint64_t) +
+                        (size_t)table_cap * sizeof(int32_t);
+    if (smem > 227 * 1024)
+        return fail(PKV_ERR_UNSUPPORTED,
+                    "pkv_decode_attention: %d tokens per partition need %zu bytes of shared "
+                    "memory; use a smaller partition_size",
+                    p.partition_size, smem);
+    auto kern = paged_decode_kernel<T, D, Warp>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return fail(PKV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    dim3 grid(p.num_seqs, num_kv_heads, p.num_partitions);
+    kern<<<grid, kWarps * 32, smem, stream>>>(kmap, vmap, p);
+    int st = launch_status("pkv_decode_attention");
+    if (st != PKV_OK || p.num_partitions == 1) return st;
+    const int64_t pairs = (int64_t)p.num_seqs * p.num_q_heads;
+    paged_decode_merge_kernel<T, D><<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(p);
+    return launch_status("pkv_decode_attention (merge)");
+}
+
+template <typename T, int D>
+int dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
+                   int num_kv_heads, cudaStream_t stream) {
+    if (p.group == 1) return launch_decode<T, D, GemvWarp<T, D>>(kmap, vmap, p, num_kv_heads, stream);
+    if (p.group <= 8)
+        return launch_decode<T, D, MmaWarp<T, D, 1>>(kmap, vmap, p, num_kv_heads, stream);
+    return launch_decode<T, D, MmaWarp<T, D, 2>>(kmap, vmap, p, num_kv_heads, stream);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int max_context_len,
+                                             int partition_size, int head_dim) {
+    using namespace pkv;
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+    int P, NP;
+    plan_partitions(max_context_len, partition_size, &P, &NP);
+    if (NP <= 1) return 0;
+    return workspace_layout(num_seqs, num_q_heads, NP, head_dim).total;
+}
+
+extern "C" int pkv_decode_attention(void* out, const void* query, const void* key_cache,
+                                    const void* value_cache, const int32_t* block_tables,
+                                    int max_blocks_per_seq, const int32_t* context_lens,
+                                    int num_seqs, int max_context_len, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int num_blocks,
+                                    int block_size, int64_t block_stride, float scale,
+                                    int partition_size, void* workspace, size_t workspace_bytes,
+                                    pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    using namespace pkv;
+    PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: dtype %d", (int)dtype);
+    PKV_REQUIRE(head_dim == 64 || head_dim == 128, PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: head_dim %d (built: 64, 128)", head_dim);
+    PKV_REQUIRE(block_size > 0 && block_size % kTile == 0 && block_size <= 256,
+                PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: block_size %d (built: multiples of 16 up to 256)",
+                block_size);
+    PKV_REQUIRE(num_seqs >= 0 && num_q_heads > 0 && num_kv_heads > 0 && num_blocks >= 0 &&
+                    max_blocks_per_seq >= 0 && max_context_len >= 0,
+                PKV_ERR_INVALID, "pkv_decode_attention: bad sizes");
+    PKV_REQUIRE(num_q_heads % num_kv_heads == 0, PKV_ERR_INVALID,
+                "pkv_decode_attention: %d query heads over %d KV heads", num_q_heads,
+                num_kv_heads);
+    const int group = num_q_heads / num_kv_heads;
+    PKV_REQUIRE(group <= 16, PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: group size %d (built: up to 16)", group);
+    PKV_REQUIRE(partition_size >= 0 && partition_size % kTile == 0, PKV_ERR_INVALID,
+                "pkv_decode_attention: partition_size %d is not a multiple of 16",
+                partition_size);
+    PKV_REQUIRE((int64_t)max_context_len <= (int64_t)max_blocks_per_seq * block_size,
+                PKV_ERR_INVALID,
+                "pkv_decode_attention: max_context_len %d exceeds the table (%d x %d)",
+                max_context_len, max_blocks_per_seq, block_size);
+    const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    PKV_REQUIRE(block_stride >= block_elems && block_stride % 8 == 0, PKV_ERR_INVALID,
+                "pkv_decode_attention: block_stride %lld", (long long)block_stride);
+    PKV_REQUIRE(num_kv_heads <= 65535, PKV_ERR_UNSUPPORTED, "too many KV heads");
+    if (num_seqs == 0) return PKV_OK;
+    PKV_REQUIRE(out && query && key_cache && value_cache && context_lens &&
+                    (block_tables || max_blocks_per_seq == 0),
+                PKV_ERR_INVALID, "pkv_decode_attention: NULL pointer");
+    PKV_REQUIRE(aligned16(out) && aligned16(query) && aligned16(key_cache) &&
+                    aligned16(value_cache),
+                PKV_ERR_INVALID, "pkv_decode_attention: pointers must be 16-byte aligned");
+    PKV_REQUIRE(num_blocks > 0, PKV_ERR_INVALID, "pkv_decode_attention: empty pool");
+
+    DecodeParams p{};
+    p.out = out;
+    p.query = query;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.dev_error = dev_error;
+    p.num_seqs = num_seqs;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.num_q_heads = num_q_heads;
+    p.group = group;
+    p.num_blocks = num_blocks;
+    p.block_size = block_size;
+    p.scale_log2 = scale * kLog2e;
+    plan_partitions(max_context_len, partition_size, &p.partition_size, &p.num_partitions);
+    PKV_REQUIRE(p.num_partitions <= 65535, PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: %d partitions (max 65535)", p.num_partitions);
+    if (p.num_partitions > 1) {
+        WorkspaceLayout w = workspace_layout(num_seqs, num_q_heads, p.num_partitions, head_dim);
+        PKV_REQUIRE(workspace != nullptr && workspace_bytes >= w.total && aligned16(workspace),
+                    PKV_ERR_WORKSPACE,
+                    "pkv_decode_attention: needs %zu bytes of 16-byte aligned workspace, got %zu",
+                    w.total, workspace ? workspace_bytes : (size_t)0);
+        uint8_t* base = static_cast<uint8_t*>(workspace);
+        p.ws_m = reinterpret_cast<float*>(base + w.m_off);
+        p.ws_l = reinterpret_cast<float*>(base + w.l_off);
+        p.ws_o = reinterpret_cast<float*>(base + w.o_off);
+    }
+
+    CUtensorMap kmap, vmap;
+    int st = encode_cache_map(&kmap, key_cache, dtype, head_dim, num_kv_heads, block_size,
+                              num_blocks, block_stride);
+    if (st != PKV_OK) return st;
+    st = encode_cache_map(&vmap, value_cache, dtype, head_dim, num_kv_heads, block_size,
+                          num_blocks, block_stride);
+    if (st != PKV_OK) return st;
+
+    DeviceGuard guard(stream, key_cache);
+    if (dtype == PKV_BF16) {
+        return head_dim == 128 ? dispatch_group<__nv_bfloat16, 128>(kmap, vmap, p, num_kv_heads, stream)
+                               : dispatch_group<__nv_bfloat16, 64>(kmap, vmap, p, num_kv_heads, stream);
+    }
+    return head_dim == 128 ? dispatch_group<__half, 128>(kmap, vmap, p, num_kv_heads, stream)
+                           : dispatch_group<__half, 64>(kmap, vmap, p, num_kv_heads, stream);
+}

@@ -1,0 +1,85 @@
+// write_slots.cu — the slot-mapped scatter of new tokens' K/V rows into the
+// paged cache ("Paged KV" wiki page, 实现原理 / 运行阶段: a decoded token is
+// written to the next slot of its sequence's current block; prefill fills
+// the blocks it took, in order).
+//
+// A token's row for all KV heads, [num_kv_heads, head_dim], is contiguous in
+// the source and, inside its block, in the cache, so the kernel is a gather
+// of 16-byte vectors: one thread per vector, K and V in one launch, slots
+// read once per vector from L1.  Bound: HBM (read + write of the rows).
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+write_slots_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                   uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
+                   const int64_t* __restrict__ slot_mapping, int num_tokens,
+                   int64_t num_slots, int block_size, int64_t row_vecs,
+                   int64_t block_stride_vecs, int32_t* __restrict__ dev_error) {
+    // work item i: token i / (2 * row_vecs), K (first half) or V, vector
+    const int64_t per_token = 2 * row_vecs;
+    const int64_t total = (int64_t)num_tokens * per_token;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int64_t r = i - t * per_token;
+        const int64_t slot = __ldg(slot_mapping + t);
+        if (slot < 0) continue;  // padding token
+        if (slot >= num_slots) {
+            if (r == 0) report_error(dev_error, PKV_DEVERR_SLOT, (int)t);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int64_t off = slot - blk * block_size;
+        const bool is_v = r >= row_vecs;
+        const int64_t v = is_v ? r - row_vecs : r;
+        const int64_t dst = blk * block_stride_vecs + off * row_vecs + v;
+        const int64_t src = t * row_vecs + v;
+        if (is_v)
+            value_cache[dst] = __ldg(value + src);
+        else
+            key_cache[dst] = __ldg(key + src);
+    }
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int pkv_write_slots(const void* key, const void* value, void* key_cache,
+                               void* value_cache, const int64_t* slot_mapping,
+                               int num_tokens, int num_blocks, int block_size,
+                               int num_kv_heads, int head_dim, int64_t block_stride,
+                               pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    using namespace pkv;
+    PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
+                "pkv_write_slots: dtype %d", (int)dtype);
+    PKV_REQUIRE(num_tokens >= 0 && num_blocks >= 0 && block_size > 0 && num_kv_heads > 0 &&
+                    head_dim > 0,
+                PKV_ERR_INVALID, "pkv_write_slots: bad sizes");
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    PKV_REQUIRE(row % 8 == 0, PKV_ERR_INVALID,
+                "pkv_write_slots: num_kv_heads * head_dim must be a multiple of 8");
+    PKV_REQUIRE(block_stride >= (int64_t)block_size * row && block_stride % 8 == 0,
+                PKV_ERR_INVALID, "pkv_write_slots: block_stride %lld", (long long)block_stride);
+    if (num_tokens == 0) return PKV_OK;
+    PKV_REQUIRE(key && value && key_cache && value_cache && slot_mapping, PKV_ERR_INVALID,
+                "pkv_write_slots: NULL pointer");
+    PKV_REQUIRE(aligned16(key) && aligned16(value) && aligned16(key_cache) &&
+                    aligned16(value_cache),
+                PKV_ERR_INVALID, "pkv_write_slots: pointers must be 16-byte aligned");
+    DeviceGuard guard(stream, key_cache);
+    const int64_t row_vecs = row / 8;
+    const int64_t total = (int64_t)num_tokens * 2 * row_vecs;
+    int64_t grid = (total + kThreads - 1) / kThreads;
+    if (grid > 148 * 64) grid = 148 * 64;  // grid-stride beyond 64 CTAs per SM
+    write_slots_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), slot_mapping,
+        num_tokens, (int64_t)num_blocks * block_size, block_size, row_vecs, block_stride / 8,
+        dev_error);
+    return launch_status("pkv_write_slots");
+}

@@ -19,26 +19,7 @@ import torch
 
 from oracle import reference as ref
 from tests.conftest import golden_lines
-
-DT = {"f16": torch.float16, "bf16": torch.bfloat16}
-
-
-# ---------------------------------------------------------------------------
-# helpers (test-side layout builders; no attention arithmetic)
-# ---------------------------------------------------------------------------
-def scatter_to_pages(k_seqs, v_seqs, tables, num_blocks, bs):
-    """Place each sequence's contiguous [L, Hkv, D] K/V into a paged cache
-    [NB, bs, Hkv, D] following its block table."""
-    Hkv, D = k_seqs[0].shape[1:]
-    dt = k_seqs[0].dtype
-    kc = torch.zeros((num_blocks, bs, Hkv, D), dtype=dt)
-    vc = torch.zeros((num_blocks, bs, Hkv, D), dtype=dt)
-    for s, (k, v) in enumerate(zip(k_seqs, v_seqs)):
-        for t in range(k.shape[0]):
-            b = int(tables[s][t // bs])
-            kc[b, t % bs] = k[t]
-            vc[b, t % bs] = v[t]
-    return kc, vc
+from tests.helpers import DT, scatter_to_pages
 
 
 def library_attention(q, k, v, scale):
