@@ -30,7 +30,9 @@
 //   an m16n8k16 tensor-core product with the 16 tokens as M and up to 8
 //   heads as N (K tiles through ldmatrix, Q^T fragments in registers);
 //   O^T += V^T P^T takes V^T tiles through ldmatrix.trans and P^T from the
-//   score fragments by movmatrix, with head_dim as M.
+//   score fragments by movmatrix, with head_dim as M; P enters as a 16-bit
+//   high part plus a 16-bit remainder (two products into one accumulator),
+//   so rounding the softmax weights costs no accuracy.
 //
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // PKV_DEVERR_TIMEOUT, waits (bounded) for its loads in flight and skips its
@@ -290,7 +292,7 @@ struct MmaWarp {
         // online softmax per head; the lane holds tokens r0, r0 + 8
         const int r0 = lane >> 2;
         const bool v0 = r0 < valid, v1 = r0 + 8 < valid;
-        uint32_t pb[NT][2];
+        uint32_t pb[NT][2], pl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const float s0 = v0 ? sacc[nt][0] * scale_log2 : -INFINITY;
@@ -318,9 +320,17 @@ struct MmaWarp {
                 acc[mt][nt][2] *= a0;
                 acc[mt][nt][3] *= a1;
             }
-            // P[token][head] as 16-bit fragments, transposed to P^T B-fragments
-            pb[nt][0] = movmatrix_trans(Storage<T>::from_float2(p0, p1));
-            pb[nt][1] = movmatrix_trans(Storage<T>::from_float2(p2, p3));
+            // P[token][head] as 16-bit fragments, transposed to P^T
+            // B-fragments.  P is split into a rounded high part and the
+            // rounded remainder, so the PV product sees P to ~16 bits of
+            // mantissa instead of the 8 of one bf16 rounding.
+            const uint32_t h01 = Storage<T>::from_float2(p0, p1);
+            const uint32_t h23 = Storage<T>::from_float2(p2, p3);
+            const float2 b01 = Storage<T>::to_float2(h01), b23 = Storage<T>::to_float2(h23);
+            pb[nt][0] = movmatrix_trans(h01);
+            pb[nt][1] = movmatrix_trans(h23);
+            pl[nt][0] = movmatrix_trans(Storage<T>::from_float2(p0 - b01.x, p1 - b01.y));
+            pl[nt][1] = movmatrix_trans(Storage<T>::from_float2(p2 - b23.x, p3 - b23.y));
         }
         // O^T[d][head] += V^T P^T over the 16 tokens
 #pragma unroll
@@ -329,7 +339,10 @@ struct MmaWarp {
             const int row = (lane & 7) + (j >> 1) * 8;
             ldmatrix_x4_trans(a, vbase + swz(row, mt * 2 + (j & 1)));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) Mma<T>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                Mma<T>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
+                Mma<T>::m16n8k16(acc[mt][nt], a, pl[nt][0], pl[nt][1]);
+            }
         }
     }
 
