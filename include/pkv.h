@@ -172,6 +172,47 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
                          size_t workspace_bytes, pkv_dtype dtype,
                          int32_t* dev_error, cudaStream_t stream);
 
+/*
+ * Scratch built into the library for pkv_decode_attention_noalloc: the
+ * largest workspace (as pkv_decode_workspace_bytes counts it) that entry
+ * point accepts.
+ */
+#define PKV_NOALLOC_WORKSPACE_BYTES (64u << 20) /* 64 MiB */
+
+/*
+ * pkv_decode_attention for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that are not allowed to call cudaMalloc, or that have no spare memory to
+ * give — for example a host framework whose allocator reserves the whole
+ * device and forbids plug-ins from allocating, or a latency-bound loop that
+ * must not pay for an allocation.  Arguments, results and errors are those
+ * of pkv_decode_attention without `workspace` / `workspace_bytes`: the
+ * caller still passes every input and output, and the split-K scratch comes
+ * from a device array built into the library.
+ *
+ *   - The array is PKV_NOALLOC_WORKSPACE_BYTES long and lives on every GPU
+ *     where this entry point has been called, until the process exits.  A
+ *     call whose sizes need more (see pkv_decode_workspace_bytes) returns
+ *     PKV_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (cudaGetSymbolAddress) and keeps the address; make that first call
+ *     before any stream capture.
+ *   - Nothing here allocates: no cudaMalloc, no cudaFree, no allocating
+ *     library routine.
+ *   - Every call on a device shares the one array, which keeps whatever the
+ *     last call left in it (the kernels write every entry they read, so no
+ *     clearing is needed).  Calls that overlap on the GPU — on different
+ *     streams, or from different host threads — race on it: serialise them.
+ */
+PKV_API int pkv_decode_attention_noalloc(void* out, const void* query, const void* key_cache,
+                                         const void* value_cache, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens,
+                                         int num_seqs, int max_context_len, int num_q_heads,
+                                         int num_kv_heads, int head_dim, int num_blocks,
+                                         int block_size, int64_t block_stride, float scale,
+                                         int partition_size, pkv_dtype dtype,
+                                         int32_t* dev_error, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Host block pool (allocator)                                             */
 /* ---------------------------------------------------------------------- */

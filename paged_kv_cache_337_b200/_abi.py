@@ -29,6 +29,8 @@ PKV_DEVERR_SLOT = 3
 PKV_DEVERR_PAIR = 4
 PKV_DEVERR_TIMEOUT = 5
 
+PKV_NOALLOC_WORKSPACE_BYTES = 64 << 20
+
 _DTYPE = {torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
 
 # name -> (restype, argtypes)
@@ -39,6 +41,8 @@ SIGNATURES = {
     "pkv_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "pkv_decode_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                   _i64, _f, _i, _p, _sz, _i, _p, _p]),
+    "pkv_decode_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
+                                          _i, _i64, _f, _i, _i, _p, _p]),
     "pkv_pool_create": (_i, [_i, _i, _p, C.POINTER(_p)]),
     "pkv_pool_destroy": (None, [_p]),
     "pkv_seq_add": (_i, [_p, _i64, _i]),
@@ -223,6 +227,35 @@ def pkv_decode_attention(out, query, key_cache, value_cache, block_tables, conte
         float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
         _ptr(dev_error), _stream(stream, query.device))
     _check(st, "pkv_decode_attention")
+
+
+def pkv_decode_attention_noalloc(out, query, key_cache, value_cache, block_tables,
+                                 context_lens, max_context_len, scale, partition_size=0,
+                                 dev_error=None, stream=None):
+    """pkv_decode_attention for callers that cannot allocate device memory:
+    the split-K scratch is the library's built-in device array (at most
+    PKV_NOALLOC_WORKSPACE_BYTES), shared by every call on the device, so
+    calls must not overlap on the GPU."""
+    _on_device("pkv_decode_attention_noalloc", out, query, key_cache, value_cache,
+               block_tables, context_lens, dev_error)
+    nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
+        raise ValueError("key_cache and value_cache differ in geometry")
+    S, hq, dq = query.shape
+    if dq != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs, num_q_heads, head_dim]")
+    _need(query, key_cache.dtype, "query")
+    _need(out, key_cache.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and context_lens [num_seqs]")
+    st = lib().pkv_decode_attention_noalloc(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, int(max_context_len), hq, hkv, d, nb, bs,
+        bstride, float(scale), int(partition_size), _dtype(query), _ptr(dev_error),
+        _stream(stream, query.device))
+    _check(st, "pkv_decode_attention_noalloc")
 
 
 def pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):

@@ -1,0 +1,82 @@
+// decode_attention_noalloc.cu — pkv_decode_attention for callers that cannot
+// allocate device memory (a host framework that owns the whole device and
+// forbids plug-ins from calling cudaMalloc, a loop that must not pay for an
+// allocation).  The split-K scratch is a device array built into the
+// library instead of a caller-provided workspace; everything else is the
+// ordinary entry point.  This file holds the array, the per-device lookup of
+// its address and the entry point, and nothing else, so a process that never
+// calls this entry point never loads the array (with lazy module loading).
+#include <mutex>
+
+#include "common.cuh"
+
+namespace pkv {
+namespace {
+
+// Shared by every call on a device; kept until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_workspace[PKV_NOALLOC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_lookup_mutex;
+void* g_workspace_addr[kMaxDevices];  // device address of the array, per device
+
+// Device address of the array on `device`, which must be current.  In host
+// code `g_noalloc_workspace` names a host-side stand-in, not device memory,
+// so the address is looked up once per device and kept.
+int workspace_address(int device, void** addr) {
+    std::lock_guard<std::mutex> lock(g_lookup_mutex);
+    if (g_workspace_addr[device] == nullptr) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(PKV_ERR_CUDA,
+                        "pkv_decode_attention_noalloc: cudaGetSymbolAddress failed on device "
+                        "%d: %s",
+                        device, cudaGetErrorString(e));
+        g_workspace_addr[device] = p;
+    }
+    *addr = g_workspace_addr[device];
+    return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int pkv_decode_attention_noalloc(void* out, const void* query, const void* key_cache,
+                                            const void* value_cache,
+                                            const int32_t* block_tables,
+                                            int max_blocks_per_seq,
+                                            const int32_t* context_lens, int num_seqs,
+                                            int max_context_len, int num_q_heads,
+                                            int num_kv_heads, int head_dim, int num_blocks,
+                                            int block_size, int64_t block_stride, float scale,
+                                            int partition_size, pkv_dtype dtype,
+                                            int32_t* dev_error, cudaStream_t stream) {
+    using namespace pkv;
+    const size_t need = pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len,
+                                                   partition_size, head_dim);
+    PKV_REQUIRE(need <= (size_t)PKV_NOALLOC_WORKSPACE_BYTES, PKV_ERR_WORKSPACE,
+                "pkv_decode_attention_noalloc: these sizes need %zu bytes of split-K scratch, "
+                "more than the %u built into the library; use a larger partition_size or "
+                "pkv_decode_attention with a workspace",
+                need, (unsigned)PKV_NOALLOC_WORKSPACE_BYTES);
+    void* ws = nullptr;
+    if (need > 0) {
+        DeviceGuard guard(stream, key_cache);
+        int device = -1;
+        cudaError_t e = cudaGetDevice(&device);
+        if (e != cudaSuccess)
+            return fail(PKV_ERR_CUDA, "pkv_decode_attention_noalloc: cudaGetDevice: %s",
+                        cudaGetErrorString(e));
+        PKV_REQUIRE(device >= 0 && device < kMaxDevices, PKV_ERR_UNSUPPORTED,
+                    "pkv_decode_attention_noalloc: device %d", device);
+        int st = workspace_address(device, &ws);
+        if (st != PKV_OK) return st;
+    }
+    return pkv_decode_attention(out, query, key_cache, value_cache, block_tables,
+                                max_blocks_per_seq, context_lens, num_seqs, max_context_len,
+                                num_q_heads, num_kv_heads, head_dim, num_blocks, block_size,
+                                block_stride, scale, partition_size, ws,
+                                need > 0 ? (size_t)PKV_NOALLOC_WORKSPACE_BYTES : 0, dtype,
+                                dev_error, stream);
+}
