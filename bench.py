@@ -378,7 +378,7 @@ def run_pkv(args, spec, world, rank, local):
                                   stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        return (1 if state["npairs"] else 0) + 1 + (2 if ws is not None else 1)
+        return (1 if state["npairs"] else 0) + 2
 
     for i in range(args.warmup):
         step(states[i % n_states])
@@ -479,7 +479,7 @@ def run_pkv(args, spec, world, rank, local):
                                                                              spec.len_hi),
                 "pool_blocks": nb, "partition_size": P,
                 "step": "host slot append + slot write + paged decode attention"
-                        " (+ copy-on-write copies, split-K merge)",
+                        " (+ copy-on-write copies; split-K partitions merged in-kernel)",
                 "l2": "inputs larger than L2 (%.2f GB of K/V read per step)" % (
                     states[0]["lens_sum"] * Hkv * D * 4 / 1e9),
                 "states": "%d consecutive decode steps prepared by the host pool, replayed "

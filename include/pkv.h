@@ -124,8 +124,10 @@ PKV_API int pkv_copy_blocks(void* key_cache, void* value_cache,
 /*
  * Bytes of workspace pkv_decode_attention needs for these sizes (0 when every
  * sequence fits one partition, i.e. partition_size == 0 or
- * partition_size >= max_context_len).  The workspace holds, per (seq, query
- * head, partition), the fp32 running maximum, sum and unnormalised output.
+ * partition_size >= max_context_len).  The workspace holds an int32 counter
+ * per (sequence, KV head) — cleared by the library on the caller's stream
+ * before each launch — and, per (seq, query head, partition), the fp32
+ * running maximum, sum and unnormalised output.
  */
 PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads,
                                   int max_context_len, int partition_size,
@@ -154,8 +156,11 @@ PKV_API size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads,
  *   scale            multiplies the dot product before the softmax
  *   partition_size   0: one pass per sequence.  Otherwise a multiple of 16:
  *                    each sequence is split into partitions of that many
- *                    tokens that run in parallel, and a second kernel merges
- *                    their fp32 partial results (split-K for long contexts).
+ *                    tokens that run in parallel; the last partition of a
+ *                    (sequence, KV head) to finish merges their fp32 partial
+ *                    results (split-K for long contexts).  PKV_ERR_UNSUPPORTED
+ *                    when a CTA cannot hold the merge of that many
+ *                    partitions (group * partitions above ~8000).
  *   workspace        device scratch of pkv_decode_workspace_bytes() bytes,
  *                    16-byte aligned (may be NULL when that is 0); its
  *                    contents on entry and exit are unspecified

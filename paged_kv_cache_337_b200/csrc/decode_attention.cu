@@ -18,8 +18,11 @@
 //   Softmax is online (running max and sum in fp32, base-2 exponentials with
 //   scale * log2(e) folded into the scores).  The warps' partial results are
 //   merged through shared memory at the end; with several partitions the CTA
-//   writes fp32 (max, sum, unnormalised output) to the workspace and a merge
-//   kernel combines them.
+//   writes fp32 (max, sum, unnormalised output) to the workspace, and the
+//   last CTA of each (sequence, KV head) to finish merges them (a counter
+//   per pair, cleared by a memset on the stream before the launch).  The
+//   flat grid runs a pair's partitions side by side, so merges overlap the
+//   streaming of later pairs.
 //
 // Arithmetic paths
 //   G == 1 (no grouping): a GEMV; FFMA with warp shuffles.  Lane l owns
@@ -51,7 +54,18 @@ namespace {
 constexpr int kTile = 16;                          // tokens per tile
 constexpr int kBoxD = 64;                          // head_dim per TMA box (128 B)
 constexpr int kSubTileBytes = kTile * kBoxD * 2;   // one swizzled box: 2 KiB
-constexpr int kWarps = 4;
+// Compile-time shape of the attention CTA: warps per CTA and TMA stages per
+// warp (one stage holds the K and V tiles of 16 tokens).
+#ifndef PKV_DECODE_WARPS
+#define PKV_DECODE_WARPS 4
+#endif
+#ifndef PKV_DECODE_STAGES_D128
+#define PKV_DECODE_STAGES_D128 2
+#endif
+#ifndef PKV_DECODE_STAGES_D64
+#define PKV_DECODE_STAGES_D64 4
+#endif
+constexpr int kWarps = PKV_DECODE_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -60,7 +74,7 @@ struct Geom {
     static constexpr int kBoxes = D / kBoxD;             // boxes per K (or V) tile
     static constexpr int kKBytes = kBoxes * kSubTileBytes;
     static constexpr int kStageBytes = 2 * kKBytes;      // K + V of one tile
-    static constexpr int kStages = D == 128 ? 3 : 4;
+    static constexpr int kStages = D == 128 ? PKV_DECODE_STAGES_D128 : PKV_DECODE_STAGES_D64;
 };
 
 struct DecodeParams {
@@ -71,8 +85,10 @@ struct DecodeParams {
     float* ws_m;
     float* ws_l;
     float* ws_o;
+    int32_t* ws_count;  // [S, Hkv]: partitions finished (zeroed before the launch)
     int32_t* dev_error;
     int num_seqs;
+    int num_kv_heads;
     int max_blocks_per_seq;
     int max_context_len;
     int num_q_heads;
@@ -403,9 +419,34 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * STAGES * Gm::kStageBytes);
     int32_t* table = reinterpret_cast<int32_t*>(bars + kWarps * STAGES);
 
-    const int s = blockIdx.x, kvh = blockIdx.y, part = blockIdx.z;
+    // Flat grid, partition fastest: the partitions of one (sequence, KV
+    // head) run side by side, so their merge happens early and in parallel
+    // with the other CTAs' streaming rather than all at the end.
+    const int part = (int)(blockIdx.x % (unsigned)p.num_partitions);
+    const int rest = (int)(blockIdx.x / (unsigned)p.num_partitions);
+    const int kvh = rest % p.num_kv_heads;
+    const int s = rest / p.num_kv_heads;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group, bs = p.block_size, P = p.partition_size;
+
+    uint64_t* my_bars = bars + warp * STAGES;
+    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+    // The partition's first table entries are read together with the
+    // context length (the row index does not depend on it), so the two
+    // global loads overlap instead of forming a chain before the first TMA.
+    const int lb0 = part * P / bs;
+    const int32_t* trow = p.block_tables + (int64_t)s * p.max_blocks_per_seq + lb0;
+    const int row_left = p.max_blocks_per_seq - lb0;  // > 0: part < NP
+    const int32_t spec = threadIdx.x < row_left ? __ldg(trow + threadIdx.x) : -1;
 
     bool bad_len;
     const int L = checked_len(p, s, &bad_len);
@@ -416,26 +457,13 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     const int t_begin = part * P;
     const int t_end = min(L, t_begin + P);
     const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
-    const int lb0 = t_begin / bs;
     const int nlb = t_end > t_begin ? (t_end - 1) / bs - lb0 + 1 : 0;
 
-    if (threadIdx.x == 0) {
-        prefetch_tensormap(&kmap);
-        prefetch_tensormap(&vmap);
-    }
-    // this partition's slice of the Block Table, one load per logical block
-    const int32_t* trow = p.block_tables + (int64_t)s * p.max_blocks_per_seq + lb0;
+    // this partition's slice of the Block Table, one entry per logical block
     for (int i = threadIdx.x; i < nlb; i += kWarps * 32) {
-        const int32_t b = __ldg(trow + i);
+        const int32_t b = i < kWarps * 32 ? spec : __ldg(trow + i);
         if (b < 0 || b >= p.num_blocks) report_error(p.dev_error, PKV_DEVERR_BLOCK_ID, s);
         table[i] = b;
-    }
-    uint64_t* my_bars = bars + warp * STAGES;
-    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
-        fence_barrier_init();
     }
     __syncthreads();
 
@@ -524,6 +552,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     __syncthreads();
 
     const int Hq = p.num_q_heads;
+    const int64_t qh0 = (int64_t)s * Hq + (int64_t)kvh * G;  // first query head
     for (int idx = threadIdx.x; idx < G * D; idx += kWarps * 32) {
         const int h = idx / D, d = idx - h * D;
         const float M = sm_M[h];
@@ -534,11 +563,11 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             Lsum += M == -INFINITY ? 0.f : sm_l[k * GP + h] * exp2f(mk - M);
             O += sm_o[(k * G + h) * D + d];
         }
-        const int64_t qh = (int64_t)s * Hq + (int64_t)kvh * G + h;
         if (np == 1) {
-            static_cast<T*>(p.out)[qh * D + d] = Storage<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+            static_cast<T*>(p.out)[(qh0 + h) * D + d] =
+                Storage<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
         } else {
-            const int64_t wi = qh * p.num_partitions + part;
+            const int64_t wi = (qh0 + h) * p.num_partitions + part;
             p.ws_o[wi * D + d] = O;
             if (d == 0) {
                 p.ws_m[wi] = M;
@@ -546,63 +575,76 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
     }
-}
+    if (np == 1) return;
 
-// ---------------------------------------------------------------------------
-// Merge of split-K partials: with M = max_p m_p and w_p = 2^(m_p - M),
-// out = sum_p w_p o_p / sum_p w_p l_p  (m in base-2 units of scaled scores).
-// One warp per (sequence, query head); sequences that fit one partition were
-// finished by the attention kernel.
-// ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
-    constexpr int DV = D / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int Hq = p.num_q_heads;
-    const int64_t qh = (int64_t)blockIdx.x * 4 + warp;
-    if (qh >= (int64_t)p.num_seqs * Hq) return;
-    const int s = (int)(qh / Hq);
-    bool bad;
-    const int L = checked_len(p, s, &bad);
-    const int P = p.partition_size;
-    const int np = L > 0 ? (L + P - 1) / P : 1;
-    if (np <= 1) return;
-    const float* m = p.ws_m + qh * p.num_partitions;
-    const float* l = p.ws_l + qh * p.num_partitions;
-    const float* o = p.ws_o + qh * p.num_partitions * D;
-    float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, m[i]);
-#pragma unroll
-    for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, x));
-    float Lsum = 0.f;
-    for (int i = lane; i < np; i += 32) Lsum += l[i] * exp2f(m[i] - M);
-#pragma unroll
-    for (int x = 16; x > 0; x >>= 1) Lsum += __shfl_xor_sync(kFull, Lsum, x);
-    float acc[DV];
-#pragma unroll
-    for (int j = 0; j < DV; ++j) acc[j] = 0.f;
-    for (int i = 0; i < np; ++i) {
-        const float wgt = exp2f(m[i] - M);
-        const float* oi = o + (int64_t)i * D + lane * DV;
-        if constexpr (DV == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(oi);
-            acc[0] = fmaf(wgt, v.x, acc[0]);
-            acc[1] = fmaf(wgt, v.y, acc[1]);
-            acc[2] = fmaf(wgt, v.z, acc[2]);
-            acc[3] = fmaf(wgt, v.w, acc[3]);
-        } else {
-            const float2 v = *reinterpret_cast<const float2*>(oi);
-            acc[0] = fmaf(wgt, v.x, acc[0]);
-            acc[1] = fmaf(wgt, v.y, acc[1]);
+    // ---- split-K merge, done by the last partition to finish ----------------
+    // Each CTA publishes its partial (m, l, o), then counts itself in; the
+    // CTA that brings the count to np merges all np partials of this
+    // (sequence, KV head):  M = max_p m_p,  w_p = 2^(m_p - M),
+    // out = sum_p w_p o_p / sum_p w_p l_p.
+    __shared__ int sm_last;
+    __threadfence();
+    __syncthreads();
+    int32_t* count = p.ws_count + (int64_t)s * p.num_kv_heads + kvh;
+    if (threadIdx.x == 0) sm_last = atomicAdd(count, 1) == np - 1;
+    __syncthreads();
+    if (!sm_last) return;
+    __threadfence();
+    float* w_m = reinterpret_cast<float*>(stages);  // [G][np]: m, then the weights
+    float* w_l = w_m + G * np;                      // [G][np]
+    float* h_M = w_l + G * np;                      // [G]
+    float* h_L = h_M + G;                           // [G]
+    for (int i = threadIdx.x; i < G * np; i += kWarps * 32) {
+        const int h = i / np, pp = i - h * np;
+        const int64_t wi = (qh0 + h) * p.num_partitions + pp;
+        w_m[i] = __ldcg(p.ws_m + wi);
+        w_l[i] = __ldcg(p.ws_l + wi);
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const float* mh = w_m + threadIdx.x * np;
+        float M = -INFINITY;
+        for (int pp = 0; pp < np; ++pp) M = fmaxf(M, mh[pp]);
+        h_M[threadIdx.x] = M;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G * np; i += kWarps * 32) {
+        const float wgt = exp2f(w_m[i] - h_M[i / np]);
+        w_m[i] = wgt;
+        w_l[i] *= wgt;
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const float* lh = w_l + threadIdx.x * np;
+        float Lsum = 0.f;
+        for (int pp = 0; pp < np; ++pp) Lsum += lh[pp];
+        h_L[threadIdx.x] = Lsum;
+    }
+    __syncthreads();
+    // four consecutive dims per thread: float4 loads of the partials
+    for (int idx = threadIdx.x; idx < G * D / 4; idx += kWarps * 32) {
+        const int h = idx / (D / 4), d4 = (idx - h * (D / 4)) * 4;
+        const float* wh = w_m + h * np;
+        const float4* o = reinterpret_cast<const float4*>(
+            p.ws_o + ((qh0 + h) * p.num_partitions) * D + d4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int pp = 0; pp < np; ++pp) {
+            const float4 v = __ldcg(o + (int64_t)pp * (D / 4));
+            const float wgt = wh[pp];
+            acc.x = fmaf(wgt, v.x, acc.x);
+            acc.y = fmaf(wgt, v.y, acc.y);
+            acc.z = fmaf(wgt, v.z, acc.z);
+            acc.w = fmaf(wgt, v.w, acc.w);
         }
+        const float inv = 1.f / h_L[h];
+        T* dst = static_cast<T*>(p.out) + (qh0 + h) * D + d4;
+        uint2 packed;
+        packed.x = Storage<T>::from_float2(acc.x * inv, acc.y * inv);
+        packed.y = Storage<T>::from_float2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(dst) = packed;
     }
-    const float inv = 1.f / Lsum;
-    T* out = static_cast<T*>(p.out) + qh * D + lane * DV;
-#pragma unroll
-    for (int j = 0; j < DV; j += 2) {
-        const uint32_t w = Storage<T>::from_float2(acc[j] * inv, acc[j + 1] * inv);
-        *reinterpret_cast<uint32_t*>(out + j) = w;
-    }
+    if (threadIdx.x == 0) *count = 0;  // ready for the next launch
 }
 
 // ---------------------------------------------------------------------------
@@ -645,18 +687,22 @@ int encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dtype, int h
 }
 
 struct WorkspaceLayout {
-    size_t m_off, l_off, o_off, total;
+    size_t count_off, m_off, l_off, o_off, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// int32 partition counters (one per (seq, KV head); room for S * Hq) |
+// m [S, Hq, NP] | l [S, Hq, NP] | o [S, Hq, NP, D], each 256-byte aligned
 WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t NP, int64_t D) {
     WorkspaceLayout w;
+    const size_t cnt = align256((size_t)(S * Hq) * sizeof(int32_t));
     const size_t ml = align256((size_t)(S * Hq * NP) * sizeof(float));
-    w.m_off = 0;
-    w.l_off = ml;
-    w.o_off = 2 * ml;
-    w.total = 2 * ml + align256((size_t)(S * Hq * NP * D) * sizeof(float));
+    w.count_off = 0;
+    w.m_off = cnt;
+    w.l_off = cnt + ml;
+    w.o_off = cnt + 2 * ml;
+    w.total = cnt + 2 * ml + align256((size_t)(S * Hq * NP * D) * sizeof(float));
     return w;
 }
 
@@ -685,18 +731,31 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
                     "pkv_decode_attention: %d tokens per partition need %zu bytes of shared "
                     "memory; use a smaller partition_size",
                     p.partition_size, smem);
+    // the merging CTA keeps the partials' m and l of its G heads in the
+    // (then idle) stage buffers
+    const size_t merge_smem = (size_t)p.group * (2 * p.num_partitions + 2) * sizeof(float);
+    if (p.num_partitions > 1 && merge_smem > (size_t)kWarps * Gm::kStages * Gm::kStageBytes)
+        return fail(PKV_ERR_UNSUPPORTED,
+                    "pkv_decode_attention: %d partitions of %d query heads are too many to "
+                    "merge in one CTA; use a larger partition_size",
+                    p.num_partitions, p.group);
     auto kern = paged_decode_kernel<T, D, Warp>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess)
         return fail(PKV_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    dim3 grid(p.num_seqs, num_kv_heads, p.num_partitions);
-    kern<<<grid, kWarps * 32, smem, stream>>>(kmap, vmap, p);
-    int st = launch_status("pkv_decode_attention");
-    if (st != PKV_OK || p.num_partitions == 1) return st;
-    const int64_t pairs = (int64_t)p.num_seqs * p.num_q_heads;
-    paged_decode_merge_kernel<T, D><<<(unsigned)((pairs + 3) / 4), 128, 0, stream>>>(p);
-    return launch_status("pkv_decode_attention (merge)");
+    if (p.num_partitions > 1) {
+        e = cudaMemsetAsync(p.ws_count, 0, (size_t)p.num_seqs * num_kv_heads * sizeof(int32_t),
+                            stream);
+        if (e != cudaSuccess)
+            return fail(PKV_ERR_CUDA, "pkv_decode_attention: clearing the partition counters: %s",
+                        cudaGetErrorString(e));
+    }
+    const int64_t ctas = (int64_t)p.num_seqs * num_kv_heads * p.num_partitions;
+    if (ctas >= (1ll << 31))
+        return fail(PKV_ERR_UNSUPPORTED, "pkv_decode_attention: %lld CTAs", (long long)ctas);
+    kern<<<(unsigned)ctas, kWarps * 32, smem, stream>>>(kmap, vmap, p);
+    return launch_status("pkv_decode_attention");
 }
 
 template <typename T, int D>
@@ -774,6 +833,7 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
     p.context_lens = context_lens;
     p.dev_error = dev_error;
     p.num_seqs = num_seqs;
+    p.num_kv_heads = num_kv_heads;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_context_len = max_context_len;
     p.num_q_heads = num_q_heads;
@@ -794,6 +854,7 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
         p.ws_m = reinterpret_cast<float*>(base + w.m_off);
         p.ws_l = reinterpret_cast<float*>(base + w.l_off);
         p.ws_o = reinterpret_cast<float*>(base + w.o_off);
+        p.ws_count = reinterpret_cast<int32_t*>(base + w.count_off);
     }
 
     CUtensorMap kmap, vmap;

@@ -47,9 +47,11 @@ def test_host_only_calls(lib):
     # no partitions -> no workspace
     assert _abi.pkv_decode_workspace_bytes(4, 8, 100, 0, 64) == 0
     assert _abi.pkv_decode_workspace_bytes(4, 8, 100, 128, 64) == 0
-    # 8 seqs x 32 heads x 64 partitions: m and l (256-byte aligned) + o
+    # 8 seqs x 32 heads x 64 partitions: counters (room for 8 x 32), m and l
+    # (each 256-byte aligned) + o
     n = 8 * 32 * 64
-    assert _abi.pkv_decode_workspace_bytes(8, 32, 32768, 512, 128) == 2 * n * 4 + n * 128 * 4
+    assert _abi.pkv_decode_workspace_bytes(8, 32, 32768, 512, 128) == \
+        1024 + 2 * n * 4 + n * 128 * 4
 
 
 def test_argument_errors_are_reported_before_any_launch(lib):
