@@ -291,20 +291,30 @@ struct MmaWarp {
         const uint32_t kbase = smem_addr(kt), vbase = smem_addr(vt);
         const int j = lane >> 3;
         // S^T[token][head] = K Q^T over head_dim
-        float sacc[NT][4];
+        // two independent accumulator chains (even / odd k-steps) halve the
+        // dependent MMA latency, then add
+        float sacc[NT][4], sacc2[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sacc[nt][i] = 0.f;
+            for (int i = 0; i < 4; ++i) sacc[nt][i] = sacc2[nt][i] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
             uint32_t a[4];
             const int row = (lane & 7) + (j & 1) * 8;
             ldmatrix_x4(a, kbase + swz(row, kk * 2 + (j >> 1)));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                Mma<T>::m16n8k16(sacc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (kk & 1)
+                    Mma<T>::m16n8k16(sacc2[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                else
+                    Mma<T>::m16n8k16(sacc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+            }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[nt][i] += sacc2[nt][i];
         // online softmax per head; the lane holds tokens r0, r0 + 8
         const int r0 = lane >> 2;
         const bool v0 = r0 < valid, v1 = r0 + 8 < valid;
@@ -429,17 +439,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group, bs = p.block_size, P = p.partition_size;
 
-    uint64_t* my_bars = bars + warp * STAGES;
-    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
-        fence_barrier_init();
-    }
-    if (threadIdx.x == 0) {
-        prefetch_tensormap(&kmap);
-        prefetch_tensormap(&vmap);
-    }
     // The partition's first table entries are read together with the
     // context length (the row index does not depend on it), so the two
     // global loads overlap instead of forming a chain before the first TMA.
@@ -453,7 +452,19 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     if (bad_len && part == 0 && kvh == 0 && threadIdx.x == 0)
         report_error(p.dev_error, PKV_DEVERR_CONTEXT_LEN, s);
     const int np = L > 0 ? (L + P - 1) / P : 1;
-    if (part >= np) return;
+    if (part >= np) return;  // a partition past this sequence's end
+
+    uint64_t* my_bars = bars + warp * STAGES;
+    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
+        fence_barrier_init();
+    }
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
     const int t_begin = part * P;
     const int t_end = min(L, t_begin + P);
     const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
@@ -517,7 +528,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             __syncwarp();
         }
         w.tile(kt, vt, valid, p.scale_log2, lane);
-        fence_proxy_async();  // our reads of this stage before TMA rewrites it
+        // Every shared-memory read of this stage feeds an instruction that
+        // precedes the next TMA issue in program order, so the reads are
+        // complete before the stage is rewritten.
         __syncwarp();
         const int next = it + STAGES;
         if (lane == 0 && next < my_tiles) issue(st, warp + next * kWarps);
