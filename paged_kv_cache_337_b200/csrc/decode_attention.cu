@@ -12,9 +12,10 @@
 //   byte is read from HBM once per step.  Each of the CTA's warps owns every
 //   NW-th 16-token tile of the partition and runs its own TMA pipeline:
 //   lane 0 resolves the tile's physical block from the partition's slice of
-//   the Block Table (staged in shared memory once per CTA) and issues 4-D
-//   tiled TMA loads of the K and V tiles into a STAGES-deep ring of
-//   128B-swizzled shared-memory buffers, completing on per-stage mbarriers.
+//   the Block Table (staged in shared memory once per CTA) and issues one
+//   5-D tiled TMA load for the K tile and one for the V tile into a
+//   STAGES-deep ring of 128B-swizzled shared-memory buffers, completing on
+//   per-stage mbarriers.
 //   Softmax is online (running max and sum in fp32, base-2 exponentials with
 //   scale * log2(e) folded into the scores).  The warps' partial results are
 //   merged through shared memory at the end; with several partitions the CTA
@@ -486,12 +487,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
         uint8_t* kdst = my_stages + st * Gm::kStageBytes;
         uint8_t* vdst = kdst + Gm::kKBytes;
         mbar_arrive_expect_tx(&my_bars[st], Gm::kStageBytes);
-#pragma unroll
-        for (int b = 0; b < Gm::kBoxes; ++b)
-            tma_load_4d(kdst + b * kSubTileBytes, &kmap, &my_bars[st], b * kBoxD, kvh, off, phys);
-#pragma unroll
-        for (int b = 0; b < Gm::kBoxes; ++b)
-            tma_load_4d(vdst + b * kSubTileBytes, &vmap, &my_bars[st], b * kBoxD, kvh, off, phys);
+        // one instruction per tile and cache: all head_dim / 64 boxes
+        tma_load_5d(kdst, &kmap, &my_bars[st], 0, kvh, off, 0, phys);
+        tma_load_5d(vdst, &vmap, &my_bars[st], 0, kvh, off, 0, phys);
     };
 
     const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
@@ -677,22 +675,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 4-D view of one cache: (head_dim, kv head, slot in block, physical block),
-// boxes of 64 x 1 x 16 x 1 elements with 128-byte swizzling.
+// 5-D view of one cache: (64 dims, kv head, slot in block, 64-dim half,
+// physical block).  The halves are 128 bytes apart; putting them after the
+// slot makes one box of 64 x 1 x 16 x (head_dim / 64) x 1 elements land in
+// shared memory as head_dim / 64 swizzled 16-row x 128-byte sub-tiles, so a
+// single TMA instruction fetches a whole K (or V) tile.
 int encode_cache_map(CUtensorMap* map, const void* cache, pkv_dtype dtype, int head_dim,
                      int num_kv_heads, int block_size, int num_blocks, int64_t block_stride) {
     auto fn = encode_fn();
     if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-    const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
-                                (cuuint64_t)block_size, (cuuint64_t)num_blocks};
-    const cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2,
+    const cuuint64_t dims[5] = {(cuuint64_t)kBoxD, (cuuint64_t)num_kv_heads,
+                                (cuuint64_t)block_size, (cuuint64_t)(head_dim / kBoxD),
+                                (cuuint64_t)num_blocks};
+    const cuuint64_t strides[4] = {(cuuint64_t)head_dim * 2,
                                    (cuuint64_t)num_kv_heads * head_dim * 2,
-                                   (cuuint64_t)block_stride * 2};
-    const cuuint32_t box[4] = {kBoxD, 1, kTile, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
+                                   (cuuint64_t)kBoxD * 2, (cuuint64_t)block_stride * 2};
+    const cuuint32_t box[5] = {kBoxD, 1, kTile, (cuuint32_t)(head_dim / kBoxD), 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     const CUtensorMapDataType ty = dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    CUresult r = fn(map, ty, 4, const_cast<void*>(cache), dims, strides, box, estr,
+    CUresult r = fn(map, ty, 5, const_cast<void*>(cache), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
