@@ -283,10 +283,11 @@ PKV_API int pkv_seq_block_table(const pkv_pool* pool, int64_t seq_id, int32_t* o
                         int cap, int* n);
 
 /* Fills a dense [n, max_blocks_per_seq] table for seq_ids (rows padded with
- * `fill`) and, if context_lens is not NULL, their token counts. */
+ * `fill`), and, where the pointers are not NULL, their token counts and the
+ * largest of them. */
 PKV_API int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t* seq_ids,
                           int32_t* out, int max_blocks_per_seq, int32_t fill,
-                          int32_t* context_lens);
+                          int32_t* context_lens, int32_t* max_context_len);
 
 PKV_API int pkv_pool_num_free(const pkv_pool* pool);
 PKV_API int pkv_pool_num_blocks(const pkv_pool* pool);
@@ -306,6 +307,14 @@ PKV_API int pkv_block_refcount(const pkv_pool* pool, int block);
  * num_layers * dtype_bytes.  Negative on bad arguments. */
 PKV_API int64_t pkv_block_bytes(int block_size, int num_kv_heads, int head_dim,
                         int num_layers, int dtype_bytes);
+
+/* Self-test of the kernels' failure path: launches one CTA that waits, with
+ * the same bounded wait the attention kernel uses, on an mbarrier that never
+ * completes.  After limit_us microseconds (1 .. 10^6) the wait gives up and
+ * records {PKV_DEVERR_TIMEOUT, 0} in dev_error (device int32[2], zeroed by
+ * the caller); the context stays usable.  No other kernel waits are
+ * affected. */
+PKV_API int pkv_selftest_bounded_wait(int32_t* dev_error, int limit_us, cudaStream_t stream);
 
 PKV_API const char* pkv_status_string(int status);
 /* Message of the calling thread's last failed call ("" if none). */

@@ -53,13 +53,14 @@ SIGNATURES = {
     "pkv_seq_num_tokens": (_i, [_p, _i64, _p]),
     "pkv_seq_block_table": (_i, [_p, _i64, _p, _i, _p]),
     "pkv_seq_slot_mapping": (_i, [_p, _i64, _i, _i, _p]),
-    "pkv_pool_block_tables": (_i, [_p, _i, _p, _p, _i, C.c_int32, _p]),
+    "pkv_pool_block_tables": (_i, [_p, _i, _p, _p, _i, C.c_int32, _p, _p]),
     "pkv_pool_num_free": (_i, [_p]),
     "pkv_pool_num_blocks": (_i, [_p]),
     "pkv_pool_block_size": (_i, [_p]),
     "pkv_pool_free_list": (_i, [_p, _p, _i, _p]),
     "pkv_block_refcount": (_i, [_p, _i]),
     "pkv_block_bytes": (_i64, [_i, _i, _i, _i, _i]),
+    "pkv_selftest_bounded_wait": (_i, [_p, _i, _p]),
     "pkv_status_string": (C.c_char_p, [_i]),
     "pkv_last_error": (C.c_char_p, []),
     "pkv_version": (_i, []),
@@ -258,6 +259,16 @@ def pkv_decode_attention_noalloc(out, query, key_cache, value_cache, block_table
     _check(st, "pkv_decode_attention_noalloc")
 
 
+def pkv_selftest_bounded_wait(dev_error, limit_us, stream=None):
+    """Run one bounded mbarrier wait that can never complete; the kernel
+    records PKV_DEVERR_TIMEOUT in dev_error (int32[2] on the device)."""
+    _on_device("pkv_selftest_bounded_wait", dev_error)
+    _need(dev_error, torch.int32, "dev_error")
+    _check(lib().pkv_selftest_bounded_wait(_ptr(dev_error), int(limit_us),
+                                           _stream(stream, dev_error.device)),
+           "pkv_selftest_bounded_wait")
+
+
 def pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):
     v = int(lib().pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes))
     if v < 0:
@@ -349,17 +360,21 @@ class BlockPool:
                "pkv_seq_block_table")
         return list(buf[:n.value])
 
-    def block_tables(self, seq_ids, max_blocks_per_seq, fill=-1, out=None, lens_out=None):
-        """Dense int32 [n, max_blocks_per_seq] tables and int32 [n] lengths."""
+    def block_tables(self, seq_ids, max_blocks_per_seq, fill=-1, out=None, lens_out=None,
+                     with_max=False):
+        """Dense int32 [n, max_blocks_per_seq] tables and int32 [n] lengths
+        (and, with with_max, the largest length)."""
         ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
         n = ids.numel()
         tables = out if out is not None else torch.empty((n, max_blocks_per_seq),
                                                          dtype=torch.int32)
         lens = lens_out if lens_out is not None else torch.empty(n, dtype=torch.int32)
+        longest = C.c_int32(0)
         st = lib().pkv_pool_block_tables(self._h, n, _ptr(ids), _ptr(tables),
-                                         max_blocks_per_seq, fill, _ptr(lens))
+                                         max_blocks_per_seq, fill, _ptr(lens),
+                                         C.byref(longest))
         _check(st, "pkv_pool_block_tables")
-        return tables, lens
+        return (tables, lens, longest.value) if with_max else (tables, lens)
 
     def num_free(self):
         v = lib().pkv_pool_num_free(self._h)

@@ -44,6 +44,9 @@ class PagedKVCache:
         self.dev_error = torch.zeros(2, dtype=torch.int32, device=self.device)
         self._workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
         self._staging = {}
+        self._seen = set()  # tensor signatures the binding has checked
+        self._geom = _abi._cache_geometry(self.key_cache)
+        self._dtype_code = _abi._dtype(self.key_cache)
 
     # -- sequence management (host) ---------------------------------------
     def add_sequence(self, seq_id, num_tokens, key=None, value=None, stream=None):
@@ -64,50 +67,56 @@ class PagedKVCache:
 
     # -- one decode step --------------------------------------------------
     def _stage(self, n):
-        """Pinned host staging and device buffers for a batch of n sequences."""
-        st = self._staging.get(n)
-        if st is None:
+        """Staging for a batch of n sequences: two banks, each one pinned host
+        buffer and one device buffer holding slots | lengths | copy pairs |
+        Block Tables, so a step's metadata travels in one copy and the next
+        step can be prepared while the previous upload is in flight."""
+        banks = self._staging.get(n)
+        if banks is None:
             pin = torch.cuda.is_available()
             mb = self.max_blocks_per_seq
-            st = dict(
-                ids=torch.empty(n, dtype=torch.int64),
-                h_slots=torch.empty(n, dtype=torch.int64, pin_memory=pin),
-                h_pairs=torch.empty((n, 2), dtype=torch.int32, pin_memory=pin),
-                h_tables=torch.empty((n, mb), dtype=torch.int32, pin_memory=pin),
-                h_lens=torch.empty(n, dtype=torch.int32, pin_memory=pin),
-                d_slots=torch.empty(n, dtype=torch.int64, device=self.device),
-                d_pairs=torch.empty((n, 2), dtype=torch.int32, device=self.device),
-                d_tables=torch.empty((n, mb), dtype=torch.int32, device=self.device),
-                d_lens=torch.empty(n, dtype=torch.int32, device=self.device),
-            )
-            self._staging[n] = st
-        return st
+            words = 2 * n + n + 2 * n + n * mb  # int32 words
+
+            def views(buf):
+                return dict(slots=buf[:2 * n].view(torch.int64), lens=buf[2 * n:3 * n],
+                            pairs=buf[3 * n:5 * n].view(n, 2), tables=buf[5 * n:].view(n, mb))
+
+            banks = []
+            for _ in range(2):
+                h = torch.empty(words, dtype=torch.int32, pin_memory=pin)
+                d = torch.empty(words, dtype=torch.int32, device=self.device)
+                hv, dv = views(h), views(d)
+                banks.append(dict(ids=torch.empty(n, dtype=torch.int64), h=h, d=d,
+                                  h_slots=hv["slots"], h_lens=hv["lens"], h_pairs=hv["pairs"],
+                                  h_tables=hv["tables"], d_slots=dv["slots"],
+                                  d_lens=dv["lens"], d_pairs=dv["pairs"],
+                                  d_tables=dv["tables"], uploaded=None))
+            self._staging[n] = banks = [banks, 0]
+        banks[1] ^= 1
+        return banks[0][banks[1]]
 
     def prepare_step(self, seq_ids):
-        """Host part of a decode step: reserve one slot per sequence and
-        gather tables and lengths into pinned buffers.  Returns a dict of
-        host tensors and the step's maximum context length."""
+        """Host part of a decode step: reserve one slot per sequence (new
+        blocks and copy-on-write pairs as needed) and gather the Block Tables
+        and lengths into pinned memory.  Returns the prepared step."""
         st = self._stage(len(seq_ids))
-        if st.get("uploaded") is not None:
-            st["uploaded"].synchronize()  # the previous copies out of these buffers are done
-        st["ids"].copy_(torch.as_tensor(seq_ids, dtype=torch.int64))
+        if st["uploaded"] is not None:
+            st["uploaded"].synchronize()  # this bank's last upload has left
+        if st.get("ids_src") is not seq_ids:  # a new id list: convert it once
+            st["ids"].copy_(torch.as_tensor(seq_ids, dtype=torch.int64))
+            st["ids_src"] = seq_ids
         slots, pairs = self.pool.append_batch(st["ids"], st["h_slots"], st["h_pairs"])
-        tables, lens = self.pool.block_tables(st["ids"], self.max_blocks_per_seq, -1,
-                                              st["h_tables"], st["h_lens"])
-        return dict(st=st, num_pairs=pairs.shape[0], max_len=int(lens.max()) if len(lens) else 0)
+        tables, lens, longest = self.pool.block_tables(
+            st["ids"], self.max_blocks_per_seq, -1, st["h_tables"], st["h_lens"], with_max=True)
+        return dict(st=st, num_pairs=pairs.shape[0], max_len=longest)
 
     def upload_step(self, prep, stream=None):
-        """Host-to-device copies of a prepared step's metadata."""
+        """One host-to-device copy of a prepared step's metadata."""
         st = prep["st"]
-        n = prep["num_pairs"]
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         with torch.cuda.stream(s):
-            st["d_slots"].copy_(st["h_slots"], non_blocking=True)
-            if n:
-                st["d_pairs"][:n].copy_(st["h_pairs"][:n], non_blocking=True)
-            st["d_tables"].copy_(st["h_tables"], non_blocking=True)
-            st["d_lens"].copy_(st["h_lens"], non_blocking=True)
-            if st.get("uploaded") is None:
+            st["d"].copy_(st["h"], non_blocking=True)
+            if st["uploaded"] is None:
                 st["uploaded"] = torch.cuda.Event()
             st["uploaded"].record(s)
 
@@ -127,14 +136,43 @@ class PagedKVCache:
         if n:
             _abi.pkv_copy_blocks(self.key_cache, self.value_cache, st["d_pairs"][:n],
                                  dev_error=self.dev_error, stream=stream)
-        _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, st["d_slots"],
-                             dev_error=self.dev_error, stream=stream)
-        _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache,
-                                  st["d_tables"], st["d_lens"], max_len,
-                                  self.scale, self.partition_size,
-                                  self.workspace(len(st["ids"]), max_len),
-                                  dev_error=self.dev_error, stream=stream)
+        ws = self.workspace(len(st["ids"]), max_len)
+        if not self._checked(query, key, value, out):
+            # first use of these tensor shapes: the binding's full checks
+            _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, st["d_slots"],
+                                 dev_error=self.dev_error, stream=stream)
+            _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache,
+                                      st["d_tables"], st["d_lens"], max_len, self.scale,
+                                      self.partition_size, ws, dev_error=self.dev_error,
+                                      stream=stream)
+            self._seen.add(self._signature(query, key, value, out))
+            return out
+        # same shapes, dtypes and device as a call already checked: pass the
+        # pointers straight to the C entry points
+        L = _abi.lib()
+        sp = _abi._stream(stream, self.device)
+        kc, vc = self.key_cache, self.value_cache
+        nb, bs, hkv, d, bstride = self._geom
+        S = query.shape[0]
+        _abi._check(L.pkv_write_slots(key.data_ptr(), value.data_ptr(), kc.data_ptr(),
+                                      vc.data_ptr(), st["d_slots"].data_ptr(), S, nb, bs, hkv,
+                                      d, bstride, self._dtype_code, self.dev_error.data_ptr(),
+                                      sp), "pkv_write_slots")
+        _abi._check(L.pkv_decode_attention(
+            out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+            st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
+            int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
+            int(self.partition_size), ws.data_ptr() if ws is not None else None,
+            ws.numel() if ws is not None else 0, self._dtype_code, self.dev_error.data_ptr(),
+            sp), "pkv_decode_attention")
         return out
+
+    def _signature(self, query, key, value, out):
+        return tuple((tuple(t.shape), t.dtype, t.device, t.is_contiguous())
+                     for t in (query, key, value, out))
+
+    def _checked(self, query, key, value, out):
+        return self._signature(query, key, value, out) in self._seen
 
     def decode_step(self, seq_ids, query, key, value, out=None, stream=None):
         """One full decode step for seq_ids (query [S, Hq, D], key/value

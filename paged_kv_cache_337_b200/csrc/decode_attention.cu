@@ -593,14 +593,20 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     // CTA that brings the count to np merges all np partials of this
     // (sequence, KV head):  M = max_p m_p,  w_p = 2^(m_p - M),
     // out = sum_p w_p o_p / sum_p w_p l_p.
+    // The barrier orders every thread's partial stores before thread 0's
+    // fence, and a fence is cumulative, so one fence publishes them all
+    // before the count; symmetrically the merging CTA's thread 0 fences
+    // after the count and the barrier passes that on to its readers.
     __shared__ int sm_last;
-    __threadfence();
     __syncthreads();
     int32_t* count = p.ws_count + (int64_t)s * p.num_kv_heads + kvh;
-    if (threadIdx.x == 0) sm_last = atomicAdd(count, 1) == np - 1;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        sm_last = atomicAdd(count, 1) == np - 1;
+        if (sm_last) __threadfence();
+    }
     __syncthreads();
     if (!sm_last) return;
-    __threadfence();
     float* w_m = reinterpret_cast<float*>(stages);  // [G][np]: m, then the weights
     float* w_l = w_m + G * np;                      // [G][np]
     float* h_M = w_l + G * np;                      // [G]

@@ -224,10 +224,11 @@ extern "C" int pkv_seq_block_table(const pkv_pool* pool, int64_t seq_id, int32_t
 
 extern "C" int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t* seq_ids,
                                      int32_t* out, int max_blocks_per_seq, int32_t fill,
-                                     int32_t* context_lens) {
+                                     int32_t* context_lens, int32_t* max_context_len) {
     PKV_REQUIRE(pool && n >= 0 && max_blocks_per_seq >= 0 &&
                     (n == 0 || (seq_ids && (out || max_blocks_per_seq == 0))),
                 PKV_ERR_INVALID, "pkv_pool_block_tables: bad argument");
+    int64_t longest = 0;
     for (int i = 0; i < n; ++i) {
         auto it = pool->seqs.find(seq_ids[i]);
         PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
@@ -240,7 +241,9 @@ extern "C" int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t*
         std::copy(t.begin(), t.end(), row);
         std::fill(row + t.size(), row + max_blocks_per_seq, fill);
         if (context_lens) context_lens[i] = (int32_t)it->second.tokens;
+        longest = std::max<int64_t>(longest, it->second.tokens);
     }
+    if (max_context_len) *max_context_len = (int32_t)longest;
     return PKV_OK;
 }
 

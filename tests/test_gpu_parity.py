@@ -313,3 +313,22 @@ def test_shared_prefix_small_workload(cuda_device):
     from tests.shared_prefix import run_shared_prefix
 
     run_shared_prefix(W.SHARED_PREFIX_SMALL, cuda_device, partition_size=32, check_all=True)
+
+
+def test_bounded_wait_expires_and_reports(cuda_device):
+    """The failure path of every mbarrier wait: a wait on a barrier nothing
+    completes gives up after its limit and reports a timeout; the context
+    stays usable afterwards."""
+    import time
+
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    t0 = time.perf_counter()
+    _abi.pkv_selftest_bounded_wait(err, 20000)  # 20 ms
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 >= 0.019
+    assert err.tolist() == [_abi.PKV_DEVERR_TIMEOUT, 0]
+    # the context still runs kernels correctly
+    p = paged_problem(40, 8, 2, 64, 16, [33, 70], "bf16")
+    got = gpu_decode(p, 2, 16, 0.125, 0, cuda_device)
+    want = oracle_decode(p, 2, 16, 0.125, "bf16")
+    assert tolerance_violation(got, want, ATOL, RTOL) <= 0
