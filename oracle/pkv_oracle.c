@@ -349,3 +349,162 @@ int pkv_oracle_max_threads(void) {
     return 1;
 #endif
 }
+
+/* ======================================================================== */
+/* FP8 (e4m3) KV cache with a scale per (block, KV head)                     */
+/* ======================================================================== */
+/*
+ * "Paged KV" wiki page, section 局限性: some KV quantisation schemes, such as
+ * FP8 with a scale per block, tie the block size to the quantisation.  The
+ * reading taken here: K and V are stored as e4m3 codes (1 sign, 4 exponent
+ * bits with bias 7, 3 fraction bits; no infinities; S.1111.111 is NaN;
+ * largest finite 448), and every (physical block, KV head) has one fp32 scale
+ * for K and one for V: value = decode(code) * scale.  A value is stored as
+ * the e4m3 code nearest to (fp32) x / scale, ties to an even code, with
+ * magnitudes beyond 448 saturating to 448.
+ */
+
+double pkv_oracle_e4m3_to_f64(uint8_t code) {
+    int sign = (code >> 7) & 1;
+    int expo = (code >> 3) & 0xf;
+    int frac = code & 0x7;
+    double mag;
+    if (expo == 0xf && frac == 0x7) {
+        mag = NAN;
+    } else if (expo == 0) {
+        mag = ldexp((double)frac, -9);               /* zero or subnormal */
+    } else {
+        mag = ldexp((double)(8 + frac), expo - 10);  /* (1 + f/8) 2^(e-7) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* Nearest e4m3 code by exhaustive search over the 127 finite magnitudes. */
+uint8_t pkv_oracle_f32_to_e4m3_sat(float x) {
+    if (x != x) return 0x7f;
+    const double a = fabs((double)x);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        const double err = fabs(pkv_oracle_e4m3_to_f64((uint8_t)c) - a);
+        /* strictly better, or as good with an even code (ties to even) */
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(best | (signbit(x) ? 0x80 : 0));  /* -0 keeps its sign */
+}
+
+static double fp8_elem(const uint8_t* cache, int64_t idx, const float* scales,
+                       int64_t scale_idx) {
+    return pkv_oracle_e4m3_to_f64(cache[idx]) * (double)scales[scale_idx];
+}
+
+/* Slot write into e4m3 caches: token t, KV head h goes to block b = slot /
+ * block_size with the code of (float)x / scale[b * Hkv + h]. */
+int pkv_oracle_write_slots_fp8(uint8_t* key_cache, uint8_t* value_cache,
+                               const uint16_t* key, const uint16_t* value,
+                               const int64_t* slot_mapping, int num_tokens,
+                               int num_blocks, int block_size, int num_kv_heads,
+                               int head_dim, int64_t block_stride,
+                               const float* k_scale, const float* v_scale,
+                               int dtype) {
+    const int Hkv = num_kv_heads, D = head_dim;
+    const int64_t nslots = (int64_t)num_blocks * block_size;
+    if (num_tokens < 0 || block_size <= 0 || Hkv <= 0 || D <= 0) return -1;
+    if (block_stride < (int64_t)block_size * Hkv * D) return -1;
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t st = slot_mapping[t];
+        if (st < 0) continue;
+        if (st >= nslots) return -1;
+        for (int u = 0; u < t; ++u)
+            if (slot_mapping[u] == st) return -1;
+    }
+    for (int t = 0; t < num_tokens; ++t) {
+        int64_t st = slot_mapping[t];
+        if (st < 0) continue;
+        int64_t b = st / block_size, o = st % block_size;
+        for (int h = 0; h < Hkv; ++h) {
+            const float ks = k_scale[b * Hkv + h], vs = v_scale[b * Hkv + h];
+            const int64_t dst = slot_offset(b, o, h, Hkv, D, block_stride);
+            const int64_t src = ((int64_t)t * Hkv + h) * D;
+            for (int d = 0; d < D; ++d) {
+                const float kx = (float)widen(key[src + d], dtype);
+                const float vx = (float)widen(value[src + d], dtype);
+                key_cache[dst + d] = pkv_oracle_f32_to_e4m3_sat(kx / ks);
+                value_cache[dst + d] = pkv_oracle_f32_to_e4m3_sat(vx / vs);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Paged decode attention over e4m3 caches: the same definition as
+ * pkv_oracle_decode_attention with K and V dequantised exactly in fp64. */
+int pkv_oracle_decode_attention_fp8(double* out, const uint16_t* query,
+                                    const uint8_t* key_cache,
+                                    const uint8_t* value_cache,
+                                    const float* k_scale, const float* v_scale,
+                                    const int32_t* block_tables,
+                                    int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int num_blocks, int block_size,
+                                    int64_t block_stride, double scale, int dtype,
+                                    int num_threads) {
+    const int S = num_seqs, Hq = num_q_heads, Hkv = num_kv_heads, D = head_dim;
+    const int MB = max_blocks_per_seq, bs = block_size;
+    if (check_shapes(S, Hq, Hkv, D, num_blocks, bs, block_stride, MB)) return -1;
+    int max_len = 0;
+    for (int s = 0; s < S; ++s) {
+        if (check_seq(block_tables, MB, context_lens, s, num_blocks, bs)) return -1;
+        if (context_lens[s] > max_len) max_len = context_lens[s];
+    }
+    const int G = Hq / Hkv;
+    int bad = 0;
+#ifdef _OPENMP
+    omp_set_num_threads(num_threads > 0 ? num_threads : omp_get_num_procs());
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel reduction(| : bad)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+        if (!scores) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t sh = 0; sh < (int64_t)S * Hq; ++sh) {
+            if (!scores) continue;
+            int s = (int)(sh / Hq), h = (int)(sh % Hq);
+            int kvh = h / G;
+            const int32_t* table = block_tables + (int64_t)s * MB;
+            const uint16_t* q = query + sh * D;
+            double* o = out + sh * D;
+            int L = context_lens[s];
+            double m = -INFINITY;
+            for (int t = 0; t < L; ++t) {
+                int64_t b = table[t / bs], off = t % bs;
+                int64_t base = slot_offset(b, off, kvh, Hkv, D, block_stride);
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += widen(q[d], dtype) * fp8_elem(key_cache, base + d, k_scale, b * Hkv + kvh);
+                scores[t] = scale * dot;
+                if (scores[t] > m) m = scores[t];
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            for (int t = 0; t < L; ++t) {
+                double w = exp(scores[t] - m);
+                l += w;
+                int64_t b = table[t / bs], off = t % bs;
+                int64_t base = slot_offset(b, off, kvh, Hkv, D, block_stride);
+                for (int d = 0; d < D; ++d)
+                    o[d] += w * fp8_elem(value_cache, base + d, v_scale, b * Hkv + kvh);
+            }
+            if (L > 0)
+                for (int d = 0; d < D; ++d) o[d] /= l;
+        }
+        free(scores);
+    }
+    return bad ? -1 : 0;
+}

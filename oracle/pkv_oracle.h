@@ -60,6 +60,27 @@ int64_t pkv_oracle_block_bytes(int block_size, int num_kv_heads, int head_dim,
 
 int pkv_oracle_max_threads(void);
 
+double pkv_oracle_e4m3_to_f64(uint8_t code);
+uint8_t pkv_oracle_f32_to_e4m3_sat(float x);
+int pkv_oracle_write_slots_fp8(uint8_t* key_cache, uint8_t* value_cache,
+                               const uint16_t* key, const uint16_t* value,
+                               const int64_t* slot_mapping, int num_tokens,
+                               int num_blocks, int block_size, int num_kv_heads,
+                               int head_dim, int64_t block_stride,
+                               const float* k_scale, const float* v_scale,
+                               int dtype);
+int pkv_oracle_decode_attention_fp8(double* out, const uint16_t* query,
+                                    const uint8_t* key_cache,
+                                    const uint8_t* value_cache,
+                                    const float* k_scale, const float* v_scale,
+                                    const int32_t* block_tables,
+                                    int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int num_blocks, int block_size,
+                                    int64_t block_stride, double scale, int dtype,
+                                    int num_threads);
+
 #ifdef __cplusplus
 }
 #endif

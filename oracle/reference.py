@@ -42,6 +42,15 @@ def lib():
         L.pkv_oracle_block_bytes.argtypes = [i, i, i, i, i]
         L.pkv_oracle_block_bytes.restype = i64
         L.pkv_oracle_max_threads.argtypes = []
+        L.pkv_oracle_e4m3_to_f64.argtypes = [C.c_uint8]
+        L.pkv_oracle_e4m3_to_f64.restype = d
+        L.pkv_oracle_f32_to_e4m3_sat.argtypes = [C.c_float]
+        L.pkv_oracle_f32_to_e4m3_sat.restype = C.c_uint8
+        L.pkv_oracle_write_slots_fp8.argtypes = [p, p, p, p, p, i, i, i, i, i, i64, p, p, i]
+        L.pkv_oracle_write_slots_fp8.restype = i
+        L.pkv_oracle_decode_attention_fp8.argtypes = [p, p, p, p, p, p, p, i, p, i, i, i, i, i,
+                                                      i, i64, d, i, i]
+        L.pkv_oracle_decode_attention_fp8.restype = i
         for name in ("pkv_oracle_decode_attention", "pkv_oracle_decode_partials",
                      "pkv_oracle_merge_partials", "pkv_oracle_write_slots",
                      "pkv_oracle_copy_blocks", "pkv_oracle_max_threads"):
@@ -219,3 +228,75 @@ def block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):
 
 def max_threads():
     return int(lib().pkv_oracle_max_threads())
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) caches with a float32 scale per (block, KV head)
+# ---------------------------------------------------------------------------
+def _u8(x):
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.uint8) if x.dtype == np.uint8 else \
+            np.ascontiguousarray(x).view(np.uint8)
+    import torch
+
+    return x.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
+def _f32(x):
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.float32)
+    return x.detach().cpu().contiguous().float().numpy()
+
+
+def e4m3_to_f64(code):
+    return lib().pkv_oracle_e4m3_to_f64(int(code))
+
+
+def f32_to_e4m3(x):
+    return int(lib().pkv_oracle_f32_to_e4m3_sat(float(x)))
+
+
+def write_slots_fp8(key_cache, value_cache, key, value, slot_mapping, block_size,
+                    num_kv_heads, k_scale, v_scale, dtype, block_stride=None):
+    """e4m3 caches (uint8) after writing 16-bit K/V rows quantised with the
+    scale of their (block, KV head)."""
+    kc = _u8(key_cache).copy()
+    vc = _u8(value_cache).copy()
+    k = bits(key)
+    v = bits(value)
+    slots = _i64(slot_mapping)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    D = k.shape[-1]
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    rc = lib().pkv_oracle_write_slots_fp8(_ptr(kc), _ptr(vc), _ptr(k), _ptr(v), _ptr(slots),
+                                          slots.shape[0], NB, block_size, num_kv_heads, D,
+                                          block_stride, _ptr(ks), _ptr(vs), _dtype_code(dtype))
+    _check(rc, "write_slots_fp8")
+    return kc, vc
+
+
+def decode_attention_fp8(query, key_cache, value_cache, k_scale, v_scale, block_tables,
+                         context_lens, scale, dtype, num_kv_heads, block_size,
+                         block_stride=None, num_threads=0):
+    """Paged decode attention in fp64 over e4m3 caches with per-(block, KV
+    head) scales; query is 16-bit ([S, Hq, D])."""
+    q = bits(query)
+    kc = _u8(key_cache)
+    vc = _u8(value_cache)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    S, Hq, D = q.shape
+    tables = _i32(block_tables)
+    lens = _i32(context_lens)
+    MB = tables.shape[1] if tables.ndim == 2 else 0
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    rc = lib().pkv_oracle_decode_attention_fp8(
+        _ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(tables), MB,
+        _ptr(lens), S, Hq, num_kv_heads, D, NB, block_size, block_stride, float(scale),
+        _dtype_code(dtype), int(num_threads))
+    _check(rc, "decode_attention_fp8")
+    return out
