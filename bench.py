@@ -11,6 +11,11 @@ heads, head_dim 128, block size 16, context lengths U[128, 2048], bf16,
 blocks scattered over a pool of 1.1x the blocks needed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pkv|reference]
+                    [--workload NAME] [--kv-dtype auto|fp8]
+
+With --kv-dtype fp8 the cache holds e4m3 codes with an fp32 scale per
+(block, KV head) and the step calls the _fp8 entry points; queries, new rows
+and outputs keep the workload's 16-bit type.
 
 `value` is effective GB/s of algorithmic bytes (every context token's K and V
 read once, plus queries, outputs, table rows, the slot write and any
@@ -36,7 +41,10 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "paged decode attention effective KV GB/s (% of HBM peak); decode tok/s"
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md")
+PROFILE_TRAFFIC = {
+    False: os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md"),
+    True: os.path.join(ROOT, "profiles", "decode_attention_fp8_7b_s256.md"),
+}
 
 
 def parse_args():
@@ -50,6 +58,8 @@ def parse_args():
                     help="tokens per split-K partition (0: one pass; -1: the workload's)")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="profiling only: run the workload's first N sequences")
+    ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
+                    help="fp8: e4m3 cache with a scale per (block, KV head)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -100,15 +110,18 @@ def sum_over_ranks(x, world, device):
 # ---------------------------------------------------------------------------
 # byte accounting (algorithmic bytes, not DRAM traffic)
 # ---------------------------------------------------------------------------
-def decode_bytes(spec, lens, partition_size):
+def decode_bytes(spec, lens, partition_size, fp8=False):
     """Bytes paged decode attention must move for one step: each context
-    token's K and V once, queries, outputs, the table entries it follows,
-    the context lengths, and with split-K the fp32 partials written and read
-    back by the merge."""
+    token's K and V once (one byte per value for an e4m3 cache, plus the K
+    and V scale of each (block, KV head) visited), queries, outputs, the
+    table entries it follows, the context lengths, and with split-K the fp32
+    partials written and read back by the merge."""
     dtb = 2
     S, Hq, Hkv, D, bs = (spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
                          spec.block_size)
-    kv = sum(lens) * Hkv * D * 2 * dtb
+    kv = sum(lens) * Hkv * D * 2 * (1 if fp8 else dtb)
+    if fp8:
+        kv += sum(-(-L // bs) for L in lens) * Hkv * 2 * 4
     qo = 2 * S * Hq * D * dtb
     table = sum(-(-L // bs) for L in lens) * 4 + S * 4
     ws = 0
@@ -119,13 +132,23 @@ def decode_bytes(spec, lens, partition_size):
     return kv + qo + table + ws
 
 
-def write_bytes(spec, num_tokens):
-    """Slot write: new K and V rows read and written, plus the slots."""
-    return num_tokens * spec.num_kv_heads * spec.head_dim * 2 * 2 * 2 + num_tokens * 8
+def write_bytes(spec, num_tokens, fp8=False):
+    """Slot write: new K and V rows read and written (written as one byte per
+    value, after reading the row's scale, for an e4m3 cache), plus the
+    slots."""
+    row = num_tokens * spec.num_kv_heads * spec.head_dim * 2  # K and V values
+    if fp8:
+        return row * (2 + 1) + num_tokens * spec.num_kv_heads * 2 * 4 + num_tokens * 8
+    return row * 2 * 2 + num_tokens * 8
 
 
-def copy_bytes(spec, num_pairs):
-    return num_pairs * spec.block_size * spec.num_kv_heads * spec.head_dim * 2 * 2 * 2
+def copy_bytes(spec, num_pairs, fp8=False):
+    """Block copy: each pair's K and V blocks read and written (and their
+    scales for an e4m3 cache)."""
+    vals = num_pairs * spec.block_size * spec.num_kv_heads * spec.head_dim * 2 * 2
+    if fp8:
+        return vals + num_pairs * spec.num_kv_heads * 2 * 4 * 2
+    return vals * 2
 
 
 # ---------------------------------------------------------------------------
@@ -190,12 +213,12 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def profiled_traffic(source_digest):
+def profiled_traffic(source_digest, fp8=False):
     """DRAM bytes per launch of the decode kernel from the committed ncu
     summary, or None when that summary is missing or was taken on other
     kernel source."""
     try:
-        with open(PROFILE_TRAFFIC) as f:
+        with open(PROFILE_TRAFFIC[fp8]) as f:
             text = f.read()
     except OSError:
         return None
@@ -226,9 +249,10 @@ def kernel_source_digest():
 # ---------------------------------------------------------------------------
 # CPU oracle timing (baseline, not a target)
 # ---------------------------------------------------------------------------
-def oracle_sample_problem(spec, lens, seed):
+def oracle_sample_problem(spec, lens, seed, fp8=False):
     """A compact copy of the workload's first sequences for the CPU oracle:
-    the same lengths and shapes, scattered over a small pool."""
+    the same lengths and shapes, scattered over a small pool (e4m3 codes and
+    per-(block, KV head) scales for an e4m3 cache)."""
     import numpy as np
 
     g = torch.Generator().manual_seed(seed)
@@ -245,24 +269,44 @@ def oracle_sample_problem(spec, lens, seed):
             i += 1
     dt = spec.torch_dtype
     shape = (nb, bs, spec.num_kv_heads, spec.head_dim)
-    kc = torch.randn(shape, generator=g).to(dt)
-    vc = torch.randn(shape, generator=g).to(dt)
     q = torch.randn(len(lens), spec.num_q_heads, spec.head_dim, generator=g).to(dt)
-    return q, kc, vc, tables, np.asarray(lens, np.int32)
+    prob = dict(q=q, tables=tables, lens=np.asarray(lens, np.int32))
+    if not fp8:
+        prob["kc"] = torch.randn(shape, generator=g).to(dt)
+        prob["vc"] = torch.randn(shape, generator=g).to(dt)
+        return prob
+    for c in ("k", "v"):
+        sc = (0.75 + 0.5 * torch.rand(nb, spec.num_kv_heads, generator=g)) * (4.0 / 448.0)
+        x = (torch.randn(shape, generator=g) / sc[:, None, :, None]).clamp_(-448.0, 448.0)
+        prob[c + "c"] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+        prob[c + "s"] = sc.numpy().astype(np.float32)
+    return prob
 
 
-def time_oracle(spec, lens, target_s):
+def oracle_step(spec, prob, fp8=False):
+    """One decode step of the oracle (all host cores) on a sample problem."""
+    from oracle import reference as ref
+
+    if fp8:
+        return ref.decode_attention_fp8(prob["q"], prob["kc"], prob["vc"], prob["ks"],
+                                        prob["vs"], prob["tables"], prob["lens"], spec.scale,
+                                        spec.dtype, spec.num_kv_heads, spec.block_size)
+    return ref.decode_attention(prob["q"], prob["kc"], prob["vc"], prob["tables"], prob["lens"],
+                                spec.scale, spec.dtype, spec.num_kv_heads, spec.block_size,
+                                num_threads=0)
+
+
+def time_oracle(spec, lens, target_s, fp8=False):
     """Times the fp64 oracle (all host cores) on the first n sequences, n
     grown until one call takes about target_s seconds.  Returns (GB/s,
-    seconds, n, cores)."""
+    seconds, n, reps, cores)."""
     from oracle import reference as ref
 
     n = 1
     while True:
-        q, kc, vc, tables, l = oracle_sample_problem(spec, lens[:n], 7)
+        prob = oracle_sample_problem(spec, lens[:n], 7, fp8)
         t0 = time.perf_counter()
-        ref.decode_attention(q, kc, vc, tables, l, spec.scale, spec.dtype, spec.num_kv_heads,
-                             spec.block_size, num_threads=0)
+        oracle_step(spec, prob, fp8)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * target_s or n >= len(lens):
             break
@@ -271,12 +315,15 @@ def time_oracle(spec, lens, target_s):
     reps, total = 1, dt
     while total < 0.8 * target_s:
         t0 = time.perf_counter()
-        ref.decode_attention(q, kc, vc, tables, l, spec.scale, spec.dtype, spec.num_kv_heads,
-                             spec.block_size, num_threads=0)
+        oracle_step(spec, prob, fp8)
         total += time.perf_counter() - t0
         reps += 1
-    byts = decode_bytes(spec, list(lens[:n]), 0) * reps
+    byts = decode_bytes(spec, list(lens[:n]), 0, fp8) * reps
     return byts / total / 1e9, total, n, reps, ref.max_threads()
+
+
+def workload_name(spec, fp8):
+    return spec.name + ("_kv_e4m3" if fp8 else "")
 
 
 # ---------------------------------------------------------------------------
@@ -290,18 +337,17 @@ def run_reference(args, spec, world, rank):
     gen = torch.Generator("cpu").manual_seed(spec.seed)
     lens = W.draw_lens(spec, gen).tolist()
     per_step = max(0.2, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
-    gbs, dt, n, reps, cores = time_oracle(spec, lens, per_step)
-    q, kc, vc, tables, l = oracle_sample_problem(spec, lens[:n], 11)
-    from oracle import reference as ref
+    fp8 = args.kv_dtype == "fp8"
+    gbs, dt, n, reps, cores = time_oracle(spec, lens, per_step, fp8)
+    prob = oracle_sample_problem(spec, lens[:n], 11, fp8)
 
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        ref.decode_attention(q, kc, vc, tables, l, spec.scale, spec.dtype, spec.num_kv_heads,
-                             spec.block_size, num_threads=0)
+        oracle_step(spec, prob, fp8)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
-    byts = decode_bytes(spec, lens[:n], 0)
+    byts = decode_bytes(spec, lens[:n], 0, fp8)
     value = byts * len(times) / sum(times) / 1e9
     sample = "first %d of %d sequences (all %d query heads), one decode step each" % (
         n, spec.num_seqs, spec.num_q_heads)
@@ -310,8 +356,8 @@ def run_reference(args, spec, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * sum(times) / len(times), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": spec.name, "oracle": "fp64 C oracle, OpenMP over (seq, head)",
-                   "sample": sample},
+        "config": {"workload": workload_name(spec, fp8),
+                   "oracle": "fp64 C oracle, OpenMP over (seq, head)", "sample": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -343,10 +389,18 @@ def run_pkv(args, spec, world, rank, local):
     n_states = 16  # decode steps whose metadata is prepared (one block's worth)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 48)
     mb = spec.max_blocks_per_seq + -(-(n_states + e2e_steps + 2) // bs)
+    fp8 = args.kv_dtype == "fp8"
     cache = PagedKVCache(nb, bs, Hq, Hkv, D, spec.torch_dtype, dev, mb, P,
-                         free_order=order.tolist(), scale=spec.scale)
-    W.fill_device_cache_(cache.key_cache, spec.seed * 10 + 2 * rank)
-    W.fill_device_cache_(cache.value_cache, spec.seed * 10 + 2 * rank + 1)
+                         free_order=order.tolist(), scale=spec.scale,
+                         kv_dtype=torch.uint8 if fp8 else None)
+    if fp8:
+        W.fill_device_scales_(cache.k_scale, spec.seed * 10 + 2 * rank + 5)
+        W.fill_device_scales_(cache.v_scale, spec.seed * 10 + 2 * rank + 6)
+        W.fill_device_cache_fp8_(cache.key_cache, cache.k_scale, spec.seed * 10 + 2 * rank)
+        W.fill_device_cache_fp8_(cache.value_cache, cache.v_scale, spec.seed * 10 + 2 * rank + 1)
+    else:
+        W.fill_device_cache_(cache.key_cache, spec.seed * 10 + 2 * rank)
+        W.fill_device_cache_(cache.value_cache, spec.seed * 10 + 2 * rank + 1)
     ids = list(range(S))
     for s in ids:
         cache.add_sequence(s, lens0[s] - 1)
@@ -369,9 +423,9 @@ def run_pkv(args, spec, world, rank, local):
             q=torch.randn((S, Hq, D), generator=dgen, device=dev).to(dt),
             k=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
             v=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
-            bytes_decode=decode_bytes(spec, lens, P),
-            bytes_step=decode_bytes(spec, lens, P) + write_bytes(spec, S) +
-            copy_bytes(spec, npairs), npairs=npairs, lens_sum=sum(lens)))
+            bytes_decode=decode_bytes(spec, lens, P, fp8),
+            bytes_step=decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
+            copy_bytes(spec, npairs, fp8), npairs=npairs, lens_sum=sum(lens)))
     max_len_all = max(s["max_len"] for s in states)
     ws_bytes = _abi.pkv_decode_workspace_bytes(S, Hq, max_len_all, P, D)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev) if ws_bytes else None
@@ -379,19 +433,35 @@ def run_pkv(args, spec, world, rank, local):
     err = cache.dev_error
     kc, vc = cache.key_cache, cache.value_cache
 
+    ks, vs = cache.k_scale, cache.v_scale
+
     def step(state, ev=None):
         if state["npairs"]:
-            _abi.pkv_copy_blocks(kc, vc, state["pairs"], dev_error=err, stream=stream)
-        _abi.pkv_write_slots(state["k"], state["v"], kc, vc, state["slots"], dev_error=err,
-                             stream=stream)
+            if fp8:
+                _abi.pkv_copy_blocks_fp8(kc, vc, ks, vs, state["pairs"], dev_error=err,
+                                         stream=stream)
+            else:
+                _abi.pkv_copy_blocks(kc, vc, state["pairs"], dev_error=err, stream=stream)
+        if fp8:
+            _abi.pkv_write_slots_fp8(state["k"], state["v"], kc, vc, ks, vs, state["slots"],
+                                     dev_error=err, stream=stream)
+        else:
+            _abi.pkv_write_slots(state["k"], state["v"], kc, vc, state["slots"], dev_error=err,
+                                 stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        _abi.pkv_decode_attention(out, state["q"], kc, vc, state["tables"], state["lens"],
-                                  state["max_len"], spec.scale, P, ws, dev_error=err,
-                                  stream=stream)
+        if fp8:
+            _abi.pkv_decode_attention_fp8(out, state["q"], kc, vc, ks, vs, state["tables"],
+                                          state["lens"], state["max_len"], spec.scale, P, ws,
+                                          dev_error=err, stream=stream)
+        else:
+            _abi.pkv_decode_attention(out, state["q"], kc, vc, state["tables"], state["lens"],
+                                      state["max_len"], spec.scale, P, ws, dev_error=err,
+                                      stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        return (1 if state["npairs"] else 0) + 2
+        # copy-on-write: a bytes kernel, plus a scale kernel for e4m3 caches
+        return (((2 if fp8 else 1) if state["npairs"] else 0)) + 2
 
     for i in range(args.warmup):
         step(states[i % n_states])
@@ -460,8 +530,8 @@ def run_pkv(args, spec, world, rank, local):
                 cache.launch_step(prep, dq, dk, dv, out, stream=stream)
                 hout.copy_(out, non_blocking=True)
                 lens = prep["st"]["h_lens"].tolist()
-                e2e_bytes += (decode_bytes(spec, lens, P) + write_bytes(spec, S) +
-                              copy_bytes(spec, prep["num_pairs"]))
+                e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
+                              copy_bytes(spec, prep["num_pairs"], fp8))
                 h2d = d_in.numel() * 2 + prep["st"]["h"].numel() * 4
                 d2h = hout.numel() * 2
                 if i + 1 < e2e_steps:
@@ -478,27 +548,30 @@ def run_pkv(args, spec, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, secs, n, reps, cores = time_oracle(spec, lens0, 10.0)
+        gbs, secs, n, reps, cores = time_oracle(spec, lens0, 10.0, fp8)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": "first %d of %d sequences (all %d query heads), decode step "
                          "repeated %d times, %.1f s" % (n, S, Hq, reps, secs)}
 
     if rank == 0:
-        traffic = profiled_traffic(kernel_source_digest())
+        traffic = profiled_traffic(kernel_source_digest(), fp8)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if dt == torch.bfloat16 else "f16", "data": "synthetic",
+            "dtype": "e4m3" if fp8 else "bf16" if dt == torch.bfloat16 else "f16",
+            "data": "synthetic",
             "config": {
-                "workload": spec.name, "num_seqs": S, "num_q_heads": Hq, "num_kv_heads": Hkv,
+                "workload": workload_name(spec, fp8), "num_seqs": S, "num_q_heads": Hq, "num_kv_heads": Hkv,
                 "head_dim": D, "block_size": bs, "context_lens": "U[%d,%d]" % (spec.len_lo,
                                                                              spec.len_hi),
                 "pool_blocks": nb, "partition_size": P,
+                "kv_cache": ("e4m3, fp32 scale per (block, KV head)" if fp8 else
+                             "bf16" if dt == torch.bfloat16 else "f16"),
                 "step": "host slot append + slot write + paged decode attention"
                         " (+ copy-on-write copies; split-K partitions merged in-kernel)",
                 "l2": "inputs larger than L2 (%.2f GB of K/V read per step)" % (
-                    states[0]["lens_sum"] * Hkv * D * 4 / 1e9),
+                    states[0]["lens_sum"] * Hkv * D * (2 if fp8 else 4) / 1e9),
                 "states": "%d consecutive decode steps prepared by the host pool, replayed "
                           "cyclically" % n_states},
             "pct_hbm_peak": round(100 * value / (world * peak), 2),

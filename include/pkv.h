@@ -219,6 +219,69 @@ PKV_API int pkv_decode_attention_noalloc(void* out, const void* query, const voi
                                          int32_t* dev_error, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
+/* FP8 (e4m3) caches with a scale per (block, KV head)                     */
+/* ---------------------------------------------------------------------- */
+/*
+ * A quantised cache ("Paged KV" wiki page, 局限性: KV FP8 with a scale per
+ * block).  Each cache holds one byte per value, an OCP e4m3 code (bias 7,
+ * finite up to 448, no infinities, 0x7f/0xff are NaN), in the layout above
+ * with block_stride counted in BYTES (a multiple of 16).  Block b, KV head h
+ * has one scale per cache, k_scale[b * num_kv_heads + h] and
+ * v_scale[b * num_kv_heads + h] (device fp32, 16-byte aligned, at least
+ * num_blocks * num_kv_heads floats rounded up to a multiple of 4).  A code c
+ * stands for the value e4m3(c) * scale.  Scales are positive and finite.
+ * The caller sets a block's scales before the block's first write and keeps
+ * them while the block holds tokens; the library reads them and copies them
+ * with the block.
+ */
+
+/*
+ * pkv_write_slots into an e4m3 cache: value x of token t (f16 or bf16 per
+ * dtype, the type of key/value) is stored as the e4m3 code nearest to the
+ * fp32 quotient x / scale (round to nearest, ties to the even code; beyond
+ * 448 in magnitude it saturates to +-448; NaN stays NaN), scale being the
+ * destination block's scale for that KV head.  Slot rules, alignment and
+ * errors are those of pkv_write_slots; num_kv_heads * head_dim a multiple
+ * of 8.
+ */
+PKV_API int pkv_write_slots_fp8(const void* key, const void* value, void* key_cache,
+                                void* value_cache, const float* k_scale, const float* v_scale,
+                                const int64_t* slot_mapping, int num_tokens, int num_blocks,
+                                int block_size, int num_kv_heads, int head_dim,
+                                int64_t block_stride, pkv_dtype dtype, int32_t* dev_error,
+                                cudaStream_t stream);
+
+/*
+ * pkv_copy_blocks for e4m3 caches: block dst of both caches becomes a copy of
+ * block src, bytes and scales (k_scale and v_scale rows of dst take src's).
+ * Pair rules and errors are those of pkv_copy_blocks; the block's bytes
+ * (block_size * num_kv_heads * head_dim) a multiple of 16.
+ */
+PKV_API int pkv_copy_blocks_fp8(void* key_cache, void* value_cache, float* k_scale,
+                                float* v_scale, const int32_t* block_pairs, int num_pairs,
+                                int num_blocks, int block_size, int num_kv_heads, int head_dim,
+                                int64_t block_stride, int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * pkv_decode_attention over e4m3 caches: K_t and V_t are the dequantised
+ * rows (code * scale of the token's block and KV head); query and out keep
+ * dtype (f16 or bf16).  Built for head_dim 128 and block_size a multiple of
+ * 16 (the kernel's tile is 16 slots of one block); the other arguments,
+ * the workspace (pkv_decode_workspace_bytes) and errors are those of
+ * pkv_decode_attention.
+ */
+PKV_API int pkv_decode_attention_fp8(void* out, const void* query, const void* key_cache,
+                                     const void* value_cache, const float* k_scale,
+                                     const float* v_scale, const int32_t* block_tables,
+                                     int max_blocks_per_seq, const int32_t* context_lens,
+                                     int num_seqs, int max_context_len, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int num_blocks,
+                                     int block_size, int64_t block_stride, float scale,
+                                     int partition_size, void* workspace,
+                                     size_t workspace_bytes, pkv_dtype dtype,
+                                     int32_t* dev_error, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* Host block pool (allocator)                                             */
 /* ---------------------------------------------------------------------- */
 /*

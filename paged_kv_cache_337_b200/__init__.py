@@ -11,9 +11,14 @@ raises if it has not been built.
 from ._abi import (  # noqa: F401
     BlockPool,
     PkvError,
+    fp8_scales,
     pkv_block_bytes,
     pkv_copy_blocks,
+    pkv_copy_blocks_fp8,
     pkv_decode_attention,
+    pkv_decode_attention_fp8,
+    pkv_decode_attention_noalloc,
     pkv_decode_workspace_bytes,
     pkv_write_slots,
+    pkv_write_slots_fp8,
 )

@@ -43,6 +43,11 @@ SIGNATURES = {
                                   _i64, _f, _i, _p, _sz, _i, _p, _p]),
     "pkv_decode_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
                                           _i, _i64, _f, _i, _i, _p, _p]),
+    "pkv_write_slots_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p,
+                                 _p]),
+    "pkv_copy_blocks_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _p, _p]),
+    "pkv_decode_attention_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i,
+                                      _i, _i, _i64, _f, _i, _p, _sz, _i, _p, _p]),
     "pkv_pool_create": (_i, [_i, _i, _p, C.POINTER(_p)]),
     "pkv_pool_destroy": (None, [_p]),
     "pkv_seq_add": (_i, [_p, _i64, _i]),
@@ -257,6 +262,103 @@ def pkv_decode_attention_noalloc(out, query, key_cache, value_cache, block_table
         bstride, float(scale), int(partition_size), _dtype(query), _ptr(dev_error),
         _stream(stream, query.device))
     _check(st, "pkv_decode_attention_noalloc")
+
+
+# ---------------------------------------------------------------------------
+# FP8 (e4m3) caches with a scale per (block, KV head)
+# ---------------------------------------------------------------------------
+_FP8_CACHE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def fp8_scales(num_blocks, num_kv_heads, device, fill=1.0):
+    """A [num_blocks, num_kv_heads] fp32 scale table whose storage is padded
+    to a multiple of 4 floats (the kernels fetch scales 16 bytes at a time)."""
+    n = num_blocks * num_kv_heads
+    buf = torch.full(((n + 3) // 4 * 4,), fill, dtype=torch.float32, device=device)
+    return buf[:n].view(num_blocks, num_kv_heads)
+
+
+def _fp8_geometry(name, key_cache, value_cache, k_scale, v_scale):
+    for c in (key_cache, value_cache):
+        if c.dtype not in _FP8_CACHE_DTYPES:
+            raise ValueError("%s: caches must be uint8 or float8_e4m3fn, got %s" % (name, c.dtype))
+    geom = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != geom:
+        raise ValueError("key_cache and value_cache differ in geometry")
+    nb, _, hkv, _, _ = geom
+    need = (nb * hkv + 3) // 4 * 4
+    for sc in (k_scale, v_scale):
+        _need(sc, torch.float32, "scales")
+        if sc.numel() != nb * hkv:
+            raise ValueError("%s: scales must hold num_blocks * num_kv_heads floats" % name)
+        if sc.untyped_storage().nbytes() < (sc.storage_offset() + need) * 4:
+            raise ValueError("%s: scale storage must be padded to a multiple of 4 floats "
+                             "(use fp8_scales)" % name)
+    return geom
+
+
+def pkv_write_slots_fp8(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping,
+                        dev_error=None, stream=None):
+    """Quantise token rows key/value [T, Hkv, D] (f16/bf16) to e4m3 with the
+    destination block's scale and write them into their slots."""
+    _on_device("pkv_write_slots_fp8", key, value, key_cache, value_cache, k_scale, v_scale,
+               slot_mapping, dev_error)
+    nb, bs, hkv, d, bstride = _fp8_geometry("pkv_write_slots_fp8", key_cache, value_cache,
+                                            k_scale, v_scale)
+    _need(slot_mapping, torch.int64, "slot_mapping")
+    _need(key, key.dtype, "key")
+    _need(value, key.dtype, "value")
+    T = slot_mapping.numel()
+    if key.shape != (T, hkv, d) or value.shape != (T, hkv, d):
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim]")
+    st = lib().pkv_write_slots_fp8(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
+                                   _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping), T, nb, bs,
+                                   hkv, d, bstride, _dtype(key), _ptr(dev_error),
+                                   _stream(stream, key_cache.device))
+    _check(st, "pkv_write_slots_fp8")
+
+
+def pkv_copy_blocks_fp8(key_cache, value_cache, k_scale, v_scale, block_pairs, dev_error=None,
+                        stream=None):
+    """Copy whole e4m3 blocks and their scales for each (src, dst) row of
+    int32 block_pairs [n, 2]."""
+    _on_device("pkv_copy_blocks_fp8", key_cache, value_cache, k_scale, v_scale, block_pairs,
+               dev_error)
+    nb, bs, hkv, d, bstride = _fp8_geometry("pkv_copy_blocks_fp8", key_cache, value_cache,
+                                            k_scale, v_scale)
+    _need(block_pairs, torch.int32, "block_pairs")
+    n = block_pairs.numel() // 2
+    st = lib().pkv_copy_blocks_fp8(_ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+                                   _ptr(v_scale), _ptr(block_pairs), n, nb, bs, hkv, d, bstride,
+                                   _ptr(dev_error), _stream(stream, key_cache.device))
+    _check(st, "pkv_copy_blocks_fp8")
+
+
+def pkv_decode_attention_fp8(out, query, key_cache, value_cache, k_scale, v_scale,
+                             block_tables, context_lens, max_context_len, scale,
+                             partition_size=0, workspace=None, dev_error=None, stream=None):
+    """pkv_decode_attention over e4m3 caches with per-(block, KV head)
+    scales; query/out stay f16 or bf16."""
+    _on_device("pkv_decode_attention_fp8", out, query, key_cache, value_cache, k_scale, v_scale,
+               block_tables, context_lens, workspace, dev_error)
+    nb, bs, hkv, d, bstride = _fp8_geometry("pkv_decode_attention_fp8", key_cache, value_cache,
+                                            k_scale, v_scale)
+    S, hq, dq = query.shape
+    if dq != d or out.shape != query.shape:
+        raise ValueError("query/out must be [num_seqs, num_q_heads, head_dim]")
+    _need(query, query.dtype, "query")
+    _need(out, query.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
+        raise ValueError("block_tables must be [num_seqs, max_blocks] and context_lens [num_seqs]")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().pkv_decode_attention_fp8(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+        int(max_context_len), hq, hkv, d, nb, bs, bstride, float(scale), int(partition_size),
+        _ptr(workspace), ws_bytes, _dtype(query), _ptr(dev_error), _stream(stream, query.device))
+    _check(st, "pkv_decode_attention_fp8")
 
 
 def pkv_selftest_bounded_wait(dev_error, limit_us, stream=None):

@@ -12,6 +12,10 @@ A decode step for a batch of sequences ("Paged KV" wiki page, 实现原理 /
 4. decode attention runs over every sequence's blocks through its Block
    Table (``pkv_decode_attention``; split-K with a merge for long contexts).
 
+With an e4m3 cache ("Paged KV" wiki page, 局限性: KV FP8 with a scale per
+block) the three device calls are their ``_fp8`` forms, which also copy and
+read the per-(block, KV head) scales.
+
 Steps 2-4 are launched on one stream; the metadata of step 1 travels to the
 device through pinned host staging buffers.  All arithmetic is in the
 library; this module only moves arguments.
@@ -24,7 +28,12 @@ from . import _abi
 class PagedKVCache:
     def __init__(self, num_blocks, block_size, num_q_heads, num_kv_heads, head_dim, dtype,
                  device, max_blocks_per_seq, partition_size=0, free_order=None,
-                 key_cache=None, value_cache=None, scale=None):
+                 key_cache=None, value_cache=None, scale=None, kv_dtype=None, kv_scale=1.0):
+        """dtype is the type of queries, new K/V rows and outputs (f16 or
+        bf16).  kv_dtype torch.uint8 (or torch.float8_e4m3fn) stores the
+        cache as e4m3 codes with a scale per (block, KV head) in k_scale /
+        v_scale ([num_blocks, num_kv_heads] fp32, every entry kv_scale until
+        the caller sets them); None stores it in dtype."""
         self.num_blocks = num_blocks
         self.block_size = block_size
         self.num_q_heads = num_q_heads
@@ -36,17 +45,23 @@ class PagedKVCache:
         self.partition_size = partition_size
         self.scale = scale if scale is not None else 1.0 / (head_dim ** 0.5)
         shape = (num_blocks, block_size, num_kv_heads, head_dim)
+        kv_dtype = dtype if kv_dtype is None else kv_dtype
+        self.fp8 = kv_dtype in (torch.uint8, torch.float8_e4m3fn)
         self.key_cache = key_cache if key_cache is not None else torch.empty(
-            shape, dtype=dtype, device=self.device)
+            shape, dtype=kv_dtype, device=self.device)
         self.value_cache = value_cache if value_cache is not None else torch.empty(
-            shape, dtype=dtype, device=self.device)
+            shape, dtype=kv_dtype, device=self.device)
+        self.k_scale = self.v_scale = None
+        if self.fp8:
+            self.k_scale = _abi.fp8_scales(num_blocks, num_kv_heads, self.device, kv_scale)
+            self.v_scale = _abi.fp8_scales(num_blocks, num_kv_heads, self.device, kv_scale)
         self.pool = _abi.BlockPool(num_blocks, block_size, free_order)
         self.dev_error = torch.zeros(2, dtype=torch.int32, device=self.device)
         self._workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
         self._staging = {}
         self._seen = set()  # tensor signatures the binding has checked
         self._geom = _abi._cache_geometry(self.key_cache)
-        self._dtype_code = _abi._dtype(self.key_cache)
+        self._dtype_code = _abi._DTYPE[dtype]
 
     # -- sequence management (host) ---------------------------------------
     def add_sequence(self, seq_id, num_tokens, key=None, value=None, stream=None):
@@ -56,8 +71,7 @@ class PagedKVCache:
         self.pool.add(seq_id, num_tokens)
         if key is not None and num_tokens > 0:
             slots = self.pool.slot_mapping(seq_id, 0, num_tokens).to(self.device)
-            _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, slots,
-                                 dev_error=self.dev_error, stream=stream)
+            self._write(key, value, slots, stream)
 
     def fork(self, parent, child):
         self.pool.fork(parent, child)
@@ -134,17 +148,12 @@ class PagedKVCache:
         n = prep["num_pairs"]
         max_len = prep["max_len"] if max_len is None else max_len
         if n:
-            _abi.pkv_copy_blocks(self.key_cache, self.value_cache, st["d_pairs"][:n],
-                                 dev_error=self.dev_error, stream=stream)
+            self._copy(st["d_pairs"][:n], stream)
         ws = self.workspace(len(st["ids"]), max_len)
         if not self._checked(query, key, value, out):
             # first use of these tensor shapes: the binding's full checks
-            _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, st["d_slots"],
-                                 dev_error=self.dev_error, stream=stream)
-            _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache,
-                                      st["d_tables"], st["d_lens"], max_len, self.scale,
-                                      self.partition_size, ws, dev_error=self.dev_error,
-                                      stream=stream)
+            self._write(key, value, st["d_slots"], stream)
+            self._attend(out, query, st["d_tables"], st["d_lens"], max_len, ws, stream)
             self._seen.add(self._signature(query, key, value, out))
             return out
         # same shapes, dtypes and device as a call already checked: pass the
@@ -154,18 +163,61 @@ class PagedKVCache:
         kc, vc = self.key_cache, self.value_cache
         nb, bs, hkv, d, bstride = self._geom
         S = query.shape[0]
+        err = self.dev_error.data_ptr()
+        wsp, wsn = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
+        if self.fp8:
+            ks, vs = self.k_scale.data_ptr(), self.v_scale.data_ptr()
+            _abi._check(L.pkv_write_slots_fp8(
+                key.data_ptr(), value.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
+                st["d_slots"].data_ptr(), S, nb, bs, hkv, d, bstride, self._dtype_code, err, sp),
+                "pkv_write_slots_fp8")
+            _abi._check(L.pkv_decode_attention_fp8(
+                out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
+                st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
+                int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
+                int(self.partition_size), wsp, wsn, self._dtype_code, err, sp),
+                "pkv_decode_attention_fp8")
+            return out
         _abi._check(L.pkv_write_slots(key.data_ptr(), value.data_ptr(), kc.data_ptr(),
                                       vc.data_ptr(), st["d_slots"].data_ptr(), S, nb, bs, hkv,
-                                      d, bstride, self._dtype_code, self.dev_error.data_ptr(),
-                                      sp), "pkv_write_slots")
+                                      d, bstride, self._dtype_code, err, sp), "pkv_write_slots")
         _abi._check(L.pkv_decode_attention(
             out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(),
             st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
             int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
-            int(self.partition_size), ws.data_ptr() if ws is not None else None,
-            ws.numel() if ws is not None else 0, self._dtype_code, self.dev_error.data_ptr(),
-            sp), "pkv_decode_attention")
+            int(self.partition_size), wsp, wsn, self._dtype_code, err, sp),
+            "pkv_decode_attention")
         return out
+
+    # -- the three device calls, for either cache type ---------------------
+    def _copy(self, pairs, stream):
+        if self.fp8:
+            _abi.pkv_copy_blocks_fp8(self.key_cache, self.value_cache, self.k_scale,
+                                     self.v_scale, pairs, dev_error=self.dev_error,
+                                     stream=stream)
+        else:
+            _abi.pkv_copy_blocks(self.key_cache, self.value_cache, pairs,
+                                 dev_error=self.dev_error, stream=stream)
+
+    def _write(self, key, value, slots, stream):
+        if self.fp8:
+            _abi.pkv_write_slots_fp8(key, value, self.key_cache, self.value_cache, self.k_scale,
+                                     self.v_scale, slots, dev_error=self.dev_error,
+                                     stream=stream)
+        else:
+            _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, slots,
+                                 dev_error=self.dev_error, stream=stream)
+
+    def _attend(self, out, query, tables, lens, max_len, ws, stream):
+        if self.fp8:
+            _abi.pkv_decode_attention_fp8(out, query, self.key_cache, self.value_cache,
+                                          self.k_scale, self.v_scale, tables, lens, max_len,
+                                          self.scale, self.partition_size, ws,
+                                          dev_error=self.dev_error, stream=stream)
+        else:
+            _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache, tables,
+                                      lens, max_len, self.scale, self.partition_size, ws,
+                                      dev_error=self.dev_error, stream=stream)
 
     def _signature(self, query, key, value, out):
         return tuple((tuple(t.shape), t.dtype, t.device, t.is_contiguous())

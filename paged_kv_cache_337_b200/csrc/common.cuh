@@ -149,6 +149,49 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Untiled bulk copy of `bytes` (a multiple of 16) from global memory into
+// shared memory, completing on `bar`; both addresses 16-byte aligned.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// FP8 (e4m3) conversions, by the hardware cvt instructions
+// ---------------------------------------------------------------------------
+// Two e4m3 codes (low byte first) to two halves (low half first); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+    return r;
+}
+
+// Two floats to two e4m3 codes (lo in the low byte), round to nearest even,
+// magnitudes beyond 448 saturating to 448.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Four e4m3 codes (one 32-bit word, lowest byte first) to four floats.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&v)[4]) {
+    const uint32_t a = e4m3x2_to_f16x2((uint16_t)(w & 0xffffu));
+    const uint32_t b = e4m3x2_to_f16x2((uint16_t)(w >> 16));
+    __half2 ha, hb;
+    memcpy(&ha, &a, 4);
+    memcpy(&hb, &b, 4);
+    const float2 fa = __half22float2(ha), fb = __half22float2(hb);
+    v[0] = fa.x;
+    v[1] = fa.y;
+    v[2] = fb.x;
+    v[3] = fb.y;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

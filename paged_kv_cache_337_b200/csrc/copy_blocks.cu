@@ -82,3 +82,60 @@ extern "C" int pkv_copy_blocks(void* key_cache, void* value_cache, const int32_t
         num_pairs, num_blocks, block_vecs, block_stride / 8, (int)chunks, dev_error);
     return launch_status("pkv_copy_blocks");
 }
+
+// ---------------------------------------------------------------------------
+// Copy-on-write for FP8 (e4m3) caches: the block's bytes (the kernel above,
+// in 16-byte vectors) and its per-KV-head scales.
+// ---------------------------------------------------------------------------
+namespace pkv {
+namespace {
+
+__global__ void copy_scales_kernel(float* __restrict__ k_scale, float* __restrict__ v_scale,
+                                   const int32_t* __restrict__ block_pairs, int num_pairs,
+                                   int num_blocks, int num_kv_heads) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)num_pairs * num_kv_heads) return;
+    const int pair = (int)(i / num_kv_heads), h = (int)(i % num_kv_heads);
+    const int32_t src = __ldg(block_pairs + 2 * pair), dst = __ldg(block_pairs + 2 * pair + 1);
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return;  // reported above
+    k_scale[(int64_t)dst * num_kv_heads + h] = k_scale[(int64_t)src * num_kv_heads + h];
+    v_scale[(int64_t)dst * num_kv_heads + h] = v_scale[(int64_t)src * num_kv_heads + h];
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int pkv_copy_blocks_fp8(void* key_cache, void* value_cache, float* k_scale,
+                                   float* v_scale, const int32_t* block_pairs, int num_pairs,
+                                   int num_blocks, int block_size, int num_kv_heads,
+                                   int head_dim, int64_t block_stride, int32_t* dev_error,
+                                   cudaStream_t stream) {
+    using namespace pkv;
+    PKV_REQUIRE(num_pairs >= 0 && num_blocks >= 0 && block_size > 0 && num_kv_heads > 0 &&
+                    head_dim > 0,
+                PKV_ERR_INVALID, "pkv_copy_blocks_fp8: bad sizes");
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim;
+    PKV_REQUIRE(block_bytes % 16 == 0 && block_stride >= block_bytes && block_stride % 16 == 0,
+                PKV_ERR_INVALID,
+                "pkv_copy_blocks_fp8: block of %lld bytes, stride %lld (multiples of 16)",
+                (long long)block_bytes, (long long)block_stride);
+    if (num_pairs == 0) return PKV_OK;
+    PKV_REQUIRE(key_cache && value_cache && k_scale && v_scale && block_pairs, PKV_ERR_INVALID,
+                "pkv_copy_blocks_fp8: NULL pointer");
+    PKV_REQUIRE(aligned16(key_cache) && aligned16(value_cache), PKV_ERR_INVALID,
+                "pkv_copy_blocks_fp8: caches must be 16-byte aligned");
+    DeviceGuard guard(stream, key_cache);
+    const int64_t block_vecs = block_bytes / 16;
+    const int64_t chunks = (block_vecs + kChunkVecs - 1) / kChunkVecs;
+    const int64_t grid = (int64_t)num_pairs * 2 * chunks;
+    PKV_REQUIRE(grid < (1ll << 31), PKV_ERR_INVALID, "pkv_copy_blocks_fp8: too many pairs");
+    copy_blocks_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(
+        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), block_pairs,
+        num_pairs, num_blocks, block_vecs, block_stride / 16, (int)chunks, dev_error);
+    int st = launch_status("pkv_copy_blocks_fp8");
+    if (st != PKV_OK) return st;
+    const int64_t n = (int64_t)num_pairs * num_kv_heads;
+    copy_scales_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+        k_scale, v_scale, block_pairs, num_pairs, num_blocks, num_kv_heads);
+    return launch_status("pkv_copy_blocks_fp8 (scales)");
+}

@@ -45,6 +45,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <type_traits>
 #include <mutex>
 
 #include "common.cuh"
@@ -87,6 +88,8 @@ struct DecodeParams {
     float* ws_l;
     float* ws_o;
     int32_t* ws_count;  // [S, Hkv]: partitions finished (zeroed before the launch)
+    const float* k_scale;  // e4m3 caches: [num_blocks, Hkv] dequantisation scales
+    const float* v_scale;
     int32_t* dev_error;
     int num_seqs;
     int num_kv_heads;
@@ -126,10 +129,11 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool* b
 // ---------------------------------------------------------------------------
 // Per-warp arithmetic, G == 1: FFMA + shuffles
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, int D, bool FP8 = false>
 struct GemvWarp {
     static constexpr int DV = D / 32;  // dims per lane
     static constexpr int GP = 1;       // heads held (padded)
+    static constexpr bool kMma = false;
     float q[DV], o[DV], m, l;
 
     __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
@@ -156,16 +160,34 @@ struct GemvWarp {
     // lane's DV elements of row r of a swizzled tile
     __device__ __forceinline__ static const uint8_t* at(const uint8_t* tile, int r, int lane) {
         const int d0 = lane * DV;
-        return tile + swz(r, d0 >> 3) + (d0 & 7) * 2;
+        if constexpr (FP8) {
+            // e4m3 tile: one 128-byte row per token, 16-byte chunks swizzled
+            return tile + r * 128 + ((((d0 >> 4) ^ (r & 7))) << 4) + (d0 & 15);
+        } else {
+            return tile + swz(r, d0 >> 3) + (d0 & 7) * 2;
+        }
     }
 
+    // lane's DV cache elements of row r as floats (codes, before the scale)
+    __device__ __forceinline__ static void load_kv(const uint8_t* tile, int r, int lane,
+                                                   float (&v)[DV]) {
+        if constexpr (FP8) {
+            static_assert(DV == 4, "e4m3 caches are built for head_dim 128");
+            e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(at(tile, r, lane)), v);
+        } else {
+            load(at(tile, r, lane), v);
+        }
+    }
+
+    // One tile.  scale_log2 multiplies q.k (with any K dequantisation scale
+    // folded in); vscale multiplies the V rows (1 for 16-bit caches).
     __device__ __forceinline__ void tile(const uint8_t* kt, const uint8_t* vt, int valid,
-                                         float scale_log2, int lane) {
+                                         float scale_log2, int lane, float vscale = 1.f) {
         float part[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             float k[DV];
-            load(at(kt, r, lane), k);
+            load_kv(kt, r, lane, k);
             float acc = 0.f;
 #pragma unroll
             for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
@@ -216,11 +238,12 @@ struct GemvWarp {
         m = m_new;
 #pragma unroll
         for (int j = 0; j < DV; ++j) o[j] *= alpha;
+        const float prv = pr * vscale;
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
-            const float pb = __shfl_sync(kFull, pr, rr * 2);
+            const float pb = __shfl_sync(kFull, prv, rr * 2);
             float v[DV];
-            load(at(vt, rr, lane), v);
+            load_kv(vt, rr, lane, v);
 #pragma unroll
             for (int j = 0; j < DV; ++j) o[j] = fmaf(pb, v[j], o[j]);
         }
@@ -256,9 +279,11 @@ template <typename T, int D, int NT>
 struct MmaWarp {
     static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
     static constexpr int GP = NT * 8;  // heads held (padded)
+    static constexpr bool kMma = true;
     uint32_t qf[KS][NT][2];            // Q^T B-fragments
     float acc[KS][NT][4];              // O^T[d][head]
     float m[NT][2], l[NT][2];          // per lane: heads nt*8 + (lane&3)*2 + {0,1}
+    float vs;                          // acc is in units of this V scale (e4m3 caches)
 
     __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
         const int G = p.group;
@@ -280,6 +305,7 @@ struct MmaWarp {
             }
             m[nt][0] = m[nt][1] = -INFINITY;
             l[nt][0] = l[nt][1] = 0.f;
+            vs = 1.f;
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
@@ -287,8 +313,13 @@ struct MmaWarp {
         }
     }
 
+    // One tile of 16-bit K and V.  scale_log2 multiplies q.k (with any K
+    // dequantisation scale folded in); vscale multiplies the V rows.  P
+    // stays in [0, 1] for the 16-bit fragments; the V scale goes into the
+    // fp32 accumulator instead, which is kept in units of the current
+    // tile's scale (rescaled by old / new scale with the softmax factor).
     __device__ __forceinline__ void tile(const uint8_t* kt, const uint8_t* vt, int valid,
-                                         float scale_log2, int lane) {
+                                         float scale_log2, int lane, float vscale = 1.f) {
         const uint32_t kbase = smem_addr(kt), vbase = smem_addr(vt);
         const int j = lane >> 3;
         // S^T[token][head] = K Q^T over head_dim
@@ -319,6 +350,8 @@ struct MmaWarp {
         // online softmax per head; the lane holds tokens r0, r0 + 8
         const int r0 = lane >> 2;
         const bool v0 = r0 < valid, v1 = r0 + 8 < valid;
+        const float ratio = vscale == vs ? 1.f : vs / vscale;
+        vs = vscale;
         uint32_t pb[NT][2], pl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -340,12 +373,13 @@ struct MmaWarp {
             l[nt][1] = l[nt][1] * a1 + (p1 + p3);
             m[nt][0] = mn0;
             m[nt][1] = mn1;
+            const float c0 = a0 * ratio, c1 = a1 * ratio;
 #pragma unroll
             for (int mt = 0; mt < KS; ++mt) {
-                acc[mt][nt][0] *= a0;
-                acc[mt][nt][1] *= a1;
-                acc[mt][nt][2] *= a0;
-                acc[mt][nt][3] *= a1;
+                acc[mt][nt][0] *= c0;
+                acc[mt][nt][1] *= c1;
+                acc[mt][nt][2] *= c0;
+                acc[mt][nt][3] *= c1;
             }
             // P[token][head] as 16-bit fragments, transposed to P^T
             // B-fragments.  P is split into a rounded high part and the
@@ -405,7 +439,7 @@ struct MmaWarp {
             for (int i = 0; i < 4; ++i) {
                 const int h = nt * 8 + (lane & 3) * 2 + (i & 1);
                 if (h >= G) continue;
-                const float f = M[h] == -INFINITY ? 0.f : exp2f(m[nt][i & 1] - M[h]);
+                const float f = M[h] == -INFINITY ? 0.f : exp2f(m[nt][i & 1] - M[h]) * vs;
 #pragma unroll
                 for (int mt = 0; mt < KS; ++mt) {
                     const int d = mt * 16 + (lane >> 2) + (i >> 1) * 8;
@@ -416,19 +450,76 @@ struct MmaWarp {
 };
 
 // ---------------------------------------------------------------------------
+// Shared-memory plan of one CTA: per warp a ring of stages (the K and V tiles
+// as stored), then, for e4m3 caches on the tensor-core path, a 16-bit copy of
+// the current tile per warp; then the mbarriers, the per-stage
+// dequantisation scales (e4m3) and the partition's table slice.  The ring and
+// the copies are reused by the epilogue once every load has landed.
+// ---------------------------------------------------------------------------
+template <int D, bool FP8, bool MMA>
+struct Plan {
+    static_assert(!FP8 || D == 128, "e4m3 caches are built for head_dim 128");
+    static constexpr int kStages = FP8 ? (MMA ? 2 : 4) : Geom<D>::kStages;
+    static constexpr int kTileBytes = FP8 ? kTile * D : Geom<D>::kKBytes;  // K (or V) as stored
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kScratchBytes = (FP8 && MMA) ? Geom<D>::kStageBytes : 0;
+    static constexpr size_t kRing = (size_t)kWarps * kStages * kStageBytes;
+    static constexpr size_t kEpilogue = kRing + (size_t)kWarps * kScratchBytes;
+    static constexpr size_t kBarOff = kEpilogue;
+    static constexpr size_t kScaleOff = kBarOff + (size_t)kWarps * kStages * 8;
+    static constexpr size_t kTableOff = kScaleOff + (FP8 ? (size_t)kWarps * kStages * 32 : 0);
+    static constexpr uint32_t kTx = kStageBytes + (FP8 ? 32 : 0);  // bytes landing per stage
+};
+
+// Widens an e4m3 tile (16 rows of 128 bytes, swizzled) into the 16-bit tile
+// layout the tensor-core path reads (two 64-column sub-tiles, swizzled).
+// e4m3 values are exact in both fp16 and bf16.
+template <typename T>
+__device__ __forceinline__ void widen_fp8_tile(const uint8_t* raw, uint8_t* dst, int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;  // 128 chunks of 16 codes
+        const int r = c >> 3, ch = c & 7;
+        const uint4 x = *reinterpret_cast<const uint4*>(raw + r * 128 + ((ch ^ (r & 7)) << 4));
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t a = e4m3x2_to_f16x2((uint16_t)(w[k] & 0xffffu));
+            const uint32_t b = e4m3x2_to_f16x2((uint16_t)(w[k] >> 16));
+            if constexpr (std::is_same<T, __half>::value) {
+                h[2 * k] = a;
+                h[2 * k + 1] = b;
+            } else {
+                __half2 ha, hb;
+                memcpy(&ha, &a, 4);
+                memcpy(&hb, &b, 4);
+                const float2 fa = __half22float2(ha), fb = __half22float2(hb);
+                h[2 * k] = Storage<T>::from_float2(fa.x, fa.y);
+                h[2 * k + 1] = Storage<T>::from_float2(fb.x, fb.y);
+            }
+        }
+        *reinterpret_cast<uint4*>(dst + swz(r, 2 * ch)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(dst + swz(r, 2 * ch + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // The attention kernel (single pass or one partition of split-K)
 // ---------------------------------------------------------------------------
-template <typename T, int D, typename Warp>
+template <typename T, int D, typename Warp, bool FP8>
 __global__ void __launch_bounds__(kWarps * 32)
 paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
     using Gm = Geom<D>;
-    constexpr int STAGES = Gm::kStages;
+    using Pl = Plan<D, FP8, Warp::kMma>;
+    constexpr int STAGES = Pl::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* stages = smem;  // [warp][stage][K tile | V tile]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * STAGES * Gm::kStageBytes);
-    int32_t* table = reinterpret_cast<int32_t*>(bars + kWarps * STAGES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Pl::kBarOff);
+    float* scales = reinterpret_cast<float*>(smem + Pl::kScaleOff);  // [warp][stage][K 4 | V 4]
+    int32_t* table = reinterpret_cast<int32_t*>(smem + Pl::kTableOff);
 
     // Flat grid, partition fastest: the partitions of one (sequence, KV
     // head) run side by side, so their merge happens early and in parallel
@@ -456,7 +547,9 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     if (part >= np) return;  // a partition past this sequence's end
 
     uint64_t* my_bars = bars + warp * STAGES;
-    uint8_t* my_stages = stages + warp * STAGES * Gm::kStageBytes;
+    uint8_t* my_stages = stages + warp * STAGES * Pl::kStageBytes;
+    float* my_scales = scales + warp * STAGES * 8;
+    uint8_t* my_wide = smem + Pl::kRing + warp * Pl::kScratchBytes;  // e4m3 + tensor cores
     if (lane == 0) {
 #pragma unroll
         for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
@@ -480,16 +573,31 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     __syncthreads();
 
     // TMA of tile `tile` (K and V, all boxes) into stage `st`; lane 0 only
+    // index of the (block, KV head) scale of a tile; a block id outside the
+    // pool (reported above, its tile read as zeros) takes block 0's
+    auto scale_index = [&](int phys) -> int64_t {
+        return (int64_t)(phys >= 0 && phys < p.num_blocks ? phys : 0) * p.num_kv_heads + kvh;
+    };
     auto issue = [&](int st, int tile) {
         const int t0 = t_begin + tile * kTile;
         const int phys = table[t0 / bs - lb0];
         const int off = t0 % bs;
-        uint8_t* kdst = my_stages + st * Gm::kStageBytes;
-        uint8_t* vdst = kdst + Gm::kKBytes;
-        mbar_arrive_expect_tx(&my_bars[st], Gm::kStageBytes);
-        // one instruction per tile and cache: all head_dim / 64 boxes
-        tma_load_5d(kdst, &kmap, &my_bars[st], 0, kvh, off, 0, phys);
-        tma_load_5d(vdst, &vmap, &my_bars[st], 0, kvh, off, 0, phys);
+        uint8_t* kdst = my_stages + st * Pl::kStageBytes;
+        uint8_t* vdst = kdst + Pl::kTileBytes;
+        mbar_arrive_expect_tx(&my_bars[st], Pl::kTx);
+        if constexpr (FP8) {
+            // one box of 16 rows x 128 codes per cache, and the 16-byte
+            // aligned groups of 4 scales holding this (block, head)'s
+            tma_load_4d(kdst, &kmap, &my_bars[st], 0, kvh, off, phys);
+            tma_load_4d(vdst, &vmap, &my_bars[st], 0, kvh, off, phys);
+            const int64_t g = scale_index(phys) & ~int64_t(3);
+            bulk_load(my_scales + st * 8, p.k_scale + g, 16, &my_bars[st]);
+            bulk_load(my_scales + st * 8 + 4, p.v_scale + g, 16, &my_bars[st]);
+        } else {
+            // one instruction per tile and cache: all head_dim / 64 boxes
+            tma_load_5d(kdst, &kmap, &my_bars[st], 0, kvh, off, 0, phys);
+            tma_load_5d(vdst, &vmap, &my_bars[st], 0, kvh, off, 0, phys);
+        }
     };
 
     const int my_tiles = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
@@ -511,21 +619,40 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             failed = true;
             break;
         }
-        uint8_t* kt = my_stages + st * Gm::kStageBytes;
-        uint8_t* vt = kt + Gm::kKBytes;
+        uint8_t* kt = my_stages + st * Pl::kStageBytes;
+        uint8_t* vt = kt + Pl::kTileBytes;
         const int valid = min(kTile, t_end - (t_begin + tile * kTile));
+        float kscale = 1.f, vscale = 1.f;
+        if constexpr (FP8) {
+            const int64_t si = scale_index(table[(t_begin + tile * kTile) / bs - lb0]) & 3;
+            kscale = my_scales[st * 8 + si];
+            vscale = my_scales[st * 8 + 4 + si];
+            if constexpr (Warp::kMma) {
+                widen_fp8_tile<T>(kt, my_wide, lane);
+                widen_fp8_tile<T>(vt, my_wide + Gm::kKBytes, lane);
+                __syncwarp();
+                kt = my_wide;
+                vt = my_wide + Gm::kKBytes;
+            }
+        }
         if (valid < kTile) {
             // rows past the context may hold anything (NaN included): zero
             // the V rows so that their zero weights contribute exactly 0
-            const int nchunks = (kTile - valid) * Gm::kBoxes * 8;
-            for (int c = lane; c < nchunks; c += 32) {
-                const int r = valid + c / (Gm::kBoxes * 8);
-                const int ch = c % (Gm::kBoxes * 8);
-                *reinterpret_cast<uint4*>(vt + swz(r, ch)) = make_uint4(0, 0, 0, 0);
+            if constexpr (FP8 && !Warp::kMma) {
+                for (int c = lane; c < (kTile - valid) * 8; c += 32)
+                    *reinterpret_cast<uint4*>(vt + (valid + c / 8) * 128 + (c % 8) * 16) =
+                        make_uint4(0, 0, 0, 0);
+            } else {
+                const int nchunks = (kTile - valid) * Gm::kBoxes * 8;
+                for (int c = lane; c < nchunks; c += 32) {
+                    const int r = valid + c / (Gm::kBoxes * 8);
+                    const int ch = c % (Gm::kBoxes * 8);
+                    *reinterpret_cast<uint4*>(vt + swz(r, ch)) = make_uint4(0, 0, 0, 0);
+                }
             }
             __syncwarp();
         }
-        w.tile(kt, vt, valid, p.scale_log2, lane);
+        w.tile(kt, vt, valid, p.scale_log2 * kscale, lane, vscale);
         // Every shared-memory read of this stage feeds an instruction that
         // precedes the next TMA issue in program order, so the reads are
         // complete before the stage is rewritten.
@@ -739,14 +866,12 @@ void plan_partitions(int max_context_len, int partition_size, int* P, int* NP) {
     }
 }
 
-template <typename T, int D, typename Warp>
+template <typename T, int D, typename Warp, bool FP8>
 int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
                   int num_kv_heads, cudaStream_t stream) {
-    using Gm = Geom<D>;
+    using Pl = Plan<D, FP8, Warp::kMma>;
     const int table_cap = (p.partition_size + p.block_size - 1) / p.block_size + 1;
-    const size_t smem = 1024 + (size_t)kWarps * Gm::kStages * Gm::kStageBytes +
-                        (size_t)kWarps * Gm::kStages * sizeof(uint64_t) +
-                        (size_t)table_cap * sizeof(int32_t);
+    const size_t smem = 1024 + Pl::kTableOff + (size_t)table_cap * sizeof(int32_t);
     if (smem > 227 * 1024)
         return fail(PKV_ERR_UNSUPPORTED,
                     "pkv_decode_attention: %d tokens per partition need %zu bytes of shared "
@@ -755,12 +880,12 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
     // the merging CTA keeps the partials' m and l of its G heads in the
     // (then idle) stage buffers
     const size_t merge_smem = (size_t)p.group * (2 * p.num_partitions + 2) * sizeof(float);
-    if (p.num_partitions > 1 && merge_smem > (size_t)kWarps * Gm::kStages * Gm::kStageBytes)
+    if (p.num_partitions > 1 && merge_smem > Pl::kEpilogue)
         return fail(PKV_ERR_UNSUPPORTED,
                     "pkv_decode_attention: %d partitions of %d query heads are too many to "
                     "merge in one CTA; use a larger partition_size",
                     p.num_partitions, p.group);
-    auto kern = paged_decode_kernel<T, D, Warp>;
+    auto kern = paged_decode_kernel<T, D, Warp, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess)
@@ -779,13 +904,34 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
     return launch_status("pkv_decode_attention");
 }
 
-template <typename T, int D>
+template <typename T, int D, bool FP8>
 int dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
                    int num_kv_heads, cudaStream_t stream) {
-    if (p.group == 1) return launch_decode<T, D, GemvWarp<T, D>>(kmap, vmap, p, num_kv_heads, stream);
+    if (p.group == 1)
+        return launch_decode<T, D, GemvWarp<T, D, FP8>, FP8>(kmap, vmap, p, num_kv_heads, stream);
     if (p.group <= 8)
-        return launch_decode<T, D, MmaWarp<T, D, 1>>(kmap, vmap, p, num_kv_heads, stream);
-    return launch_decode<T, D, MmaWarp<T, D, 2>>(kmap, vmap, p, num_kv_heads, stream);
+        return launch_decode<T, D, MmaWarp<T, D, 1>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+    return launch_decode<T, D, MmaWarp<T, D, 2>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+}
+
+// 4-D view of one e4m3 cache: (head_dim codes, kv head, slot, block), boxes
+// of 128 x 1 x 16 x 1 codes (one 128-byte row per token) with 128-byte
+// swizzling.  block_stride is in bytes.
+int encode_cache_map_fp8(CUtensorMap* map, const void* cache, int head_dim, int num_kv_heads,
+                         int block_size, int num_blocks, int64_t block_stride) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads,
+                                (cuuint64_t)block_size, (cuuint64_t)num_blocks};
+    const cuuint64_t strides[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads * head_dim,
+                                   (cuuint64_t)block_stride};
+    const cuuint32_t box[4] = {(cuuint32_t)head_dim, 1, kTile, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(cache), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PKV_OK;
 }
 
 }  // namespace
@@ -801,19 +947,24 @@ extern "C" size_t pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int 
     return workspace_layout(num_seqs, num_q_heads, NP, head_dim).total;
 }
 
-extern "C" int pkv_decode_attention(void* out, const void* query, const void* key_cache,
-                                    const void* value_cache, const int32_t* block_tables,
-                                    int max_blocks_per_seq, const int32_t* context_lens,
-                                    int num_seqs, int max_context_len, int num_q_heads,
-                                    int num_kv_heads, int head_dim, int num_blocks,
-                                    int block_size, int64_t block_stride, float scale,
-                                    int partition_size, void* workspace, size_t workspace_bytes,
-                                    pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
-    using namespace pkv;
+namespace pkv {
+namespace {
+
+// Both entry points: 16-bit caches (fp8 false) or e4m3 caches with their
+// per-(block, KV head) scales (fp8 true; block_stride then in bytes).
+int decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                const float* k_scale, const float* v_scale, bool fp8,
+                const int32_t* block_tables, int max_blocks_per_seq,
+                const int32_t* context_lens, int num_seqs, int max_context_len, int num_q_heads,
+                int num_kv_heads, int head_dim, int num_blocks, int block_size,
+                int64_t block_stride, float scale, int partition_size, void* workspace,
+                size_t workspace_bytes, pkv_dtype dtype, int32_t* dev_error,
+                cudaStream_t stream) {
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_decode_attention: dtype %d", (int)dtype);
-    PKV_REQUIRE(head_dim == 64 || head_dim == 128, PKV_ERR_UNSUPPORTED,
-                "pkv_decode_attention: head_dim %d (built: 64, 128)", head_dim);
+    PKV_REQUIRE(head_dim == 128 || (head_dim == 64 && !fp8), PKV_ERR_UNSUPPORTED,
+                "pkv_decode_attention: head_dim %d (built: 64, 128; e4m3 caches: 128)",
+                head_dim);
     PKV_REQUIRE(block_size > 0 && block_size % kTile == 0 && block_size <= 256,
                 PKV_ERR_UNSUPPORTED,
                 "pkv_decode_attention: block_size %d (built: multiples of 16 up to 256)",
@@ -835,8 +986,9 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
                 "pkv_decode_attention: max_context_len %d exceeds the table (%d x %d)",
                 max_context_len, max_blocks_per_seq, block_size);
     const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
-    PKV_REQUIRE(block_stride >= block_elems && block_stride % 8 == 0, PKV_ERR_INVALID,
-                "pkv_decode_attention: block_stride %lld", (long long)block_stride);
+    PKV_REQUIRE(block_stride >= block_elems && block_stride % (fp8 ? 16 : 8) == 0,
+                PKV_ERR_INVALID, "pkv_decode_attention: block_stride %lld",
+                (long long)block_stride);
     PKV_REQUIRE(num_kv_heads <= 65535, PKV_ERR_UNSUPPORTED, "too many KV heads");
     if (num_seqs == 0) return PKV_OK;
     PKV_REQUIRE(out && query && key_cache && value_cache && context_lens &&
@@ -846,6 +998,9 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
                     aligned16(value_cache),
                 PKV_ERR_INVALID, "pkv_decode_attention: pointers must be 16-byte aligned");
     PKV_REQUIRE(num_blocks > 0, PKV_ERR_INVALID, "pkv_decode_attention: empty pool");
+    PKV_REQUIRE(!fp8 || (k_scale && v_scale && aligned16(k_scale) && aligned16(v_scale)),
+                PKV_ERR_INVALID,
+                "pkv_decode_attention_fp8: scales must be 16-byte aligned device arrays");
 
     DecodeParams p{};
     p.out = out;
@@ -862,6 +1017,8 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
     p.num_blocks = num_blocks;
     p.block_size = block_size;
     p.scale_log2 = scale * kLog2e;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     plan_partitions(max_context_len, partition_size, &p.partition_size, &p.num_partitions);
     PKV_REQUIRE(p.num_partitions <= 65535, PKV_ERR_UNSUPPORTED,
                 "pkv_decode_attention: %d partitions (max 65535)", p.num_partitions);
@@ -879,18 +1036,63 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
     }
 
     CUtensorMap kmap, vmap;
-    int st = encode_cache_map(&kmap, key_cache, dtype, head_dim, num_kv_heads, block_size,
-                              num_blocks, block_stride);
+    int st = fp8 ? encode_cache_map_fp8(&kmap, key_cache, head_dim, num_kv_heads, block_size,
+                                        num_blocks, block_stride)
+                 : encode_cache_map(&kmap, key_cache, dtype, head_dim, num_kv_heads, block_size,
+                                    num_blocks, block_stride);
     if (st != PKV_OK) return st;
-    st = encode_cache_map(&vmap, value_cache, dtype, head_dim, num_kv_heads, block_size,
-                          num_blocks, block_stride);
+    st = fp8 ? encode_cache_map_fp8(&vmap, value_cache, head_dim, num_kv_heads, block_size,
+                                    num_blocks, block_stride)
+             : encode_cache_map(&vmap, value_cache, dtype, head_dim, num_kv_heads, block_size,
+                                num_blocks, block_stride);
     if (st != PKV_OK) return st;
 
     DeviceGuard guard(stream, key_cache);
-    if (dtype == PKV_BF16) {
-        return head_dim == 128 ? dispatch_group<__nv_bfloat16, 128>(kmap, vmap, p, num_kv_heads, stream)
-                               : dispatch_group<__nv_bfloat16, 64>(kmap, vmap, p, num_kv_heads, stream);
+    if (fp8) {
+        return dtype == PKV_BF16
+                   ? dispatch_group<__nv_bfloat16, 128, true>(kmap, vmap, p, num_kv_heads, stream)
+                   : dispatch_group<__half, 128, true>(kmap, vmap, p, num_kv_heads, stream);
     }
-    return head_dim == 128 ? dispatch_group<__half, 128>(kmap, vmap, p, num_kv_heads, stream)
-                           : dispatch_group<__half, 64>(kmap, vmap, p, num_kv_heads, stream);
+    if (dtype == PKV_BF16) {
+        return head_dim == 128
+                   ? dispatch_group<__nv_bfloat16, 128, false>(kmap, vmap, p, num_kv_heads, stream)
+                   : dispatch_group<__nv_bfloat16, 64, false>(kmap, vmap, p, num_kv_heads, stream);
+    }
+    return head_dim == 128 ? dispatch_group<__half, 128, false>(kmap, vmap, p, num_kv_heads, stream)
+                           : dispatch_group<__half, 64, false>(kmap, vmap, p, num_kv_heads, stream);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int pkv_decode_attention(void* out, const void* query, const void* key_cache,
+                                    const void* value_cache, const int32_t* block_tables,
+                                    int max_blocks_per_seq, const int32_t* context_lens,
+                                    int num_seqs, int max_context_len, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int num_blocks,
+                                    int block_size, int64_t block_stride, float scale,
+                                    int partition_size, void* workspace, size_t workspace_bytes,
+                                    pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    return pkv::decode_impl(out, query, key_cache, value_cache, nullptr, nullptr, false,
+                            block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                            block_size, block_stride, scale, partition_size, workspace,
+                            workspace_bytes, dtype, dev_error, stream);
+}
+
+extern "C" int pkv_decode_attention_fp8(void* out, const void* query, const void* key_cache,
+                                        const void* value_cache, const float* k_scale,
+                                        const float* v_scale, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* context_lens,
+                                        int num_seqs, int max_context_len, int num_q_heads,
+                                        int num_kv_heads, int head_dim, int num_blocks,
+                                        int block_size, int64_t block_stride, float scale,
+                                        int partition_size, void* workspace,
+                                        size_t workspace_bytes, pkv_dtype dtype,
+                                        int32_t* dev_error, cudaStream_t stream) {
+    return pkv::decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, true,
+                            block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                            block_size, block_stride, scale, partition_size, workspace,
+                            workspace_bytes, dtype, dev_error, stream);
 }

@@ -152,6 +152,34 @@ def fill_device_cache_(tensor, seed):
     return tensor
 
 
+def fill_device_scales_(scales, seed, amax=4.0):
+    """Seeded per-(block, KV head) e4m3 scales: amax / 448 (amax about the
+    largest |x| of the 2048 N(0,1) values a block of 16 slots x 128 dims
+    holds per head) times U[0.75, 1.25], so blocks differ."""
+    gen = torch.Generator(scales.device).manual_seed(seed)
+    u = torch.rand(scales.shape, generator=gen, device=scales.device, dtype=torch.float32)
+    scales.copy_((0.75 + 0.5 * u) * (amax / 448.0))
+    return scales
+
+
+def fill_device_cache_fp8_(cache, scales, seed):
+    """Fill an e4m3 cache ([NB, bs, Hkv, D] uint8) with N(0,1) values
+    quantised (by torch's float8 conversion, setup only; the benchmark's
+    caches are not compared with the oracle) with the block's scale for each
+    KV head."""
+    gen = torch.Generator(cache.device).manual_seed(seed)
+    nb, bs, hkv, d = cache.shape
+    step = max(1, (1 << 26) // (bs * hkv * d))
+    for b0 in range(0, nb, step):
+        b1 = min(nb, b0 + step)
+        x = torch.randn((b1 - b0, bs, hkv, d), generator=gen, device=cache.device,
+                        dtype=torch.float32)
+        x /= scales[b0:b1, None, :, None]
+        x.clamp_(-448.0, 448.0)  # saturate: the cast would give NaN beyond 448
+        cache[b0:b1].copy_(x.to(torch.float8_e4m3fn).view(torch.uint8))
+    return cache
+
+
 # ---------------------------------------------------------------------------
 # Shared-prefix parallel sampling (copy-on-write workload)
 # ---------------------------------------------------------------------------
