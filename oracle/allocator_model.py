@@ -29,6 +29,23 @@ Readings where the pages are silent:
   block, the old block loses one reference and the table entry is replaced;
   the last holder (refcount 1) writes in place;
 * slot = physical_block * block_size + offset.
+
+Block swapping ("PagedAttention 动态内存分页" page, 动态块分配与回收: when GPU
+memory runs short, a sequence's KV blocks are moved to CPU memory and
+brought back when needed).  Readings:
+
+* the host pool is a second LIFO stack of host block ids, made once
+  (``set_host_blocks``), first allocation 0, 1, ...;
+* swap-out moves one whole sequence: in table order each block takes a host
+  block (pair (gpu, host)), then the GPU block loses this sequence's
+  reference (returning to the GPU stack at zero, in table order); a block
+  still shared with a resident sequence stays on the GPU for it, and the
+  swapped sequence keeps its own host copy;
+* swap-in is the reverse: each host block takes a GPU block (pair (host,
+  gpu)) and returns to the host stack, in table order;
+* either one that runs out of blocks changes nothing and reports OOM;
+* a swapped-out sequence cannot be appended to or forked; freeing it
+  returns its host blocks.
 """
 
 OK = 0
@@ -53,6 +70,9 @@ class PoolModel:
         self.refcount = [0] * num_blocks
         self.tables = {}  # seq_id -> list of physical blocks
         self.tokens = {}  # seq_id -> number of tokens
+        self.host_free = None  # host block stack, once set_host_blocks ran
+        self.host_refcount = []
+        self.swapped = set()  # sequences whose table lists host blocks
 
     # -- helpers ---------------------------------------------------------
     def _take(self):
@@ -78,7 +98,7 @@ class PoolModel:
 
     def seq_fork(self, parent, child):
         """The child shares every block of the parent (one more reference)."""
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or child in self.tables or parent in self.swapped:
             return ERR_INVALID
         self.tables[child] = list(self.tables[parent])
         self.tokens[child] = self.tokens[parent]
@@ -89,7 +109,7 @@ class PoolModel:
     def seq_append(self, seq_id):
         """Reserve the slot of one new token.  Returns (status, slot, cow_src,
         cow_dst); cow_src/cow_dst are -1 when no copy is needed."""
-        if seq_id not in self.tables:
+        if seq_id not in self.tables or seq_id in self.swapped:
             return ERR_INVALID, -1, -1, -1
         table = self.tables[seq_id]
         off = self.tokens[seq_id] % self.block_size
@@ -113,12 +133,68 @@ class PoolModel:
     def seq_free(self, seq_id):
         if seq_id not in self.tables:
             return ERR_INVALID
+        if seq_id in self.swapped:
+            self.swapped.discard(seq_id)
+            for h in self.tables.pop(seq_id):
+                self.host_refcount[h] -= 1
+                if self.host_refcount[h] == 0:
+                    self.host_free.append(h)
+            del self.tokens[seq_id]
+            return OK
         for b in self.tables.pop(seq_id):
             self.refcount[b] -= 1
             if self.refcount[b] == 0:
                 self.free.append(b)
         del self.tokens[seq_id]
         return OK
+
+    # -- swapping ----------------------------------------------------------
+    def set_host_blocks(self, num_host_blocks):
+        """Make the host pool (once): host blocks 0 .. num_host_blocks-1."""
+        if self.host_free is not None or num_host_blocks < 0:
+            return ERR_INVALID
+        self.host_free = list(range(num_host_blocks))[::-1]
+        self.host_refcount = [0] * num_host_blocks
+        return OK
+
+    def seq_swap_out(self, seq_id):
+        """Move a resident sequence to host blocks.  Returns (status,
+        [(gpu_block, host_block), ...]) in table order."""
+        if (self.host_free is None or seq_id not in self.tables
+                or seq_id in self.swapped):
+            return ERR_INVALID, []
+        table = self.tables[seq_id]
+        if len(table) > len(self.host_free):
+            return ERR_OOM, []
+        pairs = []
+        for b in table:
+            h = self.host_free.pop()
+            self.host_refcount[h] = 1
+            pairs.append((b, h))
+        for b in table:
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free.append(b)
+        self.tables[seq_id] = [h for _, h in pairs]
+        self.swapped.add(seq_id)
+        return OK, pairs
+
+    def seq_swap_in(self, seq_id):
+        """Bring a swapped-out sequence back to GPU blocks.  Returns (status,
+        [(host_block, gpu_block), ...]) in table order."""
+        if seq_id not in self.swapped:
+            return ERR_INVALID, []
+        table = self.tables[seq_id]
+        if len(table) > len(self.free):
+            return ERR_OOM, []
+        pairs = [(h, self._take()) for h in table]
+        for h in table:
+            self.host_refcount[h] -= 1
+            if self.host_refcount[h] == 0:
+                self.host_free.append(h)
+        self.tables[seq_id] = [g for _, g in pairs]
+        self.swapped.discard(seq_id)
+        return OK, pairs
 
     # -- observations ----------------------------------------------------
     def num_free(self):
@@ -135,3 +211,8 @@ class PoolModel:
             tuple(self.refcount),
             tuple(sorted((s, tuple(t), self.tokens[s]) for s, t in self.tables.items())),
         )
+
+    def host_state(self):
+        """The host pool and which sequences are swapped out."""
+        return (tuple(self.host_free or ()), tuple(self.host_refcount),
+                tuple(sorted(self.swapped)))

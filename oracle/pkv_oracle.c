@@ -333,6 +333,30 @@ int pkv_oracle_copy_blocks(uint16_t* key_cache, uint16_t* value_cache,
     return 0;
 }
 
+/* Block swap between two pools ("PagedAttention 动态内存分页" page, 动态块分配
+ * 与回收: under memory pressure a sequence's KV blocks move to CPU memory and
+ * come back when it runs again).  For every pair (src, dst), the block_bytes
+ * bytes of block src of the source pool become block dst of the destination
+ * pool.  The pools are distinct arrays; blocks are block_bytes long at their
+ * own strides.  Any pair outside its pool: nothing is copied, -1. */
+int pkv_oracle_swap_blocks(uint8_t* dst, const uint8_t* src, const int32_t* block_pairs,
+                           int num_pairs, int src_num_blocks, int dst_num_blocks,
+                           int64_t block_bytes, int64_t src_block_stride,
+                           int64_t dst_block_stride) {
+    if (num_pairs < 0 || block_bytes < 0 || src_block_stride < block_bytes ||
+        dst_block_stride < block_bytes)
+        return -1;
+    for (int i = 0; i < num_pairs; ++i) {
+        int32_t s = block_pairs[2 * i], d = block_pairs[2 * i + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) return -1;
+    }
+    for (int i = 0; i < num_pairs; ++i) {
+        int64_t s = block_pairs[2 * i], d = block_pairs[2 * i + 1];
+        memcpy(dst + d * dst_block_stride, src + s * src_block_stride, (size_t)block_bytes);
+    }
+    return 0;
+}
+
 /* Bytes of one physical block, as the "Paged KV" wiki page's 初始化阶段
  * section gives them: block_size x num_kv_heads x head_dim x 2 (K and V)
  * x num_layers x dtype_bytes. */

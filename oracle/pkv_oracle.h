@@ -55,6 +55,11 @@ int pkv_oracle_copy_blocks(uint16_t* key_cache, uint16_t* value_cache,
                            int num_blocks, int block_size, int num_kv_heads,
                            int head_dim, int64_t block_stride);
 
+int pkv_oracle_swap_blocks(uint8_t* dst, const uint8_t* src, const int32_t* block_pairs,
+                           int num_pairs, int src_num_blocks, int dst_num_blocks,
+                           int64_t block_bytes, int64_t src_block_stride,
+                           int64_t dst_block_stride);
+
 int64_t pkv_oracle_block_bytes(int block_size, int num_kv_heads, int head_dim,
                                int num_layers, int dtype_bytes);
 

@@ -39,6 +39,7 @@ def lib():
         L.pkv_oracle_merge_partials.argtypes = [p, p, p, p, p, i, i, i, i, i]
         L.pkv_oracle_write_slots.argtypes = [p, p, p, p, p, i, i, i, i, i, i64]
         L.pkv_oracle_copy_blocks.argtypes = [p, p, p, i, i, i, i, i, i64]
+        L.pkv_oracle_swap_blocks.argtypes = [p, p, p, i, i, i, i64, i64, i64]
         L.pkv_oracle_block_bytes.argtypes = [i, i, i, i, i]
         L.pkv_oracle_block_bytes.restype = i64
         L.pkv_oracle_max_threads.argtypes = []
@@ -204,6 +205,25 @@ def write_slots(key_cache, value_cache, key, value, slot_mapping, block_size,
                                       T, NB, block_size, num_kv_heads, D, block_stride)
     _check(rc, "write_slots")
     return kc, vc
+
+
+def swap_blocks(dst_pool, src_pool, block_pairs):
+    """Returns a copy of dst_pool ([NB_dst, ...], any dtype) whose block
+    pairs[i][1] holds block pairs[i][0] of src_pool; one block is one row of
+    the leading dimension."""
+    dst = _u8(dst_pool).copy()
+    src = _u8(src_pool)
+    nd, ns = int(dst_pool.shape[0]), int(src_pool.shape[0])
+    dst = dst.reshape(nd, -1)
+    src = np.ascontiguousarray(src).reshape(ns, -1)
+    if dst.shape[1] != src.shape[1]:
+        raise ValueError("the pools' blocks differ in size")
+    pairs = _i32(block_pairs).reshape(-1, 2)
+    nbytes = dst.shape[1]
+    rc = lib().pkv_oracle_swap_blocks(_ptr(dst), _ptr(src), _ptr(pairs), pairs.shape[0], ns, nd,
+                                      nbytes, nbytes, nbytes)
+    _check(rc, "swap_blocks")
+    return dst.reshape(_u8(dst_pool).shape)
 
 
 def copy_blocks(key_cache, value_cache, block_pairs, block_size, num_kv_heads,

@@ -177,3 +177,93 @@ def test_initial_order_is_taken_front_first():
     assert pool.seq_append(0)[1] == 4 * 2 + 0
     with pytest.raises(ValueError):
         PoolModel(3, 2, free_order=[0, 0, 1])
+
+
+# ---------------------------------------------------------------------------
+# block swapping ("PagedAttention 动态内存分页" page, 动态块分配与回收)
+# ---------------------------------------------------------------------------
+def test_swap_hand_worked_trace():
+    # GPU pool of 4 blocks (first taken 0, 1, ...), host pool of 3, bs 4
+    pool = PoolModel(4, 4)
+    assert pool.seq_swap_out(1) == (ERR_INVALID, [])  # no host pool yet
+    assert pool.set_host_blocks(3) == OK
+    assert pool.set_host_blocks(3) == ERR_INVALID  # made once
+    assert pool.seq_add(1, 6) == OK  # blocks 0, 1
+    assert pool.seq_fork(1, 2) == OK  # both shared
+    # seq 1 out: host blocks 0, 1; the GPU blocks stay with seq 2
+    assert pool.seq_swap_out(1) == (OK, [(0, 0), (1, 1)])
+    assert pool.refcount == [1, 1, 0, 0] and pool.free == [3, 2]
+    assert pool.host_free == [2] and pool.tables[1] == [0, 1]
+    assert pool.seq_append(1)[0] == ERR_INVALID
+    assert pool.seq_fork(1, 3) == ERR_INVALID
+    assert pool.seq_swap_out(1) == (ERR_INVALID, [])
+    # seq 1 back in: GPU blocks 2, 3; host blocks return in table order
+    assert pool.seq_swap_in(1) == (OK, [(0, 2), (1, 3)])
+    assert pool.free == [] and pool.host_free == [2, 0, 1]
+    assert pool.tables[1] == [2, 3] and pool.tokens[1] == 6
+    assert pool.seq_swap_in(1) == (ERR_INVALID, [])
+    # seq 2 out: host 1 then 0; its GPU blocks are freed in table order
+    assert pool.seq_swap_out(2) == (OK, [(0, 1), (1, 0)])
+    assert pool.free == [0, 1] and pool.refcount == [0, 0, 1, 1]
+    # a third sequence of 3 blocks cannot go out: one host block is left
+    assert pool.seq_free(1) == OK  # pushes 2, 3: free [0, 1, 2, 3]
+    assert pool.seq_add(3, 12) == OK  # takes 3, 2, 1 (LIFO)
+    assert pool.tables[3] == [3, 2, 1]
+    before = (pool.state(), pool.host_state())
+    assert pool.seq_swap_out(3) == (ERR_OOM, [])
+    assert (pool.state(), pool.host_state()) == before
+    # swapped-out seq 2 (2 blocks) cannot come back while only block 0 is free
+    assert pool.free == [0]
+    assert pool.seq_swap_in(2) == (ERR_OOM, [])
+    assert (pool.state(), pool.host_state()) == before
+    # freeing a swapped sequence returns its host blocks
+    assert pool.seq_free(2) == OK
+    assert pool.host_free == [2, 1, 0] and pool.host_refcount == [0, 0, 0]
+
+
+def _check_swap_invariants(pool):
+    resident = {s: t for s, t in pool.tables.items() if s not in pool.swapped}
+    swapped = {s: t for s, t in pool.tables.items() if s in pool.swapped}
+    for b in range(pool.num_blocks):
+        holders = sum(t.count(b) for t in resident.values())
+        assert pool.refcount[b] == holders
+        assert (b in pool.free) == (holders == 0)
+    for h in range(len(pool.host_refcount)):
+        holders = sum(t.count(h) for t in swapped.values())
+        assert pool.host_refcount[h] == holders <= 1
+        assert (h in pool.host_free) == (holders == 0)
+    assert len(pool.free) == len(set(pool.free))
+    assert len(pool.host_free) == len(set(pool.host_free))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_swap_invariants_under_random_operations(seed):
+    rnd = random.Random(seed)
+    pool = PoolModel(40, 4)
+    pool.set_host_blocks(30)
+    tokens_before = {}
+    for _ in range(600):
+        op = rnd.random()
+        ids = list(pool.tables)
+        if op < 0.2 or not ids:
+            pool.seq_add(rnd.randrange(100), rnd.randrange(0, 30))
+        elif op < 0.3:
+            pool.seq_fork(rnd.choice(ids), rnd.randrange(100))
+        elif op < 0.55:
+            pool.seq_append(rnd.choice(ids))
+        elif op < 0.7:
+            s = rnd.choice(ids)
+            tokens_before[s] = pool.tokens[s]
+            st, pairs = pool.seq_swap_out(s)
+            if st == OK:
+                assert [h for _, h in pairs] == pool.tables[s]
+        elif op < 0.85:
+            s = rnd.choice(ids)
+            table = list(pool.tables[s])
+            st, pairs = pool.seq_swap_in(s)
+            if st == OK:
+                assert [h for h, _ in pairs] == table
+                assert pool.tokens[s] == tokens_before[s]
+        else:
+            pool.seq_free(rnd.choice(ids))
+        _check_swap_invariants(pool)

@@ -394,3 +394,33 @@ def test_block_bytes_golden():
     for r in golden_lines("block_bytes.txt"):
         bs, hkv, d, layers, dtb, want = map(int, r)
         assert ref.block_bytes(bs, hkv, d, layers, dtb) == want
+
+
+# ---------------------------------------------------------------------------
+# block swap copy ("PagedAttention 动态内存分页" page, 动态块分配与回收)
+# ---------------------------------------------------------------------------
+def test_swap_blocks_matches_fancy_indexing_and_round_trips():
+    rng = np.random.default_rng(5)
+    gpu = rng.integers(0, 2**16, size=(12, 4, 2, 8), dtype=np.uint16)
+    host = rng.integers(0, 2**16, size=(9, 4, 2, 8), dtype=np.uint16)
+    src = rng.permutation(12)[:6]
+    dst = rng.permutation(9)[:6]
+    pairs = np.stack([src, dst], axis=1).astype(np.int32)
+    out = ref.swap_blocks(host, gpu, pairs).view(np.uint16).reshape(host.shape)
+    want = host.copy()
+    want[dst] = gpu[src]  # the library's gather/scatter
+    assert np.array_equal(out, want)
+    # and back: the inverse pairs restore the original blocks elsewhere
+    fresh = np.zeros_like(gpu)
+    back = ref.swap_blocks(fresh, out, pairs[:, ::-1]).view(np.uint16).reshape(gpu.shape)
+    assert np.array_equal(back[src], gpu[src])
+    assert not back[np.setdiff1d(np.arange(12), src)].any()
+
+
+def test_swap_blocks_rejects_pairs_outside_either_pool():
+    gpu = np.zeros((4, 16), np.uint8)
+    host = np.zeros((2, 16), np.uint8)
+    with pytest.raises(Exception):
+        ref.swap_blocks(host, gpu, [[3, 2]])  # host block 2 of 2
+    with pytest.raises(Exception):
+        ref.swap_blocks(host, gpu, [[4, 0]])  # gpu block 4 of 4
