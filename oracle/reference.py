@@ -207,6 +207,16 @@ def write_slots(key_cache, value_cache, key, value, slot_mapping, block_size,
     return kc, vc
 
 
+def copy_blocks_layers(key_caches, value_caches, block_pairs, block_size, num_kv_heads,
+                       head_dim):
+    """Copy-on-write over a multi-layer cache: one physical block id names
+    the block in every layer ("Paged KV" wiki page, 初始化阶段: a block holds
+    K and V of all layers), so each pair is copied in each layer.  Returns
+    the new per-layer (key, value) bit arrays."""
+    return [copy_blocks(k, v, block_pairs, block_size, num_kv_heads, head_dim)
+            for k, v in zip(key_caches, value_caches)]
+
+
 def swap_blocks(dst_pool, src_pool, block_pairs):
     """Returns a copy of dst_pool ([NB_dst, ...], any dtype) whose block
     pairs[i][1] holds block pairs[i][0] of src_pool; one block is one row of

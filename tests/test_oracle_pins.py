@@ -424,3 +424,19 @@ def test_swap_blocks_rejects_pairs_outside_either_pool():
         ref.swap_blocks(host, gpu, [[3, 2]])  # host block 2 of 2
     with pytest.raises(Exception):
         ref.swap_blocks(host, gpu, [[4, 0]])  # gpu block 4 of 4
+
+
+def test_copy_blocks_layers_copies_each_layer_and_nothing_else():
+    import torch
+
+    g = torch.Generator().manual_seed(8)
+    L, nb, bs, H, D = 3, 10, 4, 2, 8
+    ks = [torch.randn(nb, bs, H, D, generator=g).to(torch.bfloat16) for _ in range(L)]
+    vs = [torch.randn(nb, bs, H, D, generator=g).to(torch.bfloat16) for _ in range(L)]
+    pairs = np.array([[2, 7], [5, 0], [9, 3]], np.int32)
+    out = ref.copy_blocks_layers(ks, vs, pairs, bs, H, D)
+    for l in range(L):
+        for c, (k_or_v) in enumerate((ks[l], vs[l])):
+            want = ref.bits(k_or_v).copy()
+            want[pairs[:, 1]] = want[pairs[:, 0]]  # the library's gather/scatter
+            assert np.array_equal(out[l][c].reshape(want.shape), want)
