@@ -197,6 +197,66 @@ int pkv_oracle_decode_attention(double* out, const uint16_t* query,
     return bad ? -1 : 0;
 }
 
+/* Paged prefill attention ("Paged KV" wiki page, 实现原理 / 运行阶段: prefill
+ * takes blocks in order and fills them with the prompt's K/V; the prompt's
+ * tokens then attend to the sequence through the same Block Table).  The
+ * query rows of sequence s are query_start[s] .. query_start[s+1]-1: the
+ * last n_s of its L_s = context_lens[s] cached tokens (a prompt, or a later
+ * chunk of one after L_s - n_s tokens already cached).  Row query_start[s]
+ * + i is token p = L_s - n_s + i and attends causally, to tokens 0 .. p:
+ *     out[row, h] = sum_{t <= p} softmax_t(scale * <query[row, h], K_t>) V_t. */
+int pkv_oracle_prefill_attention(double* out, const uint16_t* query,
+                                 const uint16_t* key_cache, const uint16_t* value_cache,
+                                 const int32_t* block_tables, int max_blocks_per_seq,
+                                 const int32_t* context_lens, const int32_t* query_start,
+                                 int num_seqs, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int num_blocks, int block_size,
+                                 int64_t block_stride, double scale, int dtype,
+                                 int num_threads) {
+    const int S = num_seqs, Hq = num_q_heads, Hkv = num_kv_heads, D = head_dim;
+    const int MB = max_blocks_per_seq, bs = block_size;
+    if (check_shapes(S, Hq, Hkv, D, num_blocks, bs, block_stride, MB)) return -1;
+    if (query_start[0] != 0) return -1;
+    int max_len = 0;
+    for (int s = 0; s < S; ++s) {
+        if (check_seq(block_tables, MB, context_lens, s, num_blocks, bs)) return -1;
+        const int n = query_start[s + 1] - query_start[s];
+        if (n < 0 || n > context_lens[s]) return -1;
+        if (context_lens[s] > max_len) max_len = context_lens[s];
+    }
+    const int64_t rows = query_start[S];
+    const int G = Hq / Hkv;
+    int bad = 0;
+#ifdef _OPENMP
+    omp_set_num_threads(num_threads > 0 ? num_threads : omp_get_num_procs());
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel reduction(| : bad)
+    {
+        double* scores = (double*)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+        if (!scores) bad = 1;
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t rh = 0; rh < rows * Hq; ++rh) {
+            if (!scores) continue;
+            const int64_t row = rh / Hq;
+            const int h = (int)(rh % Hq);
+            int s = 0; /* the sequence holding this row */
+            while (query_start[s + 1] <= row) ++s;
+            const int n = query_start[s + 1] - query_start[s];
+            const int p = context_lens[s] - n + (int)(row - query_start[s]);
+            double m, l;
+            double* o = out + rh * D;
+            attend_range(&m, &l, o, query + rh * D, key_cache, value_cache,
+                         block_tables + (int64_t)s * MB, 0, p + 1, h / G, Hkv, D, bs,
+                         block_stride, scale, dtype, scores);
+            for (int d = 0; d < D; ++d) o[d] /= l;
+        }
+        free(scores);
+    }
+    return bad ? -1 : 0;
+}
+
 int pkv_oracle_decode_partials(double* m_out, double* l_out, double* o_out,
                                const uint16_t* query, const uint16_t* key_cache,
                                const uint16_t* value_cache,

@@ -28,6 +28,15 @@ int pkv_oracle_decode_attention(double* out, const uint16_t* query,
                                 int64_t block_stride, double scale, int dtype,
                                 int num_threads);
 
+int pkv_oracle_prefill_attention(double* out, const uint16_t* query,
+                                 const uint16_t* key_cache, const uint16_t* value_cache,
+                                 const int32_t* block_tables, int max_blocks_per_seq,
+                                 const int32_t* context_lens, const int32_t* query_start,
+                                 int num_seqs, int num_q_heads, int num_kv_heads,
+                                 int head_dim, int num_blocks, int block_size,
+                                 int64_t block_stride, double scale, int dtype,
+                                 int num_threads);
+
 int pkv_oracle_decode_partials(double* m_out, double* l_out, double* o_out,
                                const uint16_t* query, const uint16_t* key_cache,
                                const uint16_t* value_cache,

@@ -40,6 +40,8 @@ def lib():
         L.pkv_oracle_write_slots.argtypes = [p, p, p, p, p, i, i, i, i, i, i64]
         L.pkv_oracle_copy_blocks.argtypes = [p, p, p, i, i, i, i, i, i64]
         L.pkv_oracle_swap_blocks.argtypes = [p, p, p, i, i, i, i64, i64, i64]
+        L.pkv_oracle_prefill_attention.argtypes = [p, p, p, p, p, i, p, p, i, i, i, i, i, i,
+                                                   i64, d, i, i]
         L.pkv_oracle_block_bytes.argtypes = [i, i, i, i, i]
         L.pkv_oracle_block_bytes.restype = i64
         L.pkv_oracle_max_threads.argtypes = []
@@ -205,6 +207,34 @@ def write_slots(key_cache, value_cache, key, value, slot_mapping, block_size,
                                       T, NB, block_size, num_kv_heads, D, block_stride)
     _check(rc, "write_slots")
     return kc, vc
+
+
+def prefill_attention(query, key_cache, value_cache, block_tables, context_lens, query_start,
+                      scale, dtype, num_kv_heads, block_size, block_stride=None, num_threads=0):
+    """Causal paged attention of each sequence's last n_s tokens (query rows
+    query_start[s] .. query_start[s+1]-1 of query [T, Hq, D]) over its
+    cached K/V, in fp64.  Returns [T, Hq, D]."""
+    q = bits(query)
+    kc = bits(key_cache)
+    vc = bits(value_cache)
+    T, Hq, D = q.shape
+    tables = _i32(block_tables)
+    lens = _i32(context_lens)
+    qs = _i32(query_start)
+    S = lens.shape[0]
+    if qs.shape[0] != S + 1 or qs[-1] != T:
+        raise ValueError("query_start must be [num_seqs + 1] ending at the number of rows")
+    MB = tables.shape[1] if tables.ndim == 2 else 0
+    if block_stride is None:
+        block_stride = block_size * num_kv_heads * D
+    NB = _num_blocks(kc.size, block_stride, block_size * num_kv_heads * D)
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = lib().pkv_oracle_prefill_attention(
+        _ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables), MB, _ptr(lens), _ptr(qs), S, Hq,
+        num_kv_heads, D, NB, block_size, block_stride, float(scale), _dtype_code(dtype),
+        int(num_threads))
+    _check(rc, "prefill_attention")
+    return out
 
 
 def copy_blocks_layers(key_caches, value_caches, block_pairs, block_size, num_kv_heads,

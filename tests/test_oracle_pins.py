@@ -440,3 +440,79 @@ def test_copy_blocks_layers_copies_each_layer_and_nothing_else():
             want = ref.bits(k_or_v).copy()
             want[pairs[:, 1]] = want[pairs[:, 0]]  # the library's gather/scatter
             assert np.array_equal(out[l][c].reshape(want.shape), want)
+
+
+# ---------------------------------------------------------------------------
+# paged prefill attention ("Paged KV" wiki page, 实现原理 / 运行阶段)
+# ---------------------------------------------------------------------------
+def _prefill_case(seed, lens, chunk, Hq, Hkv, D, bs, dtype="bf16"):
+    import torch
+
+    from tests.helpers import paged_problem
+
+    p = paged_problem(seed, Hq, Hkv, D, bs, lens, dtype)
+    g = torch.Generator().manual_seed(seed + 1)
+    n = [min(c, L) for c, L in zip(chunk, lens)]
+    qs = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = torch.randn(int(qs[-1]), Hq, D, generator=g).to(p["q"].dtype)
+    return p, q, qs, n
+
+
+def _dense_causal(p, q, qs, n, lens, Hq, Hkv, D, bs, scale):
+    """The definition on gathered dense K/V with numpy and scipy's softmax."""
+    from scipy.special import softmax
+
+    kc = p["kc"].double().numpy()
+    vc = p["vc"].double().numpy()
+    qd = q.double().numpy()
+    out = np.zeros_like(qd)
+    G = Hq // Hkv
+    for s, L in enumerate(lens):
+        idx = [(p["tables"][s][t // bs], t % bs) for t in range(L)]
+        K = np.stack([kc[b, o] for b, o in idx]) if L else np.zeros((0, Hkv, D))
+        V = np.stack([vc[b, o] for b, o in idx]) if L else np.zeros((0, Hkv, D))
+        for i in range(n[s]):
+            pos = L - n[s] + i
+            for h in range(Hq):
+                sc = scale * K[:pos + 1, h // G] @ qd[qs[s] + i, h]
+                out[qs[s] + i, h] = softmax(sc) @ V[:pos + 1, h // G]
+    return out
+
+
+@pytest.mark.parametrize("lens,chunk", [([5, 17, 33], [5, 17, 33]),  # whole prompts
+                                        ([40, 9, 70], [8, 9, 31]),   # later chunks
+                                        ([1, 16, 0], [1, 3, 0])])    # tiny and empty
+def test_prefill_matches_dense_causal_softmax(lens, chunk):
+    Hq, Hkv, D, bs, scale = 6, 2, 16, 8, 0.3
+    p, q, qs, n = _prefill_case(11, lens, chunk, Hq, Hkv, D, bs)
+    got = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                Hkv, bs)
+    want = _dense_causal(p, q, qs, n, lens, Hq, Hkv, D, bs, scale)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_with_one_row_per_sequence_is_decode():
+    Hq, Hkv, D, bs, scale = 8, 2, 32, 16, 0.2
+    lens = [3, 16, 47, 100]
+    p, q, qs, n = _prefill_case(12, lens, [1] * 4, Hq, Hkv, D, bs)
+    got = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                Hkv, bs)
+    want = ref.decode_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], scale, "bf16",
+                                Hkv, bs)
+    assert np.array_equal(got, want)
+
+
+def test_prefill_first_prompt_row_is_v0_and_chunks_compose():
+    Hq, Hkv, D, bs, scale = 4, 4, 16, 8, 0.25
+    L = 29
+    p, q, qs, n = _prefill_case(13, [L], [L], Hq, Hkv, D, bs)
+    full = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                 Hkv, bs)
+    b0 = p["tables"][0][0]
+    assert np.array_equal(full[0], p["vc"][b0, 0].double().numpy())  # one token: weight 1
+    # the same prompt in two chunks: 12 tokens, then 17 more
+    a = ref.prefill_attention(q[:12], p["kc"], p["vc"], p["tables"], [12], [0, 12], scale,
+                              "bf16", Hkv, bs)
+    b = ref.prefill_attention(q[12:], p["kc"], p["vc"], p["tables"], [L], [0, 17], scale,
+                              "bf16", Hkv, bs)
+    assert np.array_equal(np.concatenate([a, b]), full)
