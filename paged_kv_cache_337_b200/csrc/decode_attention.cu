@@ -129,16 +129,38 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool* b
 // ---------------------------------------------------------------------------
 // Per-warp arithmetic, G == 1: FFMA + shuffles
 // ---------------------------------------------------------------------------
+// FP8 (e4m3 caches): the lane's query dims are also kept as f16 pairs,
+// scaled by a power of two into f16 range, so that the K dot products run
+// on the mixed-precision fma straight from the widened codes.
 template <typename T, int D, bool FP8 = false>
 struct GemvWarp {
     static constexpr int DV = D / 32;  // dims per lane
     static constexpr int GP = 1;       // heads held (padded)
     static constexpr bool kMma = false;
     float q[DV], o[DV], m, l;
+    uint32_t qh[DV / 2];               // e4m3 caches: q * 2^sh as f16x2
+    float qinv;                        // 2^-sh
 
     __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
         const T* qrow = static_cast<const T*>(p.query) + ((int64_t)s * p.num_q_heads + kvh) * D;
         load(reinterpret_cast<const uint8_t*>(qrow + lane * DV), q);
+        qinv = 1.f;
+        if constexpr (FP8) {
+            float mx = 0.f;
+#pragma unroll
+            for (int j = 0; j < DV; ++j) mx = fmaxf(mx, fabsf(q[j]));
+#pragma unroll
+            for (int x = 1; x < 32; x <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, x));
+            // largest |q| into [2^14, 2^15)
+            int ex = 0;
+            frexpf(mx, &ex);
+            const int sh = mx > 0.f ? max(-120, min(120, 15 - ex)) : 0;
+            const float qs = ldexpf(1.f, sh);
+            qinv = ldexpf(1.f, -sh);
+#pragma unroll
+            for (int j = 0; j < DV / 2; ++j)
+                qh[j] = Storage<__half>::from_float2(q[2 * j] * qs, q[2 * j + 1] * qs);
+        }
 #pragma unroll
         for (int j = 0; j < DV; ++j) o[j] = 0.f;
         m = -INFINITY;
@@ -186,13 +208,21 @@ struct GemvWarp {
         float part[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float k[DV];
-            load_kv(kt, r, lane, k);
-            float acc = 0.f;
+            if constexpr (FP8) {
+                static_assert(DV == 4, "e4m3 caches are built for head_dim 128");
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(at(kt, r, lane));
+                const float acc = dot2_f16_f32(e4m3x2_to_f16x2((uint16_t)w), qh[0], 0.f);
+                part[r] = dot2_f16_f32(e4m3x2_to_f16x2((uint16_t)(w >> 16)), qh[1], acc);
+            } else {
+                float k[DV];
+                load_kv(kt, r, lane, k);
+                float acc = 0.f;
 #pragma unroll
-            for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
-            part[r] = acc;
+                for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
+                part[r] = acc;
+            }
         }
+        if constexpr (FP8) scale_log2 *= qinv;
         // reduce-scatter the 16 partial sums over the 32 lanes: after the
         // rounds with masks 16, 8, 4, 2 and a final pairwise add, lane l
         // holds the full dot product of token l / 2
@@ -275,8 +305,13 @@ struct GemvWarp {
 // ---------------------------------------------------------------------------
 // Per-warp arithmetic, G >= 2: mma.sync m16n8k16 on the head group
 // ---------------------------------------------------------------------------
-template <typename T, int D, int NT>
+// E4 (e4m3 caches): K comes straight from the e4m3 tile and every product
+// runs on f16 (e4m3 values are exact in f16), whatever T is; the queries
+// are scaled by a power of two into f16 range and the scale is undone on
+// the scores.
+template <typename T, int D, int NT, bool E4 = false>
 struct MmaWarp {
+    using MT = typename std::conditional<E4, __half, T>::type;  // MMA operand type
     static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
     static constexpr int GP = NT * 8;  // heads held (padded)
     static constexpr bool kMma = true;
@@ -284,25 +319,76 @@ struct MmaWarp {
     float acc[KS][NT][4];              // O^T[d][head]
     float m[NT][2], l[NT][2];          // per lane: heads nt*8 + (lane&3)*2 + {0,1}
     float vs;                          // acc is in units of this V scale (e4m3 caches)
+    float qinv;                        // undoes the queries' power-of-two scale
 
     __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
         const int G = p.group;
         const T* qbase = static_cast<const T*>(p.query) +
                          ((int64_t)s * p.num_q_heads + (int64_t)kvh * G) * D;
+        if constexpr (E4) {
+            // k-step kk of head h holds dims 16kk + 4j .. 16kk + 4j + 3 in
+            // the lane with j = lane & 3: the order the e4m3 K fragments
+            // arrive in (see tile)
+            float qv[KS][NT][4];
+            float mx = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int h = nt * 8 + (lane >> 2);
+            for (int nt = 0; nt < NT; ++nt) {
+                const int h = nt * 8 + (lane >> 2);
 #pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                if (h < G) {
-                    const T* qrow = qbase + (int64_t)h * D + kk * 16 + (lane & 3) * 2;
-                    qf[kk][nt][0] = *reinterpret_cast<const uint32_t*>(qrow);
-                    qf[kk][nt][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
-                } else {
-                    qf[kk][nt][0] = 0u;
-                    qf[kk][nt][1] = 0u;
+                for (int kk = 0; kk < KS; ++kk) {
+                    if (h < G) {
+                        const uint2 w = *reinterpret_cast<const uint2*>(
+                            qbase + (int64_t)h * D + kk * 16 + (lane & 3) * 4);
+                        const float2 a = Storage<T>::to_float2(w.x), b = Storage<T>::to_float2(w.y);
+                        qv[kk][nt][0] = a.x;
+                        qv[kk][nt][1] = a.y;
+                        qv[kk][nt][2] = b.x;
+                        qv[kk][nt][3] = b.y;
+                    } else {
+                        qv[kk][nt][0] = qv[kk][nt][1] = qv[kk][nt][2] = qv[kk][nt][3] = 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fabsf(qv[kk][nt][i]));
                 }
             }
+#pragma unroll
+            for (int x = 1; x < 32; x <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, x));
+            // largest |q| into [2^14, 2^15): below f16's maximum, and every
+            // value within 2^29 of it keeps its bits
+            int ex = 0;
+            frexpf(mx, &ex);
+            const int sh = mx > 0.f ? max(-120, min(120, 15 - ex)) : 0;
+            const float qs = ldexpf(1.f, sh);
+            qinv = ldexpf(1.f, -sh);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    qf[kk][nt][0] = Storage<__half>::from_float2(qv[kk][nt][0] * qs,
+                                                                 qv[kk][nt][1] * qs);
+                    qf[kk][nt][1] = Storage<__half>::from_float2(qv[kk][nt][2] * qs,
+                                                                 qv[kk][nt][3] * qs);
+                }
+        } else {
+            qinv = 1.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int h = nt * 8 + (lane >> 2);
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    if (h < G) {
+                        const T* qrow = qbase + (int64_t)h * D + kk * 16 + (lane & 3) * 2;
+                        qf[kk][nt][0] = *reinterpret_cast<const uint32_t*>(qrow);
+                        qf[kk][nt][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+                    } else {
+                        qf[kk][nt][0] = 0u;
+                        qf[kk][nt][1] = 0u;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
             m[nt][0] = m[nt][1] = -INFINITY;
             l[nt][0] = l[nt][1] = 0.f;
             vs = 1.f;
@@ -330,19 +416,50 @@ struct MmaWarp {
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) sacc[nt][i] = sacc2[nt][i] = 0.f;
+        if constexpr (E4) {
+            // kt is the e4m3 tile (16 rows of 128 codes, 16-byte chunks
+            // swizzled).  One ldmatrix (read as 16-bit pairs) gives the lane
+            // codes 4j .. 4j+3 of chunks 2pp and 2pp + 1 for rows g and
+            // g + 8; converted pairwise to f16x2 they are the A fragments of
+            // k-steps 2pp and 2pp + 1 with the dims of each k-step in the
+            // order init gave the queries.
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            uint32_t a[4];
-            const int row = (lane & 7) + (j & 1) * 8;
-            ldmatrix_x4(a, kbase + swz(row, kk * 2 + (j >> 1)));
+            for (int pp = 0; pp < KS / 2; ++pp) {
+                uint32_t r[4];
+                const int row = (lane & 7) + (j & 1) * 8;
+                const int chunk = 2 * pp + (j >> 1);
+                ldmatrix_x4(r, kbase + row * 128 + ((chunk ^ (row & 7)) << 4));
+                const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)r[0]),
+                                        e4m3x2_to_f16x2((uint16_t)r[1]),
+                                        e4m3x2_to_f16x2((uint16_t)(r[0] >> 16)),
+                                        e4m3x2_to_f16x2((uint16_t)(r[1] >> 16))};
+                const uint32_t a1[4] = {e4m3x2_to_f16x2((uint16_t)r[2]),
+                                        e4m3x2_to_f16x2((uint16_t)r[3]),
+                                        e4m3x2_to_f16x2((uint16_t)(r[2] >> 16)),
+                                        e4m3x2_to_f16x2((uint16_t)(r[3] >> 16))};
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                if (kk & 1)
-                    Mma<T>::m16n8k16(sacc2[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
-                else
-                    Mma<T>::m16n8k16(sacc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                for (int nt = 0; nt < NT; ++nt) {
+                    Mma<MT>::m16n8k16(sacc[nt], a0, qf[2 * pp][nt][0], qf[2 * pp][nt][1]);
+                    Mma<MT>::m16n8k16(sacc2[nt], a1, qf[2 * pp + 1][nt][0],
+                                      qf[2 * pp + 1][nt][1]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                uint32_t a[4];
+                const int row = (lane & 7) + (j & 1) * 8;
+                ldmatrix_x4(a, kbase + swz(row, kk * 2 + (j >> 1)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (kk & 1)
+                        Mma<MT>::m16n8k16(sacc2[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                    else
+                        Mma<MT>::m16n8k16(sacc[nt], a, qf[kk][nt][0], qf[kk][nt][1]);
+                }
             }
         }
+        scale_log2 *= qinv;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -385,13 +502,13 @@ struct MmaWarp {
             // B-fragments.  P is split into a rounded high part and the
             // rounded remainder, so the PV product sees P to ~16 bits of
             // mantissa instead of the 8 of one bf16 rounding.
-            const uint32_t h01 = Storage<T>::from_float2(p0, p1);
-            const uint32_t h23 = Storage<T>::from_float2(p2, p3);
-            const float2 b01 = Storage<T>::to_float2(h01), b23 = Storage<T>::to_float2(h23);
+            const uint32_t h01 = Storage<MT>::from_float2(p0, p1);
+            const uint32_t h23 = Storage<MT>::from_float2(p2, p3);
+            const float2 b01 = Storage<MT>::to_float2(h01), b23 = Storage<MT>::to_float2(h23);
             pb[nt][0] = movmatrix_trans(h01);
             pb[nt][1] = movmatrix_trans(h23);
-            pl[nt][0] = movmatrix_trans(Storage<T>::from_float2(p0 - b01.x, p1 - b01.y));
-            pl[nt][1] = movmatrix_trans(Storage<T>::from_float2(p2 - b23.x, p3 - b23.y));
+            pl[nt][0] = movmatrix_trans(Storage<MT>::from_float2(p0 - b01.x, p1 - b01.y));
+            pl[nt][1] = movmatrix_trans(Storage<MT>::from_float2(p2 - b23.x, p3 - b23.y));
         }
         // O^T[d][head] += V^T P^T over the 16 tokens
 #pragma unroll
@@ -401,8 +518,8 @@ struct MmaWarp {
             ldmatrix_x4_trans(a, vbase + swz(row, mt * 2 + (j & 1)));
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                Mma<T>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
-                Mma<T>::m16n8k16(acc[mt][nt], a, pl[nt][0], pl[nt][1]);
+                Mma<MT>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
+                Mma<MT>::m16n8k16(acc[mt][nt], a, pl[nt][0], pl[nt][1]);
             }
         }
     }
@@ -451,18 +568,18 @@ struct MmaWarp {
 
 // ---------------------------------------------------------------------------
 // Shared-memory plan of one CTA: per warp a ring of stages (the K and V tiles
-// as stored), then, for e4m3 caches on the tensor-core path, a 16-bit copy of
-// the current tile per warp; then the mbarriers, the per-stage
+// as stored), then, for e4m3 caches on the tensor-core path, an f16 copy of
+// the current V tile per warp; then the mbarriers, the per-stage
 // dequantisation scales (e4m3) and the partition's table slice.  The ring and
 // the copies are reused by the epilogue once every load has landed.
 // ---------------------------------------------------------------------------
 template <int D, bool FP8, bool MMA>
 struct Plan {
     static_assert(!FP8 || D == 128, "e4m3 caches are built for head_dim 128");
-    static constexpr int kStages = FP8 ? (MMA ? 2 : 4) : Geom<D>::kStages;
+    static constexpr int kStages = FP8 ? (MMA ? 3 : 4) : Geom<D>::kStages;
     static constexpr int kTileBytes = FP8 ? kTile * D : Geom<D>::kKBytes;  // K (or V) as stored
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kScratchBytes = (FP8 && MMA) ? Geom<D>::kStageBytes : 0;
+    static constexpr int kScratchBytes = (FP8 && MMA) ? Geom<D>::kKBytes : 0;  // f16 V tile
     static constexpr size_t kRing = (size_t)kWarps * kStages * kStageBytes;
     static constexpr size_t kEpilogue = kRing + (size_t)kWarps * kScratchBytes;
     static constexpr size_t kBarOff = kEpilogue;
@@ -628,11 +745,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             kscale = my_scales[st * 8 + si];
             vscale = my_scales[st * 8 + 4 + si];
             if constexpr (Warp::kMma) {
-                widen_fp8_tile<T>(kt, my_wide, lane);
-                widen_fp8_tile<T>(vt, my_wide + Gm::kKBytes, lane);
+                // K is read from the e4m3 tile itself; V is transposed by
+                // ldmatrix.trans, which moves 16-bit elements, so it is
+                // widened to f16 first
+                widen_fp8_tile<__half>(vt, my_wide, lane);
                 __syncwarp();
-                kt = my_wide;
-                vt = my_wide + Gm::kKBytes;
+                vt = my_wide;
             }
         }
         if (valid < kTile) {
@@ -910,8 +1028,9 @@ int dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decod
     if (p.group == 1)
         return launch_decode<T, D, GemvWarp<T, D, FP8>, FP8>(kmap, vmap, p, num_kv_heads, stream);
     if (p.group <= 8)
-        return launch_decode<T, D, MmaWarp<T, D, 1>, FP8>(kmap, vmap, p, num_kv_heads, stream);
-    return launch_decode<T, D, MmaWarp<T, D, 2>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+        return launch_decode<T, D, MmaWarp<T, D, 1, FP8>, FP8>(kmap, vmap, p, num_kv_heads,
+                                                               stream);
+    return launch_decode<T, D, MmaWarp<T, D, 2, FP8>, FP8>(kmap, vmap, p, num_kv_heads, stream);
 }
 
 // 4-D view of one e4m3 cache: (head_dim codes, kv head, slot, block), boxes
