@@ -585,6 +585,286 @@ def run_pkv(args, spec, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+SWAP_WORKLOAD = "swap_7b_s256_q64_h32_d128_bs16_bf16"
+
+
+def host_link_peak(dev, nbytes=1 << 30):
+    """Copy-engine bandwidth of one large pinned <-> device copy each way
+    (cudaMemcpyAsync through torch), GB/s: the host link's practical peak."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, (dst, src) in (("d2h", (h, d)), ("h2d", (d, h))):
+        dst.copy_(src, non_blocking=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for _ in range(3):
+            a.record()
+            dst.copy_(src, non_blocking=True)
+            b.record()
+            torch.cuda.synchronize(dev)
+            times.append(a.elapsed_time(b))
+        out[name] = nbytes / (min(times) * 1e-3) / 1e9
+    del h, d
+    return out
+
+
+def run_swap(args, world, rank, local):
+    """Block swap of the 7B-shaped batch: each step swaps the first 64 of
+    the 256 sequences out to pinned host memory and back in
+    (pkv_seq_swap_out / _in on the host pool, one pkv_swap_blocks launch
+    per direction).  `value` is the bytes moved (K and V blocks, both
+    directions) over the swap kernels' device time; the roofline peak is
+    the copy engine's bandwidth for one 1 GiB pinned copy each way, measured
+    in the same run.  `e2e` times PagedKVCache.swap_out / swap_in from the
+    host, pool bookkeeping and pair upload included."""
+    from paged_kv_cache_337_b200 import _abi
+    from paged_kv_cache_337_b200 import workloads as W
+    from paged_kv_cache_337_b200.cache import PagedKVCache
+
+    spec = W.SPECS["7b_s256_h32_d128_bs16_bf16"]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _abi.lib()
+    gen = torch.Generator("cpu").manual_seed(spec.seed)
+    lens = W.draw_lens(spec, gen).tolist()
+    nb = W.pool_size(spec, lens)
+    order = torch.randperm(nb, generator=gen, dtype=torch.int64).to(torch.int32)
+    S, Hq, Hkv, D, bs = (spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim,
+                         spec.block_size)
+    moved = list(range(64))
+    host_blocks = sum(-(-lens[s] // bs) for s in moved)
+    cache = PagedKVCache(nb, bs, Hq, Hkv, D, spec.torch_dtype, dev, spec.max_blocks_per_seq,
+                         0, free_order=order.tolist(), scale=spec.scale)
+    W.fill_device_cache_(cache.key_cache, spec.seed * 10 + 2 * rank)
+    W.fill_device_cache_(cache.value_cache, spec.seed * 10 + 2 * rank + 1)
+    cache.enable_swap(host_blocks)
+    for s in range(S):
+        cache.add_sequence(s, lens[s])
+    block_bytes = bs * Hkv * D * cache.key_cache.element_size()
+    stream = torch.cuda.Stream(dev)
+    err = cache.dev_error
+    kc, vc, hk, hv = cache.key_cache, cache.value_cache, cache.host_key_cache, cache.host_value_cache
+
+    def step(ev=None):
+        pairs = torch.cat([cache.pool.swap_out(s) for s in moved]).to(dev)
+        if ev:
+            ev[0].record(stream)
+        _abi.pkv_swap_blocks(kc, vc, hk, hv, pairs, dev_error=err, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        pairs = torch.cat([cache.pool.swap_in(s) for s in moved]).to(dev)
+        if ev:
+            ev[2].record(stream)
+        _abi.pkv_swap_blocks(hk, hv, kc, vc, pairs, dev_error=err, stream=stream)
+        if ev:
+            ev[3].record(stream)
+        return 2 * pairs.shape[0] * 2 * block_bytes
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    total = 0
+    for i in range(K):
+        total += step(evs[i])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clock_info = clocks.stop() if clocks else None
+    out_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    in_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    cache.check_errors()
+    t_max = max_over_ranks(out_ms + in_ms, world, dev)
+    value = sum_over_ranks(total, world, dev) / (t_max * 1e-3) / 1e9
+    per_dir = total / 2
+    out_gbs = per_dir / (out_ms * 1e-3) / 1e9
+    in_gbs = per_dir / (in_ms * 1e-3) / 1e9
+    step_bytes = total // K  # both directions, one step
+
+    # end to end through the driver: pool bookkeeping + pair upload + kernel
+    e2e_steps = min(K, 10)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        cache.swap_out(moved, stream=stream)
+        cache.swap_in(moved, stream=stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
+    cache.check_errors()
+    peak = host_link_peak(dev)
+    if rank == 0:
+        peak_both = 2 / (1 / peak["d2h"] + 1 / peak["h2d"])  # same bytes each way
+        line = {
+            "metric": "block swap GB/s (K/V blocks to pinned host memory and back)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(t_max / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": SWAP_WORKLOAD, "num_seqs": S, "swapped_seqs": len(moved),
+                       "blocks_per_direction": int(step_bytes // (2 * 2 * block_bytes)),
+                       "block_bytes_kv": 2 * block_bytes, "pool_blocks": nb,
+                       "step": "swap-out of 64 sequences then swap-in (new GPU blocks)"},
+            "swap_out_gbs": round(out_gbs, 2), "swap_in_gbs": round(in_gbs, 2),
+            "roofline": {"bound": "host-link", "achieved": round(value, 2),
+                         "peak": round(peak_both, 2), "unit": "GB/s",
+                         "frac": round(value / peak_both, 4), "traffic": None,
+                         "kernel": "swap_blocks_kernel",
+                         "peak_source": "measured in this run: 1 GiB pinned copy, "
+                                        "d2h %.1f / h2d %.1f GB/s" % (peak["d2h"], peak["h2d"])},
+            "e2e": {"value": round(e2e_steps * step_bytes / e2e_s / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(step_bytes // 2),
+                    "d2h_bytes_per_step": int(step_bytes // 2)},
+            "gpu_launches": 2 * K, "clocks": clock_info, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+
+
+PREFILL_WORKLOAD = "prefill_s8_l2048_hq32_hkv8_d128_bs16_bf16"
+
+
+def prefill_flops(lens, n, Hq, D):
+    """Algorithmic FLOPs of causal attention: for each query row at
+    position p, S (p + 1 dot products) and P V (p + 1 axpys), 2 * D each."""
+    f = 0
+    for L, k in zip(lens, n):
+        first = L - k  # positions L - k .. L - 1
+        keys = k * (first + 1) + k * (k - 1) // 2
+        f += 4 * D * Hq * keys
+    return f
+
+
+def run_prefill(args, world, rank, local):
+    """Paged prefill of 8 prompts of 2048 tokens (Hq 32 / Hkv 8, head_dim
+    128, block size 16, bf16) over scattered blocks: each step writes the
+    prompts' K/V into their slots (pkv_write_slots) and runs causal paged
+    attention (pkv_prefill_attention).  `value` is the attention's
+    algorithmic TFLOP/s (S = QK^T and PV, causal) over its device time."""
+    import numpy as np
+
+    from paged_kv_cache_337_b200 import _abi
+    from paged_kv_cache_337_b200.cache import PagedKVCache
+
+    S, L, Hq, Hkv, D, bs = 8, 2048, 32, 8, 128, 16
+    dt = torch.bfloat16
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _abi.lib()
+    gen = torch.Generator("cpu").manual_seed(2000 + rank)
+    lens = [L] * S
+    nb = int(math.ceil(1.1 * S * (L // bs)))
+    order = torch.randperm(nb, generator=gen).tolist()
+    cache = PagedKVCache(nb, bs, Hq, Hkv, D, dt, dev, L // bs, 0, free_order=order,
+                         scale=1.0 / math.sqrt(D))
+    for s in range(S):
+        cache.pool.add(s, L)
+    slots = torch.cat([cache.pool.slot_mapping(s, 0, L) for s in range(S)]).to(dev)
+    tables, tl = cache.pool.block_tables(list(range(S)), L // bs)
+    tables, tl = tables.to(dev), tl.to(dev)
+    qs = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    dgen = torch.Generator(dev).manual_seed(3000 + rank)
+    T = S * L
+    q = torch.randn((T, Hq, D), generator=dgen, device=dev).to(dt)
+    k = torch.randn((T, Hkv, D), generator=dgen, device=dev).to(dt)
+    v = torch.randn((T, Hkv, D), generator=dgen, device=dev).to(dt)
+    out = torch.empty_like(q)
+    stream = torch.cuda.Stream(dev)
+    err = cache.dev_error
+    flops = prefill_flops(lens, lens, Hq, D)
+
+    def step(ev=None):
+        _abi.pkv_write_slots(k, v, cache.key_cache, cache.value_cache, slots, dev_error=err,
+                             stream=stream)
+        if ev:
+            ev[0].record(stream)
+        _abi.pkv_prefill_attention(out, q, cache.key_cache, cache.value_cache, tables, tl, qs, L,
+                                   cache.scale, dev_error=err, stream=stream)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clock_info = clocks.stop() if clocks else None
+    cache.check_errors()
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    t_max = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    value = sum_over_ranks(flops * K, world, dev) / (t_max * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    peak = measured_tensor_peak()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import reference as ref
+
+        n_rows = 64  # the last 64 rows of one prompt: the heaviest rows
+        hq = q[L - n_rows:L].cpu()
+        sub = torch.tensor([0, n_rows], dtype=torch.int32)
+        kc, vc = cache.key_cache.cpu(), cache.value_cache.cpu()
+        tc = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - tc < 10.0:
+            ref.prefill_attention(hq, kc, vc, tables[:1].cpu(), tl[:1].cpu(), sub, cache.scale,
+                                  "bf16", Hkv, bs)
+            reps += 1
+        secs = time.perf_counter() - tc
+        cpu = {"value": round(reps * prefill_flops([L], [n_rows], Hq, D) / secs / 1e12, 6),
+               "unit": "TFLOP/s", "cores": ref.max_threads(), "kind": "oracle",
+               "sample": "last %d rows of one 2048-token prompt (all 32 heads), %d times, "
+                         "%.1f s" % (n_rows, reps, secs)}
+    if rank == 0:
+        line = {
+            "metric": "paged prefill attention TFLOP/s (causal, algorithmic)",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(t_max / K, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": PREFILL_WORKLOAD, "num_seqs": S, "prompt_len": L,
+                       "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                       "block_size": bs, "pool_blocks": nb,
+                       "step": "prompt K/V slot write + causal paged prefill attention",
+                       "l2": "K/V %.2f GB, Q %.2f GB per step" % (
+                           2 * T * Hkv * D * 2 / 1e9, T * Hq * D * 2 / 1e9)},
+            "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
+                         "peak": peak[0], "unit": "TFLOP/s",
+                         "frac": round(attn_tflops / peak[0], 4), "traffic": None,
+                         "kernel": "paged_prefill_kernel", "peak_source": peak[1]},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 burst)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
 def run_shared_prefix(args, world, rank, local):
     """The shared-prefix parallel-sampling workload (16 prompts x 8 samples,
     1024-token prefix): the fork step (112 copy-on-write copies + slot write
@@ -708,6 +988,22 @@ def main():
     args = parse_args()
     from paged_kv_cache_337_b200 import workloads as W
 
+    if args.workload == PREFILL_WORKLOAD:
+        world, rank, local = dist_setup()
+        try:
+            run_prefill(args, world, rank, local)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+        return
+    if args.workload == SWAP_WORKLOAD:
+        world, rank, local = dist_setup()
+        try:
+            run_swap(args, world, rank, local)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+        return
     if args.workload == W.SHARED_PREFIX.name:
         world, rank, local = dist_setup()
         try:

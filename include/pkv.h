@@ -118,6 +118,27 @@ PKV_API int pkv_copy_blocks(void* key_cache, void* value_cache,
                     int64_t block_stride, pkv_dtype dtype, int32_t* dev_error,
                     cudaStream_t stream);
 
+/*
+ * pkv_copy_blocks over every layer of a multi-layer cache in one launch.  A
+ * physical block id names the block in all layers ("Paged KV" wiki page,
+ * 初始化阶段: a block holds K and V of every layer), so one copy-on-write
+ * pair from the pool is copied in each layer.
+ *
+ *   key_caches, value_caches  device arrays of num_layers device pointers
+ *                (layer l's K and V caches, each 16-byte aligned, all with
+ *                the same geometry)
+ *   block_pairs  device int32 [num_pairs, 2]; rules and errors as for
+ *                pkv_copy_blocks
+ *   block_bytes, block_stride_bytes
+ *                one block of one cache and the distance between blocks,
+ *                in bytes (multiples of 16; any element type, e4m3 too)
+ */
+PKV_API int pkv_copy_blocks_layers(void* const* key_caches, void* const* value_caches,
+                                   int num_layers, const int32_t* block_pairs, int num_pairs,
+                                   int num_blocks, int64_t block_bytes,
+                                   int64_t block_stride_bytes, int32_t* dev_error,
+                                   cudaStream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Paged decode attention                                                  */
 /* ---------------------------------------------------------------------- */
@@ -176,6 +197,39 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
                          int partition_size, void* workspace,
                          size_t workspace_bytes, pkv_dtype dtype,
                          int32_t* dev_error, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Paged prefill attention                                                 */
+/* ---------------------------------------------------------------------- */
+/*
+ * Causal attention of a prompt (or a later chunk of one) over the paged
+ * cache ("Paged KV" wiki page, 实现原理 / 运行阶段: prefill takes blocks in
+ * order and fills them with the prompt's K/V — pkv_write_slots with the
+ * prompt's slots — and its tokens then attend through the same Block
+ * Table).  Sequence s owns query rows query_start[s] .. query_start[s+1]-1,
+ * n_s of them: the last n_s of its L = context_lens[s] cached tokens.  Row
+ * query_start[s] + i is token p = L - n_s + i, and for each query head h
+ * (KV head h / (num_q_heads / num_kv_heads)):
+ *     out[row, h] = sum_{t <= p} softmax_t(scale * <query[row, h], K_t>) V_t.
+ *
+ *   out, query       device [total rows, num_q_heads, head_dim], dtype
+ *   block_tables     device int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens     device int32 [num_seqs]: L, the chunk's tokens included
+ *   query_start      device int32 [num_seqs + 1], non-decreasing from 0
+ *   max_query_len    host bound on every n_s: it sizes the grid
+ * A sequence with n_s > L, n_s > max_query_len or L > max_blocks_per_seq *
+ * block_size is reported (PKV_DEVERR_CONTEXT_LEN) and its rows are left
+ * unwritten.  Built for head_dim 128 and block_size a multiple of 16;
+ * f16 or bf16.  Caches 16-byte aligned, block_stride in elements.
+ */
+PKV_API int pkv_prefill_attention(void* out, const void* query, const void* key_cache,
+                                  const void* value_cache, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* context_lens,
+                                  const int32_t* query_start, int num_seqs, int max_query_len,
+                                  int num_q_heads, int num_kv_heads, int head_dim,
+                                  int num_blocks, int block_size, int64_t block_stride,
+                                  float scale, pkv_dtype dtype, int32_t* dev_error,
+                                  cudaStream_t stream);
 
 /*
  * Scratch built into the library for pkv_decode_attention_noalloc: the
@@ -361,6 +415,80 @@ PKV_API int pkv_pool_free_list(const pkv_pool* pool, int32_t* out, int cap, int*
 
 /* Refcount of a block (number of tables holding it), or a negative status. */
 PKV_API int pkv_block_refcount(const pkv_pool* pool, int block);
+
+/* ---------------------------------------------------------------------- */
+/* Block swapping to pinned host memory                                    */
+/* ---------------------------------------------------------------------- */
+/*
+ * When GPU memory runs short, a sequence's KV blocks can move to CPU memory
+ * and come back when it runs again ("PagedAttention 动态内存分页" page,
+ * 动态块分配与回收; 性能监控要点 names the swap bandwidth as a figure to
+ * watch).  The pool keeps a second stack of host block ids; the caller owns
+ * the host caches those ids index (pinned, e.g. cudaHostAlloc) and moves the
+ * bytes with pkv_swap_blocks.
+ *
+ * Rules: a swap moves one whole sequence, in table order.  Swap-out gives
+ * each block a host block (pair (gpu, host)) and then drops the sequence's
+ * reference to the GPU block, which returns to the pool at refcount 0 (a
+ * block still shared with a resident sequence stays for it).  Swap-in gives
+ * each host block a GPU block (pair (host, gpu)) and returns the host block.
+ * Either one that runs out of blocks changes nothing (PKV_ERR_OOM).  While
+ * swapped out, a sequence cannot be appended to, forked, or listed by
+ * pkv_pool_block_tables / pkv_seq_slot_mapping (PKV_ERR_INVALID);
+ * pkv_seq_block_table lists its host blocks; pkv_seq_free returns them.
+ */
+
+/* Makes the host pool (once): host blocks 0 .. num_host_blocks-1, handed out
+ * 0, 1, ... first, freed blocks reused last-in first-out. */
+PKV_API int pkv_pool_set_host_blocks(pkv_pool* pool, int num_host_blocks);
+
+/* Swap-out of a resident sequence.  pairs (host int32, capacity cap pairs)
+ * receives (gpu block, host block) per block in table order, *num_pairs
+ * their count (PKV_ERR_INVALID, nothing changed, if cap is too small). */
+PKV_API int pkv_seq_swap_out(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int cap,
+                             int* num_pairs);
+
+/* Swap-in of a swapped-out sequence: pairs receives (host block, gpu block). */
+PKV_API int pkv_seq_swap_in(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int cap,
+                            int* num_pairs);
+
+PKV_API int pkv_seq_is_swapped(const pkv_pool* pool, int64_t seq_id, int* swapped);
+PKV_API int pkv_pool_num_free_host(const pkv_pool* pool);
+
+/* The host free stack from bottom to top (the next block taken is the last). */
+PKV_API int pkv_pool_host_free_list(const pkv_pool* pool, int32_t* out, int cap, int* n);
+
+/* Refcount of a host block (1 while a swapped sequence holds it, else 0). */
+PKV_API int pkv_host_block_refcount(const pkv_pool* pool, int block);
+
+/*
+ * Copies whole blocks from one pool to another: for each pair (src, dst),
+ * block dst of dst_key (and dst_value) becomes block src of src_key (and
+ * src_value).  One side is the GPU cache, the other a host cache in pinned
+ * memory mapped for the device (cudaHostAlloc; the library passes the
+ * kernel the mapping cudaPointerGetAttributes reports).  Swap-out copies
+ * GPU -> host with the pairs of pkv_seq_swap_out, swap-in host -> GPU with
+ * those of pkv_seq_swap_in.  The kernel reads or writes host memory over
+ * the host link directly, one launch for all pairs.
+ *
+ *   src_value, dst_value  both NULL to copy one pool (e.g. the fp32 scales
+ *                  of an e4m3 cache: block_bytes = num_kv_heads * 4)
+ *   block_pairs    int32 [num_pairs, 2] in device memory or mapped pinned
+ *                  host memory.  Pairs run concurrently: destinations
+ *                  distinct.  A pair outside [0, src_num_blocks) x
+ *                  [0, dst_num_blocks) is skipped and reported
+ *                  (PKV_DEVERR_PAIR).
+ *   block_bytes, src_block_stride, dst_block_stride
+ *                  in bytes, multiples of 4 (16-byte vectors are used when
+ *                  every pointer, size and stride allows)
+ * Pageable host memory, or host memory without a device mapping, is
+ * rejected (PKV_ERR_INVALID) before anything is launched.
+ */
+PKV_API int pkv_swap_blocks(const void* src_key, const void* src_value, void* dst_key,
+                            void* dst_value, const int32_t* block_pairs, int num_pairs,
+                            int src_num_blocks, int dst_num_blocks, int64_t block_bytes,
+                            int64_t src_block_stride, int64_t dst_block_stride,
+                            int32_t* dev_error, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* Sizing and diagnostics                                                  */

@@ -38,11 +38,14 @@ _p, _i, _i64, _sz, _f = C.c_void_p, C.c_int, C.c_int64, C.c_size_t, C.c_float
 SIGNATURES = {
     "pkv_write_slots": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p, _p]),
     "pkv_copy_blocks": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p, _p]),
+    "pkv_copy_blocks_layers": (_i, [_p, _p, _i, _p, _i, _i, _i64, _i64, _p, _p]),
     "pkv_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "pkv_decode_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                   _i64, _f, _i, _p, _sz, _i, _p, _p]),
     "pkv_decode_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
                                           _i, _i64, _f, _i, _i, _p, _p]),
+    "pkv_prefill_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i,
+                                   _i64, _f, _i, _p, _p]),
     "pkv_write_slots_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _i, _p,
                                  _p]),
     "pkv_copy_blocks_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _p, _p]),
@@ -64,6 +67,14 @@ SIGNATURES = {
     "pkv_pool_block_size": (_i, [_p]),
     "pkv_pool_free_list": (_i, [_p, _p, _i, _p]),
     "pkv_block_refcount": (_i, [_p, _i]),
+    "pkv_pool_set_host_blocks": (_i, [_p, _i]),
+    "pkv_seq_swap_out": (_i, [_p, _i64, _p, _i, _p]),
+    "pkv_seq_swap_in": (_i, [_p, _i64, _p, _i, _p]),
+    "pkv_seq_is_swapped": (_i, [_p, _i64, _p]),
+    "pkv_pool_num_free_host": (_i, [_p]),
+    "pkv_pool_host_free_list": (_i, [_p, _p, _i, _p]),
+    "pkv_host_block_refcount": (_i, [_p, _i]),
+    "pkv_swap_blocks": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i64, _i64, _i64, _p, _p]),
     "pkv_block_bytes": (_i64, [_i, _i, _i, _i, _i]),
     "pkv_selftest_bounded_wait": (_i, [_p, _i, _p]),
     "pkv_status_string": (C.c_char_p, [_i]),
@@ -197,6 +208,37 @@ def pkv_copy_blocks(key_cache, value_cache, block_pairs, dev_error=None, stream=
     _check(st, "pkv_copy_blocks")
 
 
+def layer_pointers(caches, device):
+    """A device int64 array of the caches' data pointers (one per layer),
+    for pkv_copy_blocks_layers."""
+    return torch.tensor([c.data_ptr() for c in caches], dtype=torch.int64, device=device)
+
+
+def pkv_copy_blocks_layers(key_caches, value_caches, block_pairs, dev_error=None, stream=None,
+                           key_ptrs=None, value_ptrs=None):
+    """Copy whole blocks in every layer for each (src, dst) row of int32
+    block_pairs [n, 2]; key_caches / value_caches are per-layer
+    [NB, bs, Hkv, D] caches of one geometry.  key_ptrs / value_ptrs may pass
+    prebuilt layer_pointers arrays."""
+    if len(key_caches) != len(value_caches) or not key_caches:
+        raise ValueError("one K and one V cache per layer")
+    _on_device("pkv_copy_blocks_layers", *key_caches, *value_caches, block_pairs, dev_error)
+    geom = _cache_geometry(key_caches[0])
+    for c in list(key_caches) + list(value_caches):
+        if _cache_geometry(c) != geom or c.dtype != key_caches[0].dtype:
+            raise ValueError("pkv_copy_blocks_layers: every layer's caches must match")
+    _need(block_pairs, torch.int32, "block_pairs")
+    nb, bs, hkv, d, stride = geom
+    es = key_caches[0].element_size()
+    dev = key_caches[0].device
+    kp = key_ptrs if key_ptrs is not None else layer_pointers(key_caches, dev)
+    vp = value_ptrs if value_ptrs is not None else layer_pointers(value_caches, dev)
+    st = lib().pkv_copy_blocks_layers(_ptr(kp), _ptr(vp), len(key_caches), _ptr(block_pairs),
+                                      block_pairs.numel() // 2, nb, bs * hkv * d * es,
+                                      stride * es, _ptr(dev_error), _stream(stream, dev))
+    _check(st, "pkv_copy_blocks_layers")
+
+
 def pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len, partition_size,
                                head_dim):
     return int(lib().pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len,
@@ -233,6 +275,35 @@ def pkv_decode_attention(out, query, key_cache, value_cache, block_tables, conte
         float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
         _ptr(dev_error), _stream(stream, query.device))
     _check(st, "pkv_decode_attention")
+
+
+def pkv_prefill_attention(out, query, key_cache, value_cache, block_tables, context_lens,
+                          query_start, max_query_len, scale, dev_error=None, stream=None):
+    """Causal paged attention of each sequence's last n_s tokens: query/out
+    [T, Hq, D] (rows query_start[s] .. query_start[s+1]-1 for sequence s),
+    int32 block_tables [S, MB], context_lens [S], query_start [S + 1]."""
+    _on_device("pkv_prefill_attention", out, query, key_cache, value_cache, block_tables,
+               context_lens, query_start, dev_error)
+    nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
+    if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
+        raise ValueError("key_cache and value_cache differ in geometry")
+    T, hq, dq = query.shape
+    if dq != d or out.shape != query.shape:
+        raise ValueError("query/out must be [rows, num_q_heads, head_dim]")
+    _need(query, key_cache.dtype, "query")
+    _need(out, key_cache.dtype, "out")
+    _need(block_tables, torch.int32, "block_tables")
+    _need(context_lens, torch.int32, "context_lens")
+    _need(query_start, torch.int32, "query_start")
+    S = context_lens.numel()
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or query_start.numel() != S + 1:
+        raise ValueError("block_tables [S, MB], context_lens [S], query_start [S + 1]")
+    st = lib().pkv_prefill_attention(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), _ptr(query_start), S, int(max_query_len), hq,
+        hkv, d, nb, bs, bstride, float(scale), _dtype(query), _ptr(dev_error),
+        _stream(stream, query.device))
+    _check(st, "pkv_prefill_attention")
 
 
 def pkv_decode_attention_noalloc(out, query, key_cache, value_cache, block_tables,
@@ -499,3 +570,95 @@ class BlockPool:
 
     def refcounts(self):
         return [self.refcount(b) for b in range(self.num_blocks)]
+
+    # -- swapping to host blocks ------------------------------------------
+    def set_host_blocks(self, num_host_blocks):
+        _check(lib().pkv_pool_set_host_blocks(self._h, num_host_blocks),
+               "pkv_pool_set_host_blocks")
+        self.num_host_blocks = num_host_blocks
+
+    def _swap(self, fn, name, seq_id):
+        n = C.c_int()
+        cap = max(self.num_blocks, 1)
+        pairs = torch.empty((cap, 2), dtype=torch.int32)
+        _check(fn(self._h, seq_id, _ptr(pairs), cap, C.byref(n)), name)
+        return pairs[:n.value]
+
+    def swap_out(self, seq_id):
+        """int32 [n, 2] (gpu block, host block) pairs, in table order."""
+        return self._swap(lib().pkv_seq_swap_out, "pkv_seq_swap_out", seq_id)
+
+    def swap_in(self, seq_id):
+        """int32 [n, 2] (host block, gpu block) pairs, in table order."""
+        return self._swap(lib().pkv_seq_swap_in, "pkv_seq_swap_in", seq_id)
+
+    def is_swapped(self, seq_id):
+        v = C.c_int()
+        _check(lib().pkv_seq_is_swapped(self._h, seq_id, C.byref(v)), "pkv_seq_is_swapped")
+        return bool(v.value)
+
+    def num_free_host(self):
+        v = lib().pkv_pool_num_free_host(self._h)
+        if v < 0:
+            _check(v, "pkv_pool_num_free_host")
+        return v
+
+    def host_free_list(self):
+        cap = max(getattr(self, "num_host_blocks", 0), 1)
+        n = C.c_int()
+        buf = (C.c_int32 * cap)()
+        _check(lib().pkv_pool_host_free_list(self._h, buf, cap, C.byref(n)),
+               "pkv_pool_host_free_list")
+        return list(buf[:n.value])
+
+    def host_refcounts(self):
+        out = []
+        for h in range(getattr(self, "num_host_blocks", 0)):
+            v = lib().pkv_host_block_refcount(self._h, h)
+            if v < 0:
+                _check(v, "pkv_host_block_refcount")
+            out.append(v)
+        return out
+
+
+def _pool_geometry(name, t):
+    """(num_blocks, block_bytes, block_stride_bytes) of a [NB, ...] pool
+    whose blocks are contiguous."""
+    if t.dim() < 1:
+        raise ValueError("%s must be [num_blocks, ...]" % name)
+    nb = t.shape[0]
+    inner = t[0] if nb else t
+    if nb and not inner.is_contiguous():
+        raise ValueError("%s: each block must be contiguous" % name)
+    es = t.element_size()
+    block_bytes = (t.numel() // nb if nb else 0) * es
+    stride = t.stride(0) * es if nb > 1 else block_bytes
+    return nb, block_bytes, stride
+
+
+def pkv_swap_blocks(src_key, src_value, dst_key, dst_value, block_pairs, dev_error=None,
+                    stream=None):
+    """Copy blocks src -> dst for each (src, dst) row of int32 block_pairs
+    [n, 2] between a device pool and a pinned host pool ([NB, ...] tensors
+    of one block layout; src_value / dst_value may both be None)."""
+    if (src_value is None) != (dst_value is None):
+        raise ValueError("src_value and dst_value must both be given or both be None")
+    dev = next(t.device for t in (src_key, dst_key) if t.is_cuda)
+    for name, t in (("src_key", src_key), ("dst_key", dst_key), ("src_value", src_value),
+                    ("dst_value", dst_value)):
+        if t is not None and not t.is_cuda and not t.is_pinned():
+            raise ValueError("pkv_swap_blocks: %s must be a CUDA tensor or pinned" % name)
+    _need(block_pairs, torch.int32, "block_pairs")
+    snb, sbytes, sstride = _pool_geometry("src_key", src_key)
+    dnb, dbytes, dstride = _pool_geometry("dst_key", dst_key)
+    if sbytes != dbytes:
+        raise ValueError("pkv_swap_blocks: the pools' blocks differ in size")
+    if src_value is not None:
+        if (_pool_geometry("src_value", src_value) != (snb, sbytes, sstride)
+                or _pool_geometry("dst_value", dst_value) != (dnb, dbytes, dstride)):
+            raise ValueError("pkv_swap_blocks: K and V pools differ in geometry")
+    n = block_pairs.numel() // 2
+    st = lib().pkv_swap_blocks(_ptr(src_key), _ptr(src_value), _ptr(dst_key), _ptr(dst_value),
+                               _ptr(block_pairs), n, snb, dnb, sbytes, sstride, dstride,
+                               _ptr(dev_error), _stream(stream, dev))
+    _check(st, "pkv_swap_blocks")

@@ -235,6 +235,53 @@ class PagedKVCache:
             out = torch.empty_like(query)
         return self.launch_step(prep, query, key, value, out, stream=stream)
 
+    # -- swapping to pinned host memory -------------------------------------
+    def enable_swap(self, num_host_blocks):
+        """Host caches of num_host_blocks blocks in pinned memory (and the
+        pool's host block stack), for swap_out / swap_in."""
+        self.pool.set_host_blocks(num_host_blocks)
+        shape = (num_host_blocks,) + tuple(self.key_cache.shape[1:])
+        pin = dict(dtype=self.key_cache.dtype, pin_memory=True)
+        self.host_key_cache = torch.empty(shape, **pin)
+        self.host_value_cache = torch.empty(shape, **pin)
+        if self.fp8:
+            hs = dict(dtype=torch.float32, pin_memory=True)
+            self.host_k_scale = torch.empty((num_host_blocks, self.num_kv_heads), **hs)
+            self.host_v_scale = torch.empty((num_host_blocks, self.num_kv_heads), **hs)
+
+    def _swap(self, seq_ids, out, stream):
+        fn = self.pool.swap_out if out else self.pool.swap_in
+        pairs = [fn(s) for s in seq_ids]
+        pairs = torch.cat(pairs) if pairs else torch.empty((0, 2), dtype=torch.int32)
+        if pairs.numel() == 0:
+            return 0
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            d_pairs = pairs.pin_memory().to(self.device, non_blocking=True)
+        dev = (self.key_cache, self.value_cache)
+        host = (self.host_key_cache, self.host_value_cache)
+        src, dst = (dev, host) if out else (host, dev)
+        _abi.pkv_swap_blocks(src[0], src[1], dst[0], dst[1], d_pairs, dev_error=self.dev_error,
+                             stream=s)
+        if self.fp8:
+            dev = (self.k_scale, self.v_scale)
+            host = (self.host_k_scale, self.host_v_scale)
+            src, dst = (dev, host) if out else (host, dev)
+            _abi.pkv_swap_blocks(src[0], src[1], dst[0], dst[1], d_pairs,
+                                 dev_error=self.dev_error, stream=s)
+        return int(pairs.shape[0])
+
+    def swap_out(self, seq_ids, stream=None):
+        """Moves the sequences' blocks to the host caches ("PagedAttention 动态
+        内存分页" page, 动态块分配与回收); their GPU blocks return to the pool.
+        Returns the number of blocks moved."""
+        return self._swap(seq_ids, True, stream)
+
+    def swap_in(self, seq_ids, stream=None):
+        """Brings swapped-out sequences back into (new) GPU blocks.  Returns
+        the number of blocks moved."""
+        return self._swap(seq_ids, False, stream)
+
     def check_errors(self):
         """Raises if a kernel recorded bad metadata since the last check."""
         err = self.dev_error.tolist()

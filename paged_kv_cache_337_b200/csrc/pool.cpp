@@ -15,6 +15,13 @@
 // recently freed block is reused first, which keeps hot blocks in L2); a
 // fresh pool hands blocks out in a caller-given order (default 0, 1, ...);
 // an operation that would run out of blocks changes nothing.
+//
+// Block swapping (same page, 动态块分配与回收: when GPU memory runs short, a
+// sequence's KV blocks move to CPU memory and come back when needed): a
+// second LIFO stack of host block ids, made once.  A swap moves one whole
+// sequence, in table order, and returns the (src, dst) pairs to copy; a GPU
+// block still shared with a resident sequence stays on the GPU for it.  A
+// swapped-out sequence cannot be appended to or forked.
 #include <algorithm>
 #include <new>
 #include <unordered_map>
@@ -25,8 +32,9 @@
 namespace {
 
 struct Seq {
-    std::vector<int32_t> table;  // physical block ids in logical order
+    std::vector<int32_t> table;  // physical block ids in logical order (host ids if swapped)
     int64_t tokens = 0;
+    bool swapped = false;
 };
 
 }  // namespace
@@ -37,6 +45,9 @@ struct pkv_pool {
     std::vector<int32_t> free_stack;  // top = back()
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Seq> seqs;
+    bool has_host = false;
+    std::vector<int32_t> host_free;  // top = back()
+    std::vector<int32_t> host_refcount;
 
     int32_t take() {
         int32_t b = free_stack.back();
@@ -103,6 +114,8 @@ extern "C" int pkv_seq_fork(pkv_pool* pool, int64_t parent, int64_t child) {
     auto it = pool->seqs.find(parent);
     PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
                 "pkv_seq_fork: no sequence %lld", (long long)parent);
+    PKV_REQUIRE(!it->second.swapped, PKV_ERR_INVALID,
+                "pkv_seq_fork: sequence %lld is swapped out", (long long)parent);
     PKV_REQUIRE(!pool->seqs.count(child), PKV_ERR_INVALID,
                 "pkv_seq_fork: sequence %lld exists", (long long)child);
     Seq c = it->second;  // copy before emplace: emplace may rehash
@@ -119,6 +132,8 @@ extern "C" int pkv_seq_append(pkv_pool* pool, int64_t seq_id, int64_t* slot,
     PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
                 "pkv_seq_append: no sequence %lld", (long long)seq_id);
     Seq& s = it->second;
+    PKV_REQUIRE(!s.swapped, PKV_ERR_INVALID, "pkv_seq_append: sequence %lld is swapped out",
+                (long long)seq_id);
     const int bs = pool->block_size;
     const int off = (int)(s.tokens % bs);
     int32_t src = -1, dst = -1;
@@ -173,8 +188,13 @@ extern "C" int pkv_seq_free(pkv_pool* pool, int64_t seq_id) {
     auto it = pool->seqs.find(seq_id);
     PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
                 "pkv_seq_free: no sequence %lld", (long long)seq_id);
-    for (int32_t b : it->second.table)
-        if (--pool->refcount[b] == 0) pool->free_stack.push_back(b);
+    if (it->second.swapped) {
+        for (int32_t h : it->second.table)
+            if (--pool->host_refcount[h] == 0) pool->host_free.push_back(h);
+    } else {
+        for (int32_t b : it->second.table)
+            if (--pool->refcount[b] == 0) pool->free_stack.push_back(b);
+    }
     pool->seqs.erase(it);
     return PKV_OK;
 }
@@ -196,6 +216,8 @@ extern "C" int pkv_seq_slot_mapping(const pkv_pool* pool, int64_t seq_id, int fi
     PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
                 "pkv_seq_slot_mapping: no sequence %lld", (long long)seq_id);
     const Seq& s = it->second;
+    PKV_REQUIRE(!s.swapped, PKV_ERR_INVALID, "pkv_seq_slot_mapping: sequence %lld is swapped out",
+                (long long)seq_id);
     PKV_REQUIRE(first_token >= 0 && num_tokens >= 0 &&
                     (int64_t)first_token + num_tokens <= s.tokens,
                 PKV_ERR_INVALID, "pkv_seq_slot_mapping: tokens [%d, %d) outside 0..%lld",
@@ -233,6 +255,9 @@ extern "C" int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t*
         auto it = pool->seqs.find(seq_ids[i]);
         PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
                     "pkv_pool_block_tables: no sequence %lld", (long long)seq_ids[i]);
+        PKV_REQUIRE(!it->second.swapped, PKV_ERR_INVALID,
+                    "pkv_pool_block_tables: sequence %lld is swapped out",
+                    (long long)seq_ids[i]);
         const auto& t = it->second.table;
         PKV_REQUIRE((int64_t)t.size() <= max_blocks_per_seq, PKV_ERR_INVALID,
                     "pkv_pool_block_tables: sequence %lld has %zu blocks > %d",
@@ -277,4 +302,112 @@ extern "C" int pkv_block_refcount(const pkv_pool* pool, int block) {
     PKV_REQUIRE(pool && block >= 0 && block < pool->num_blocks, PKV_ERR_INVALID,
                 "pkv_block_refcount: bad block %d", block);
     return pool->refcount[block];
+}
+
+// ---------------------------------------------------------------------------
+// block swapping
+// ---------------------------------------------------------------------------
+extern "C" int pkv_pool_set_host_blocks(pkv_pool* pool, int num_host_blocks) {
+    PKV_REQUIRE(pool && num_host_blocks >= 0, PKV_ERR_INVALID,
+                "pkv_pool_set_host_blocks: bad argument");
+    PKV_REQUIRE(!pool->has_host, PKV_ERR_INVALID,
+                "pkv_pool_set_host_blocks: the host pool exists");
+    pool->has_host = true;
+    pool->host_refcount.assign(num_host_blocks, 0);
+    pool->host_free.resize(num_host_blocks);
+    for (int i = 0; i < num_host_blocks; ++i) pool->host_free[i] = num_host_blocks - 1 - i;
+    return PKV_OK;
+}
+
+extern "C" int pkv_seq_swap_out(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int cap,
+                                int* num_pairs) {
+    PKV_REQUIRE(pool && num_pairs, PKV_ERR_INVALID, "pkv_seq_swap_out: NULL argument");
+    *num_pairs = 0;
+    PKV_REQUIRE(pool->has_host, PKV_ERR_INVALID, "pkv_seq_swap_out: no host pool");
+    auto it = pool->seqs.find(seq_id);
+    PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
+                "pkv_seq_swap_out: no sequence %lld", (long long)seq_id);
+    Seq& s = it->second;
+    PKV_REQUIRE(!s.swapped, PKV_ERR_INVALID, "pkv_seq_swap_out: sequence %lld is swapped out",
+                (long long)seq_id);
+    const size_t n = s.table.size();
+    PKV_REQUIRE((int64_t)cap >= (int64_t)n && (n == 0 || pairs), PKV_ERR_INVALID,
+                "pkv_seq_swap_out: capacity %d < %zu pairs", cap, n);
+    PKV_REQUIRE(n <= pool->host_free.size(), PKV_ERR_OOM,
+                "pkv_seq_swap_out: needs %zu host blocks, %zu free", n, pool->host_free.size());
+    for (size_t i = 0; i < n; ++i) {
+        const int32_t h = pool->host_free.back();
+        pool->host_free.pop_back();
+        pool->host_refcount[h] = 1;
+        pairs[2 * i] = s.table[i];
+        pairs[2 * i + 1] = h;
+    }
+    for (size_t i = 0; i < n; ++i) {
+        const int32_t b = s.table[i];
+        if (--pool->refcount[b] == 0) pool->free_stack.push_back(b);
+        s.table[i] = pairs[2 * i + 1];
+    }
+    s.swapped = true;
+    *num_pairs = (int)n;
+    return PKV_OK;
+}
+
+extern "C" int pkv_seq_swap_in(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int cap,
+                               int* num_pairs) {
+    PKV_REQUIRE(pool && num_pairs, PKV_ERR_INVALID, "pkv_seq_swap_in: NULL argument");
+    *num_pairs = 0;
+    auto it = pool->seqs.find(seq_id);
+    PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
+                "pkv_seq_swap_in: no sequence %lld", (long long)seq_id);
+    Seq& s = it->second;
+    PKV_REQUIRE(s.swapped, PKV_ERR_INVALID, "pkv_seq_swap_in: sequence %lld is resident",
+                (long long)seq_id);
+    const size_t n = s.table.size();
+    PKV_REQUIRE((int64_t)cap >= (int64_t)n && (n == 0 || pairs), PKV_ERR_INVALID,
+                "pkv_seq_swap_in: capacity %d < %zu pairs", cap, n);
+    PKV_REQUIRE(n <= pool->free_stack.size(), PKV_ERR_OOM,
+                "pkv_seq_swap_in: needs %zu blocks, %zu free", n, pool->free_stack.size());
+    for (size_t i = 0; i < n; ++i) {
+        pairs[2 * i] = s.table[i];
+        pairs[2 * i + 1] = pool->take();
+    }
+    for (size_t i = 0; i < n; ++i) {
+        const int32_t h = s.table[i];
+        if (--pool->host_refcount[h] == 0) pool->host_free.push_back(h);
+        s.table[i] = pairs[2 * i + 1];
+    }
+    s.swapped = false;
+    *num_pairs = (int)n;
+    return PKV_OK;
+}
+
+extern "C" int pkv_seq_is_swapped(const pkv_pool* pool, int64_t seq_id, int* swapped) {
+    PKV_REQUIRE(pool && swapped, PKV_ERR_INVALID, "pkv_seq_is_swapped: NULL argument");
+    auto it = pool->seqs.find(seq_id);
+    PKV_REQUIRE(it != pool->seqs.end(), PKV_ERR_INVALID,
+                "pkv_seq_is_swapped: no sequence %lld", (long long)seq_id);
+    *swapped = it->second.swapped ? 1 : 0;
+    return PKV_OK;
+}
+
+extern "C" int pkv_pool_num_free_host(const pkv_pool* pool) {
+    PKV_REQUIRE(pool, PKV_ERR_INVALID, "pkv_pool_num_free_host: pool is NULL");
+    return (int)pool->host_free.size();
+}
+
+extern "C" int pkv_pool_host_free_list(const pkv_pool* pool, int32_t* out, int cap, int* n) {
+    PKV_REQUIRE(pool && n, PKV_ERR_INVALID, "pkv_pool_host_free_list: NULL argument");
+    *n = (int)pool->host_free.size();
+    PKV_REQUIRE((int64_t)cap >= (int64_t)pool->host_free.size() &&
+                    (pool->host_free.empty() || out),
+                PKV_ERR_INVALID, "pkv_pool_host_free_list: capacity %d < %zu", cap,
+                pool->host_free.size());
+    std::copy(pool->host_free.begin(), pool->host_free.end(), out);
+    return PKV_OK;
+}
+
+extern "C" int pkv_host_block_refcount(const pkv_pool* pool, int block) {
+    PKV_REQUIRE(pool && block >= 0 && block < (int)pool->host_refcount.size(), PKV_ERR_INVALID,
+                "pkv_host_block_refcount: bad host block %d", block);
+    return pool->host_refcount[block];
 }

@@ -154,3 +154,88 @@ def test_oom_and_invalid_statuses():
     assert status_of(native.free, 3)[0] == ERR_INVALID
     with pytest.raises(_abi.PkvError):
         _abi.BlockPool(3, 4, free_order=[0, 0, 1])
+
+
+# ---------------------------------------------------------------------------
+# block swapping: the native pool follows the model's host pool too
+# ---------------------------------------------------------------------------
+def native_host_state(pool, seq_ids):
+    swapped = tuple(sorted(s for s in seq_ids if pool.is_swapped(s)))
+    return tuple(pool.host_free_list()), tuple(pool.host_refcounts()), swapped
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_native_matches_model_with_swaps(seed):
+    rng = random.Random(300 + seed)
+    nb = rng.choice([8, 24, 60])
+    nh = rng.choice([4, 16, 50])
+    bs = rng.choice([1, 4, 16])
+    order = list(range(nb))
+    rng.shuffle(order)
+    model = PoolModel(nb, bs, free_order=order)
+    native = _abi.BlockPool(nb, bs, free_order=order)
+    assert model.set_host_blocks(nh) == OK
+    native.set_host_blocks(nh)
+    assert status_of(native.set_host_blocks, nh)[0] == model.set_host_blocks(nh) == ERR_INVALID
+    live, next_id = [], 0
+    for step in range(600):
+        r = rng.random()
+        if r < 0.15 or not live:
+            n = rng.randint(0, 3 * bs)
+            a = model.seq_add(next_id, n)
+            assert status_of(native.add, next_id, n)[0] == a
+            if a == OK:
+                live.append(next_id)
+            next_id += 1
+        elif r < 0.25:
+            parent = rng.choice(live)
+            a = model.seq_fork(parent, next_id)
+            assert status_of(native.fork, parent, next_id)[0] == a
+            if a == OK:
+                live.append(next_id)
+            next_id += 1
+        elif r < 0.55:
+            s = rng.choice(live)
+            st, slot, src, dst = model.seq_append(s)
+            nst, res = status_of(native.append, s)
+            assert nst == st
+            if st == OK:
+                assert res == (slot, src, dst)
+        elif r < 0.7:
+            s = rng.choice(live)
+            st, pairs = model.seq_swap_out(s)
+            nst, res = status_of(native.swap_out, s)
+            assert nst == st
+            if st == OK:
+                assert res.tolist() == [list(p) for p in pairs]
+        elif r < 0.85:
+            s = rng.choice(live)
+            st, pairs = model.seq_swap_in(s)
+            nst, res = status_of(native.swap_in, s)
+            assert nst == st
+            if st == OK:
+                assert res.tolist() == [list(p) for p in pairs]
+        else:
+            s = rng.choice(live)
+            assert model.seq_free(s) == OK
+            assert status_of(native.free, s)[0] == OK
+            live.remove(s)
+        assert native_state(native, live) == model.state(), step
+        assert native_host_state(native, live) == model.host_state(), step
+
+
+def test_swapped_sequences_leave_the_decode_tables():
+    native = _abi.BlockPool(8, 4)
+    native.set_host_blocks(8)
+    native.add(1, 5)
+    native.add(2, 3)
+    native.swap_out(1)
+    with pytest.raises(_abi.PkvError):
+        native.block_tables([1, 2], 4)
+    with pytest.raises(_abi.PkvError):
+        native.slot_mapping(1, 0, 5)
+    tables, lens = native.block_tables([2], 4)
+    assert lens.tolist() == [3]
+    native.swap_in(1)
+    tables, lens = native.block_tables([1, 2], 4)
+    assert lens.tolist() == [5, 3]

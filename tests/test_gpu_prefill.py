@@ -1,0 +1,132 @@
+"""Paged prefill attention on the GPU against the fp64 oracle ("Paged KV"
+wiki page, 实现原理 / 运行阶段), elementwise within |gpu - oracle| <= 2e-3 +
+1e-2 |oracle|: whole prompts and later chunks, ragged lengths across row
+and key tiles, every built GQA group, f16 and bf16, block sizes 16-64,
+plus the prompt write through the pool's slot mapping."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import reference as ref
+from paged_kv_cache_337_b200 import _abi, build
+from paged_kv_cache_337_b200.cache import PagedKVCache
+from tests.helpers import DT, paged_problem, tolerance_violation
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-3, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    build.build()
+    _abi.lib()
+
+
+def run_prefill(p, q, qs, scale, dev, dev_error=None):
+    out = torch.full_like(q, float("nan")).to(dev)
+    n = np.diff(qs)
+    _abi.pkv_prefill_attention(out, q.to(dev), p["kc"].to(dev), p["vc"].to(dev),
+                               torch.as_tensor(p["tables"]).to(dev),
+                               torch.as_tensor(p["lens"]).to(dev),
+                               torch.as_tensor(qs, dtype=torch.int32).to(dev),
+                               int(n.max()) if n.size else 0, scale, dev_error=dev_error)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def case(seed, Hq, Hkv, bs, lens, chunks, dtype):
+    p = paged_problem(seed, Hq, Hkv, 128, bs, lens, dtype)
+    g = torch.Generator().manual_seed(seed + 7)
+    n = [min(c, L) for c, L in zip(chunks, lens)]
+    qs = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = torch.randn(int(qs[-1]), Hq, 128, generator=g).to(DT[dtype])
+    return p, q, qs
+
+
+WHOLE = ([1, 16, 17, 65, 130, 257], [1, 16, 17, 65, 130, 257])
+CHUNKED = ([40, 129, 300, 64, 77, 5], [8, 64, 100, 1, 77, 0])
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2), (12, 4), (32, 8), (6, 6)])
+@pytest.mark.parametrize("bs", [16, 32, 64])
+@pytest.mark.parametrize("lens,chunks", [WHOLE, CHUNKED], ids=["whole", "chunked"])
+def test_prefill_matches_oracle(dtype, Hq, Hkv, bs, lens, chunks, cuda_device):
+    seed = zlib.crc32(repr((dtype, Hq, Hkv, bs, lens)).encode()) % 10000
+    p, q, qs = case(seed, Hq, Hkv, bs, lens, chunks, dtype)
+    scale = 1.0 / np.sqrt(128)
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    got = run_prefill(p, q, qs, scale, cuda_device, err)
+    want = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, dtype,
+                                 Hkv, bs)
+    assert err.tolist() == [0, 0]
+    assert torch.isfinite(got).all()
+    assert tolerance_violation(got, want, ATOL, RTOL) <= 0
+
+
+def test_prefill_large_scores_stay_finite(cuda_device):
+    p, q, qs = case(5, 8, 8, 16, [200], [200], "bf16")
+    got = run_prefill(p, q * 8, qs, 1.0, cuda_device)
+    want = ref.prefill_attention(q * 8, p["kc"], p["vc"], p["tables"], p["lens"], qs, 1.0,
+                                 "bf16", 8, 16)
+    assert torch.isfinite(got).all()
+    assert tolerance_violation(got, want, ATOL, RTOL) <= 0
+
+
+def test_prefill_bad_lengths_are_reported(cuda_device):
+    p, q, qs = case(6, 4, 4, 16, [10, 20], [10, 20], "f16")
+    lens = torch.tensor([10, 5], dtype=torch.int32)  # sequence 1: 20 rows but 5 tokens
+    out = torch.zeros(q.shape, dtype=q.dtype, device=cuda_device)
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    _abi.pkv_prefill_attention(out, q.to(cuda_device), p["kc"].to(cuda_device),
+                               p["vc"].to(cuda_device), torch.as_tensor(p["tables"]).to(cuda_device),
+                               lens.to(cuda_device), torch.as_tensor(qs).to(cuda_device), 20, 0.1,
+                               dev_error=err)
+    torch.cuda.synchronize()
+    assert err.tolist() == [_abi.PKV_DEVERR_CONTEXT_LEN, 1]
+    assert not out[10:].any()  # its rows are left unwritten
+    want = ref.prefill_attention(q[:10], p["kc"], p["vc"], p["tables"][:1], [10], [0, 10], 0.1,
+                                 "f16", 4, 16)
+    assert tolerance_violation(out[:10].cpu(), want, ATOL, RTOL) <= 0
+
+
+def test_prompt_write_then_prefill_through_the_pool(cuda_device):
+    """The prefill step as the driver runs it: the pool takes each prompt's
+    blocks, pkv_write_slots fills them through the slot mapping, and prefill
+    attention reads them back through the Block Tables."""
+    dev = cuda_device
+    g = torch.Generator().manual_seed(9)
+    bs, Hq, Hkv, D = 16, 16, 4, 128
+    prompts = [37, 160, 1, 96]
+    nb = sum(-(-L // bs) for L in prompts) + 5
+    cache = PagedKVCache(nb, bs, Hq, Hkv, D, torch.float16, dev, 16,
+                         free_order=torch.randperm(nb, generator=g).tolist())
+    qs = np.concatenate([[0], np.cumsum(prompts)]).astype(np.int32)
+    T = int(qs[-1])
+    q = torch.randn(T, Hq, D, generator=g).to(torch.float16)
+    k = torch.randn(T, Hkv, D, generator=g).to(torch.float16)
+    v = torch.randn(T, Hkv, D, generator=g).to(torch.float16)
+    for s, L in enumerate(prompts):
+        cache.add_sequence(s, L, k[qs[s]:qs[s + 1]].to(dev), v[qs[s]:qs[s + 1]].to(dev))
+    tables, lens = cache.pool.block_tables(list(range(len(prompts))), 16)
+    out = torch.empty(T, Hq, D, dtype=torch.float16, device=dev)
+    _abi.pkv_prefill_attention(out, q.to(dev), cache.key_cache, cache.value_cache, tables.to(dev),
+                               lens.to(dev), torch.as_tensor(qs).to(dev), max(prompts),
+                               cache.scale)
+    torch.cuda.synchronize()
+    # the oracle reads its own write of the same prompts (into zeroed
+    # caches) through the same Block Tables
+    kc0 = np.zeros((nb, bs, Hkv, D), np.uint16)
+    slots = np.concatenate([cache.pool.slot_mapping(s, 0, L).numpy()
+                            for s, L in enumerate(prompts)])
+    wk, wv = ref.write_slots(kc0, kc0, k, v, slots, bs, Hkv)
+    want = ref.prefill_attention(q, wk, wv, tables, lens, qs, cache.scale, "f16", Hkv, bs)
+    assert tolerance_violation(out.cpu(), want, ATOL, RTOL) <= 0
+    # and the prompt write itself is bit-exact at every slot it filled
+    got_k = ref.bits(cache.key_cache.cpu()).reshape(nb * bs, Hkv, D)[slots]
+    got_v = ref.bits(cache.value_cache.cpu()).reshape(nb * bs, Hkv, D)[slots]
+    assert np.array_equal(got_k, wk.reshape(nb * bs, Hkv, D)[slots])
+    assert np.array_equal(got_v, wv.reshape(nb * bs, Hkv, D)[slots])
