@@ -305,6 +305,13 @@ struct GemvWarp {
 // ---------------------------------------------------------------------------
 // Per-warp arithmetic, G >= 2: mma.sync m16n8k16 on the head group
 // ---------------------------------------------------------------------------
+// Token held by row r of the e4m3 path's S^T fragments: rows 2j, 2j+1 are
+// tokens 4j, 4j+1 and rows 8+2j, 9+2j are tokens 4j+2, 4j+3, the order in
+// which the transposing byte load delivers V (so P's fragments line up).
+__device__ __forceinline__ int token_of_row(int r) {
+    return r < 8 ? 4 * (r >> 1) + (r & 1) : 4 * ((r - 8) >> 1) + 2 + (r & 1);
+}
+
 // E4 (e4m3 caches): K comes straight from the e4m3 tile and every product
 // runs on f16 (e4m3 values are exact in f16), whatever T is; the queries
 // are scaled by a power of two into f16 range and the scale is undone on
@@ -426,7 +433,7 @@ struct MmaWarp {
 #pragma unroll
             for (int pp = 0; pp < KS / 2; ++pp) {
                 uint32_t r[4];
-                const int row = (lane & 7) + (j & 1) * 8;
+                const int row = token_of_row((lane & 7) + (j & 1) * 8);
                 const int chunk = 2 * pp + (j >> 1);
                 ldmatrix_x4(r, kbase + row * 128 + ((chunk ^ (row & 7)) << 4));
                 const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)r[0]),
@@ -466,7 +473,8 @@ struct MmaWarp {
             for (int i = 0; i < 4; ++i) sacc[nt][i] += sacc2[nt][i];
         // online softmax per head; the lane holds tokens r0, r0 + 8
         const int r0 = lane >> 2;
-        const bool v0 = r0 < valid, v1 = r0 + 8 < valid;
+        const bool v0 = (E4 ? token_of_row(r0) : r0) < valid;
+        const bool v1 = (E4 ? token_of_row(r0 + 8) : r0 + 8) < valid;
         const float ratio = vscale == vs ? 1.f : vs / vscale;
         vs = vscale;
         uint32_t pb[NT][2], pl[NT][2];
@@ -511,15 +519,41 @@ struct MmaWarp {
             pl[nt][1] = movmatrix_trans(Storage<MT>::from_float2(p2 - b23.x, p3 - b23.y));
         }
         // O^T[d][head] += V^T P^T over the 16 tokens
+        if constexpr (E4) {
+            // vt is the e4m3 tile.  The transposing byte load gives the lane
+            // tokens 4j .. 4j+3 of dims g and g + 8 of two 16-dim m-tiles;
+            // converted pairwise they are the A fragments with the token
+            // order of P's fragments (token_of_row).
+            const int tok = lane & 15;
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-            uint32_t a[4];
-            const int row = (lane & 7) + (j >> 1) * 8;
-            ldmatrix_x4_trans(a, vbase + swz(row, mt * 2 + (j & 1)));
+            for (int mp = 0; mp < KS / 2; ++mp) {
+                uint32_t r[4];
+                const int chunk = 2 * mp + (lane >> 4);
+                ldmatrix_b8_x2_trans(r, vbase + tok * 128 + ((chunk ^ (tok & 7)) << 4));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                Mma<MT>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
-                Mma<MT>::m16n8k16(acc[mt][nt], a, pl[nt][0], pl[nt][1]);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a[4] = {e4m3x2_to_f16x2((uint16_t)r[2 * h]),
+                                           e4m3x2_to_f16x2((uint16_t)r[2 * h + 1]),
+                                           e4m3x2_to_f16x2((uint16_t)(r[2 * h] >> 16)),
+                                           e4m3x2_to_f16x2((uint16_t)(r[2 * h + 1] >> 16))};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        Mma<MT>::m16n8k16(acc[2 * mp + h][nt], a, pb[nt][0], pb[nt][1]);
+                        Mma<MT>::m16n8k16(acc[2 * mp + h][nt], a, pl[nt][0], pl[nt][1]);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                uint32_t a[4];
+                const int row = (lane & 7) + (j >> 1) * 8;
+                ldmatrix_x4_trans(a, vbase + swz(row, mt * 2 + (j & 1)));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    Mma<MT>::m16n8k16(acc[mt][nt], a, pb[nt][0], pb[nt][1]);
+                    Mma<MT>::m16n8k16(acc[mt][nt], a, pl[nt][0], pl[nt][1]);
+                }
             }
         }
     }
@@ -568,10 +602,9 @@ struct MmaWarp {
 
 // ---------------------------------------------------------------------------
 // Shared-memory plan of one CTA: per warp a ring of stages (the K and V tiles
-// as stored), then, for e4m3 caches on the tensor-core path, an f16 copy of
-// the current V tile per warp; then the mbarriers, the per-stage
-// dequantisation scales (e4m3) and the partition's table slice.  The ring and
-// the copies are reused by the epilogue once every load has landed.
+// as stored), then the mbarriers, the per-stage dequantisation scales (e4m3)
+// and the partition's table slice.  The ring is reused by the epilogue once
+// every load has landed.
 // ---------------------------------------------------------------------------
 template <int D, bool FP8, bool MMA>
 struct Plan {
@@ -579,47 +612,13 @@ struct Plan {
     static constexpr int kStages = FP8 ? (MMA ? 3 : 4) : Geom<D>::kStages;
     static constexpr int kTileBytes = FP8 ? kTile * D : Geom<D>::kKBytes;  // K (or V) as stored
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kScratchBytes = (FP8 && MMA) ? Geom<D>::kKBytes : 0;  // f16 V tile
     static constexpr size_t kRing = (size_t)kWarps * kStages * kStageBytes;
-    static constexpr size_t kEpilogue = kRing + (size_t)kWarps * kScratchBytes;
+    static constexpr size_t kEpilogue = kRing;
     static constexpr size_t kBarOff = kEpilogue;
     static constexpr size_t kScaleOff = kBarOff + (size_t)kWarps * kStages * 8;
     static constexpr size_t kTableOff = kScaleOff + (FP8 ? (size_t)kWarps * kStages * 32 : 0);
     static constexpr uint32_t kTx = kStageBytes + (FP8 ? 32 : 0);  // bytes landing per stage
 };
-
-// Widens an e4m3 tile (16 rows of 128 bytes, swizzled) into the 16-bit tile
-// layout the tensor-core path reads (two 64-column sub-tiles, swizzled).
-// e4m3 values are exact in both fp16 and bf16.
-template <typename T>
-__device__ __forceinline__ void widen_fp8_tile(const uint8_t* raw, uint8_t* dst, int lane) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = lane + 32 * j;  // 128 chunks of 16 codes
-        const int r = c >> 3, ch = c & 7;
-        const uint4 x = *reinterpret_cast<const uint4*>(raw + r * 128 + ((ch ^ (r & 7)) << 4));
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t h[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t a = e4m3x2_to_f16x2((uint16_t)(w[k] & 0xffffu));
-            const uint32_t b = e4m3x2_to_f16x2((uint16_t)(w[k] >> 16));
-            if constexpr (std::is_same<T, __half>::value) {
-                h[2 * k] = a;
-                h[2 * k + 1] = b;
-            } else {
-                __half2 ha, hb;
-                memcpy(&ha, &a, 4);
-                memcpy(&hb, &b, 4);
-                const float2 fa = __half22float2(ha), fb = __half22float2(hb);
-                h[2 * k] = Storage<T>::from_float2(fa.x, fa.y);
-                h[2 * k + 1] = Storage<T>::from_float2(fb.x, fb.y);
-            }
-        }
-        *reinterpret_cast<uint4*>(dst + swz(r, 2 * ch)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(dst + swz(r, 2 * ch + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
-    }
-}
 
 // ---------------------------------------------------------------------------
 // The attention kernel (single pass or one partition of split-K)
@@ -666,7 +665,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     uint64_t* my_bars = bars + warp * STAGES;
     uint8_t* my_stages = stages + warp * STAGES * Pl::kStageBytes;
     float* my_scales = scales + warp * STAGES * 8;
-    uint8_t* my_wide = smem + Pl::kRing + warp * Pl::kScratchBytes;  // e4m3 + tensor cores
     if (lane == 0) {
 #pragma unroll
         for (int st = 0; st < STAGES; ++st) mbar_init(&my_bars[st], 1);
@@ -744,19 +742,12 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
             const int64_t si = scale_index(table[(t_begin + tile * kTile) / bs - lb0]) & 3;
             kscale = my_scales[st * 8 + si];
             vscale = my_scales[st * 8 + 4 + si];
-            if constexpr (Warp::kMma) {
-                // K is read from the e4m3 tile itself; V is transposed by
-                // ldmatrix.trans, which moves 16-bit elements, so it is
-                // widened to f16 first
-                widen_fp8_tile<__half>(vt, my_wide, lane);
-                __syncwarp();
-                vt = my_wide;
-            }
+
         }
         if (valid < kTile) {
             // rows past the context may hold anything (NaN included): zero
             // the V rows so that their zero weights contribute exactly 0
-            if constexpr (FP8 && !Warp::kMma) {
+            if constexpr (FP8) {
                 for (int c = lane; c < (kTile - valid) * 8; c += 32)
                     *reinterpret_cast<uint4*>(vt + (valid + c / 8) * 128 + (c % 8) * 16) =
                         make_uint4(0, 0, 0, 0);
