@@ -5,40 +5,49 @@
 //
 // Sequence s has n_s query rows (query_start[s] .. query_start[s+1]-1), the
 // last n_s of its L_s cached tokens: row i is token p = L_s - n_s + i and
-// attends causally to tokens 0 .. p.  A whole prompt has n_s = L_s; a later
-// chunk of a long prompt has n_s < L_s.
+// attends causally to tokens 0 .. p.
 //
-// One CTA takes 64 rows of one (sequence, KV head): the rows are (query
-// token, head of the GQA group) pairs, so the K/V tile the CTA streams is
-// shared by the group's heads.  A producer warp brings 64-key K and V tiles
-// through a 2-stage ring (one 5-D TMA box per 16 slots of a block; block
-// size a multiple of 16), and four consumer warps each own 16 rows:
-// S = Q K^T and O += P V on mma.sync m16n8k16 with fp32 accumulators, the
-// online softmax in base 2, and the causal mask as a per-row select.  The
-// grid is flat and dispatches every sequence's last (heaviest) row tile
-// first.  Bound: the tensor pipe for long prompts.
+// One CTA takes 128 rows of one (sequence, KV head): (query token, head of
+// the GQA group) pairs, so each K/V tile is streamed once for the group.
+// The work runs on the 5th-generation tensor cores with the accumulators in
+// tensor memory:
+//   - a producer warp brings 128-key K and V tiles through a 2-stage ring
+//     (one TMA box per 16 slots of a block and per 64-dim half);
+//   - an MMA warp issues S = Q K^T (M 128, N 128, K 16 steps; Q and K from
+//     shared memory) into tensor memory, then O += P V with P read from
+//     tensor memory and V from shared memory (B operand MN-major);
+//   - four softmax warps (one tensor-memory lane quarter each, one row per
+//     thread) read S, apply the causal mask, keep the running max and sum,
+//     write P (a 16-bit high part and its 16-bit remainder, two MMAs) and
+//     rescale O when the running max grows by more than 2^8, then write the
+//     normalised output.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 #include "tensor_maps.h"
 
 namespace pkv {
 namespace {
 
-constexpr int kD = 128;                          // head_dim (built)
-constexpr int kRows = 64;                        // (token, head) rows per CTA
-constexpr int kKeys = 64;                        // keys per tile
-constexpr int kConsumers = 4;                    // warps of 16 rows
-constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
+constexpr int kD = 128;                 // head_dim (built)
+constexpr int kRows = 128;              // (token, head) rows per CTA = UMMA M
+constexpr int kKeys = 128;              // keys per tile = UMMA N of S, K of P V
 constexpr int kStages = 2;
-constexpr int kBoxKeys = 16;                          // slots per TMA box
-constexpr int kBoxBytes = kBoxKeys * kD * 2;          // 4 KiB: two 16 x 128 B sub-tiles
-constexpr int kTileBytes = kKeys * kD * 2;            // 16 KiB of K (or V)
-constexpr int kStageBytes = 2 * kTileBytes;           // K + V
-constexpr int kQBytes = kRows * kD * 2;               // 16 KiB
-constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + (2 * kStages + 1) * 8;
+constexpr int kHalfBytes = kKeys * 128; // one 64-dim half of a K (or V) tile: 16 KiB
+constexpr int kTileBytes = 2 * kHalfBytes;          // 32 KiB
+constexpr int kStageBytes = 2 * kTileBytes;         // K + V
+constexpr int kQHalfBytes = kRows * 128;            // 16 KiB
+constexpr int kQBytes = 2 * kQHalfBytes;
+constexpr int kBoxKeys = 16;                        // slots per TMA box
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4;
+constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;
+// tensor-memory columns: S | P high | P low | O
+constexpr uint32_t kColS = 0, kColPh = 128, kColPl = 192, kColO = 256, kTmemCols = 512;
+constexpr int kNumBars = 2 * kStages + 4;  // kv_full, kv_empty, s_full, p_full, o_done, drain
+constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr unsigned kFull = 0xffffffffu;
+constexpr float kRescaleLog2 = 8.f;  // rescale O when the max grows by more than 2^8
 
 struct PrefillParams {
     void* out;
@@ -52,15 +61,11 @@ struct PrefillParams {
     float scale_log2;
 };
 
-// byte offset of (row, 16-byte chunk) in a swizzled tile of 16-row x 128-B
-// sub-tiles (the layout one TMA box lands in; chunk >> 3 picks the 64-dim half)
-__device__ __forceinline__ uint32_t swz16(int r, int chunk) {
-    return (chunk >> 3) * (kBoxKeys * 128) + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
-}
-
-// the Q tile: two 64-row x 128-B halves, swizzled the same way
-__device__ __forceinline__ uint32_t swz_q(int r, int chunk) {
-    return (chunk >> 3) * (kRows * 128) + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
+// swizzled byte offset of (row, 16-byte chunk) inside one 64-dim half laid
+// out as rows of 128 bytes (the TMA 128-byte swizzle and the UMMA canonical
+// K-major / MN-major 128-byte swizzle agree on it)
+__device__ __forceinline__ uint32_t swz(int r, int chunk) {
+    return r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
 }
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -72,55 +77,242 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// The producer: lane 0 of the last warp streams the K and V tiles of keys
-// [0, kv_end) into the ring.  A box past the context still loads a block
-// (the last one) so that every stage receives its full byte count; its rows
-// are masked (K) or zeroed (V) by the consumers.
+struct Bars {
+    uint64_t* kv_full;   // [kStages]: TMA bytes landed
+    uint64_t* kv_empty;  // [kStages]: the P V MMAs reading the stage completed
+    uint64_t* s_full;    // S in tensor memory
+    uint64_t* p_full;    // P written (and O rescaled) by the softmax warps
+    uint64_t* o_done;    // the P V MMAs of the tile completed
+    uint64_t* drain;     // every MMA issued completed (exit)
+};
+
+// Producer: lane 0 of warp 0.  A box past the context still loads a block
+// (the last one) so that every stage receives its full byte count; those
+// rows are masked (K) or zeroed (V) downstream.
 __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const PrefillParams& p,
-                        int s, int kvh, int L, int ntiles, uint8_t* stages, uint64_t* full,
-                        uint64_t* empty) {
+                        int s, int kvh, int L, int ntiles, uint8_t* stages, const Bars& b,
+                        bool* failed) {
     const int bs = p.block_size;
     const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     const int last_block = L > 0 ? (L - 1) / bs : 0;
+    int issued = 0;
     for (int j = 0; j < ntiles; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait_bounded(&empty[st], ((j / kStages) - 1) & 1)) {
-            report_error(p.dev_error, PKV_DEVERR_TIMEOUT, s);
-            return;
+        if (j >= kStages && !mbar_wait_bounded(&b.kv_empty[st], ((j / kStages) - 1) & 1)) {
+            *failed = true;
+            break;
         }
         uint8_t* kdst = stages + st * kStageBytes;
         uint8_t* vdst = kdst + kTileBytes;
-        mbar_arrive_expect_tx(&full[st], kStageBytes);
-#pragma unroll
-        for (int b = 0; b < kKeys / kBoxKeys; ++b) {
-            const int key0 = j * kKeys + b * kBoxKeys;
+        mbar_arrive_expect_tx(&b.kv_full[st], kStageBytes);
+#pragma unroll 1
+        for (int bx = 0; bx < kKeys / kBoxKeys; ++bx) {
+            const int key0 = j * kKeys + bx * kBoxKeys;
             const int lb = min(key0 / bs, last_block);
             const int off = key0 < L ? key0 % bs : 0;
             const int32_t phys = __ldg(row + lb);
             if (phys < 0 || phys >= p.num_blocks) report_error(p.dev_error, PKV_DEVERR_BLOCK_ID, s);
-            // an out-of-range block id reads as zeros (TMA fill), never out of the cache
-            tma_load_5d(kdst + b * kBoxBytes, &kmap, &full[st], 0, kvh, off, 0, phys);
-            tma_load_5d(vdst + b * kBoxBytes, &vmap, &full[st], 0, kvh, off, 0, phys);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap, &b.kv_full[st], 0,
+                            kvh, off, h, phys);
+                tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap, &b.kv_full[st], 0,
+                            kvh, off, h, phys);
+            }
+        }
+        ++issued;
+    }
+    // before leaving, every issued load has landed (bounded)
+    for (int j = max(0, issued - kStages); j < issued; ++j)
+        mbar_wait_bounded(&b.kv_full[j % kStages], (j / kStages) & 1);
+}
+
+// MMA issuer: lane 0 of warp 1.
+template <bool BF16>
+__device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t* stages,
+                           int ntiles, bool* failed) {
+    constexpr uint32_t kIdS = tc::f16_idesc(BF16, false, kRows, kKeys);  // K: K-major B
+    constexpr uint32_t kIdPV = tc::f16_idesc(BF16, true, kRows, kD);     // V: MN-major B
+    for (int j = 0; j < ntiles; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait_bounded(&b.kv_full[st], (j / kStages) & 1)) {
+            *failed = true;
+            break;
+        }
+        tc::fence_after_sync();
+        const uint32_t kaddr = smem_addr(stages + st * kStageBytes);
+        const uint32_t vaddr = kaddr + kTileBytes;
+        // S = Q K^T: 8 steps of 16 dims (4 per 128-byte swizzle atom)
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * kQHalfBytes + (uint32_t)(kk & 3) * 32;
+            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
+            tc::mma_ss(tmem + kColS, tc::sw128_desc(qaddr + off, 16, 1024),
+                       tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_addr(b.s_full));
+        if (!mbar_wait_bounded(b.p_full, j & 1)) {
+            *failed = true;
+            break;
+        }
+        tc::fence_after_sync();
+        // O += P V: 8 steps of 16 keys; V's 8-key groups 1 KiB apart (SBO),
+        // its 64-dim halves 16 KiB apart (LBO)
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+            const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
+            tc::mma_ts(tmem + kColO, tmem + kColPh + kk * 8, vd, kIdPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_ts(tmem + kColO, tmem + kColPl + kk * 8, vd, kIdPV, 1u);
+        }
+        tc::commit(smem_addr(&b.kv_empty[st]));
+        tc::commit(smem_addr(b.o_done));
+    }
+    // every MMA issued has completed before the tensor memory is freed
+    tc::commit(smem_addr(b.drain));
+    mbar_wait_bounded(b.drain, 0);
+}
+
+// A bounded wait whose outcome is the same for the whole warp (the
+// tensor-memory loads and stores that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait_bounded(bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <typename T>
+__device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tmem,
+                             uint8_t* stages, int L, int n, int q0, int kvh, int r0, int nrows,
+                             int ntiles, int warp, int lane, bool* failed) {
+    const int quarter = warp & 3;  // tensor-memory lanes 32 * quarter .. + 31
+    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int r = 32 * quarter + lane;
+    const int R = r0 + r;
+    const bool ok = R < nrows;
+    const int pos = L - n + (ok ? R / p.group : 0);
+    const float sl = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    int j = 0;
+    for (; j < ntiles; ++j) {
+        if (!warp_wait(b.s_full, j & 1)) break;
+        tc::fence_after_sync();
+        float sv[kKeys];
+        {
+            uint32_t u[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::ld32(trow + kColS + 32 * c, u[c]);
+            tc::wait_ld();
+            const int key0 = j * kKeys;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int key = key0 + 32 * c + e;
+                    sv[32 * c + e] = (ok && key <= pos) ? __uint_as_float(u[c][e]) * sl : -INFINITY;
+                }
+        }
+        float mt = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kKeys; ++e) mt = fmaxf(mt, sv[e]);
+        const bool resc = mt > m + kRescaleLog2;  // also the first finite max
+        const float alpha = resc ? exp2f(m - mt) : 1.f;
+        if (resc) m = mt;
+        l *= alpha;
+        const float mu = m == -INFINITY ? 0.f : m;
+        // the P V of the previous tile must be done before P and O change
+        if (j > 0) {
+            if (!warp_wait(b.o_done, (j - 1) & 1)) break;
+            tc::fence_after_sync();
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tc::ld32(trow + kColO + 32 * c, o);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tc::st32(trow + kColO + 32 * c, o);
+                }
+            }
+        }
+        // P = 2^(s - m) as a 16-bit high part and the 16-bit remainder
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float a = exp2f(sv[32 * c + 2 * e] - mu);
+                const float d = exp2f(sv[32 * c + 2 * e + 1] - mu);
+                l += a + d;
+                hi[e] = Storage<T>::from_float2(a, d);
+                const float2 back = Storage<T>::to_float2(hi[e]);
+                lo[e] = Storage<T>::from_float2(a - back.x, d - back.y);
+            }
+            tc::st16(trow + kColPh + 16 * c, hi);
+            tc::st16(trow + kColPl + 16 * c, lo);
+        }
+        // keys past the context in the last tile: zero their V rows (NaN
+        // bit patterns there must not meet their zero weights)
+        const int key0 = j * kKeys;
+        if (key0 + kKeys > L) {
+            const int st = j % kStages;
+            if (!warp_wait(&b.kv_full[st], (j / kStages) & 1)) break;
+            uint8_t* vt = stages + st * kStageBytes + kTileBytes;
+            const int first = max(L - key0, 0);
+            const int t = (warp - kSoftmaxWarp0) * 32 + lane;
+            for (int c = t; c < (kKeys - first) * 16; c += kSoftmaxWarps * 32) {
+                const int k = first + (c >> 4), ch = c & 15;
+                *reinterpret_cast<uint4*>(vt + (ch >> 3) * kHalfBytes + swz(k, ch)) =
+                    make_uint4(0, 0, 0, 0);
+            }
+            tc::fence_proxy_async_smem();
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_one(b.p_full);
+    }
+    if (j < ntiles || !warp_wait(b.o_done, (ntiles - 1) & 1)) {
+        *failed = true;
+        return;
+    }
+    tc::fence_after_sync();
+    // every lane takes part in the (warp-collective) tensor-memory loads;
+    // only rows of this sequence are stored
+    const int tok = ok ? R / p.group : 0, g = ok ? R - tok * p.group : 0;
+    T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * p.num_q_heads + kvh * p.group + g) * kD;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tc::ld32(trow + kColO + 32 * c, o);
+        tc::wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            pk[e] = Storage<T>::from_float2(__uint_as_float(o[2 * e]) * inv,
+                                            __uint_as_float(o[2 * e + 1]) * inv);
+        if (ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                reinterpret_cast<uint4*>(dst + 32 * c)[v] =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
     }
 }
 
 template <typename T>
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    return Storage<T>::from_float2(a, b);
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_1024(smem_raw);
     uint8_t* qsm = smem;
     uint8_t* stages = smem + kQBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* zeroed = empty + kStages;  // the last tile's V rows are zeroed
+    uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + 1,
+           bars + 2 * kStages + 2, bars + 2 * kStages + 3};
 
     // flat grid: the heaviest row tile of every (sequence, KV head) first
     const int pairs = p.num_seqs * p.num_kv_heads;
@@ -141,201 +333,65 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     if (r0 >= nrows) return;  // a row tile past this sequence's rows
     const int last_row = min(nrows, r0 + kRows) - 1;
-    const int kv_end = L - n + last_row / G + 1;  // keys the tile's last row sees
+    const int kv_end = L - n + last_row / G + 1;
     const int ntiles = (kv_end + kKeys - 1) / kKeys;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
+    if (warp == kProducerWarp) {
+        tc::tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (threadIdx.x == 32 * kMmaWarp) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kConsumers);
+            mbar_init(&b.kv_full[i], 1);
+            mbar_init(&b.kv_empty[i], 1);
         }
-        mbar_init(zeroed, kConsumers);
+        mbar_init(b.s_full, 1);
+        mbar_init(b.p_full, kSoftmaxWarps);
+        mbar_init(b.o_done, 1);
+        mbar_init(b.drain, 1);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
+    // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA reads them
     const int Hq = p.num_q_heads;
-    if (warp < kConsumers) {
-        // Q rows (token r / G, head kvh * G + r % G) into the swizzled tile
-        for (int c = threadIdx.x; c < kRows * (kD / 8); c += kConsumers * 32) {
-            const int r = c >> 4, ch = c & 15;
-            const int row = r0 + r;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (row < nrows) {
-                const int tok = row / G, g = row - tok * G;
-                v = *reinterpret_cast<const uint4*>(
-                    static_cast<const T*>(p.query) +
-                    ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD + ch * 8);
-            }
-            *reinterpret_cast<uint4*>(qsm + swz_q(r, ch)) = v;
+    for (int c = threadIdx.x; c < kRows * (kD / 8); c += kThreads) {
+        const int r = c >> 4, ch = c & 15;
+        const int row = r0 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < nrows) {
+            const int tok = row / G, g = row - tok * G;
+            v = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.query) +
+                                                ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD +
+                                                ch * 8);
         }
+        *reinterpret_cast<uint4*>(qsm + (ch >> 3) * kQHalfBytes + swz(r, ch)) = v;
     }
+    tc::fence_proxy_async_smem();  // the tensor cores read Q through the async proxy
+    tc::fence_before_sync();
     __syncthreads();
-    if (warp == kConsumers) {
-        if (lane == 0) produce(kmap, vmap, p, s, kvh, L, ntiles, stages, full, empty);
-        return;
-    }
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
 
-    // ---- consumer warp: rows 16 * warp + (lane >> 2) and that + 8 ----
-    const uint32_t qbase = smem_addr(qsm);
-    uint32_t qf[kD / 16][4];
-#pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk)
-        ldmatrix_x4(qf[kk], qbase + swz_q(16 * warp + (lane & 15), 2 * kk + (lane >> 4)));
-    int pos[2];
-    bool ok[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int row = r0 + 16 * warp + (lane >> 2) + 8 * h;
-        ok[h] = row < nrows;
-        pos[h] = L - n + (ok[h] ? row / G : 0);
-    }
-    float o[kD / 8][4];
-#pragma unroll
-    for (int i = 0; i < kD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-    const float sl = p.scale_log2;
     bool failed = false;
-    int j = 0;
-    for (; j < ntiles; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait_bounded(&full[st], (j / kStages) & 1)) {
-            failed = true;
-            break;
-        }
-        uint8_t* kt = stages + st * kStageBytes;
-        uint8_t* vt = kt + kTileBytes;
-        const int key0 = j * kKeys;
-        if (key0 + kKeys > L) {
-            // rows past the context may hold anything (NaN included): zero V
-            // there so that their zero weights contribute exactly 0
-            // (only the last tile can reach past L: one use of `zeroed`)
-            const int first = max(L - key0, 0);
-            for (int c = threadIdx.x; c < (kKeys - first) * 16; c += kConsumers * 32) {
-                const int k = first + (c >> 4), ch = c & 15;
-                *reinterpret_cast<uint4*>(vt + (k >> 4) * kBoxBytes + swz16(k & 15, ch)) =
-                    make_uint4(0, 0, 0, 0);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive_one(zeroed);
-            if (!mbar_wait_bounded(zeroed, 0)) {
-                failed = true;
-                ++j;  // this tile's loads have landed
-                break;
-            }
-        }
-        const uint32_t kb = smem_addr(kt), vb = smem_addr(vt);
-        // S = Q K^T for 64 keys: 8 n-tiles of 8 keys
-        float sacc[kKeys / 8][4];
-#pragma unroll
-        for (int i = 0; i < kKeys / 8; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-#pragma unroll
-            for (int np = 0; np < kKeys / 16; ++np) {
-                uint32_t b[4];
-                const int mtx = lane >> 3;
-                const int r = (mtx >> 1) * 8 + (lane & 7);
-                ldmatrix_x4(b, kb + np * kBoxBytes + swz16(r, 2 * kk + (mtx & 1)));
-                Mma<T>::m16n8k16(sacc[2 * np], qf[kk], b[0], b[1]);
-                Mma<T>::m16n8k16(sacc[2 * np + 1], qf[kk], b[2], b[3]);
-            }
-        }
-        // causal mask, online softmax (base 2)
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < kKeys / 8; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int h = i >> 1;
-                const int key = key0 + nt * 8 + 2 * (lane & 3) + (i & 1);
-                const float v = (ok[h] && key <= pos[h]) ? sacc[nt][i] * sl : -INFINITY;
-                sacc[nt][i] = v;
-                mx[h] = fmaxf(mx[h], v);
-            }
-        float alpha[2], mu[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 1));
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(kFull, mx[h], 2));
-            const float mn = fmaxf(m[h], mx[h]);
-            mu[h] = mn == -INFINITY ? 0.f : mn;  // a row with no key yet stays at zero
-            alpha[h] = exp2f(m[h] - mu[h]);
-            m[h] = mn;
-            l[h] *= alpha[h];
-        }
-#pragma unroll
-        for (int i = 0; i < kD / 8; ++i) {
-            o[i][0] *= alpha[0];
-            o[i][1] *= alpha[0];
-            o[i][2] *= alpha[1];
-            o[i][3] *= alpha[1];
-        }
-        // P as A fragments: the C fragments of n-tiles 2k, 2k + 1 are the A
-        // fragment of key step k.  P goes in as a 16-bit high part plus the
-        // 16-bit remainder (two products into one accumulator).
-#pragma unroll
-        for (int k = 0; k < kKeys / 16; ++k) {
-            float pv[2][4];
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    pv[t][i] = exp2f(sacc[2 * k + t][i] - mu[i >> 1]);
-                    l[i >> 1] += pv[t][i];
-                }
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float a = pv[t][2 * h], c = pv[t][2 * h + 1];
-                    const uint32_t w = pack2<T>(a, c);
-                    const float2 back = Storage<T>::to_float2(w);
-                    hi[2 * t + h] = w;
-                    lo[2 * t + h] = pack2<T>(a - back.x, c - back.y);
-                }
-            const int mtx = lane >> 3;
-            const int r = (mtx & 1) * 8 + (lane & 7);
-#pragma unroll
-            for (int dp = 0; dp < kD / 16; ++dp) {
-                uint32_t b[4];
-                ldmatrix_x4_trans(b, vb + k * kBoxBytes + swz16(r, 2 * dp + (mtx >> 1)));
-                Mma<T>::m16n8k16(o[2 * dp], hi, b[0], b[1]);
-                Mma<T>::m16n8k16(o[2 * dp], lo, b[0], b[1]);
-                Mma<T>::m16n8k16(o[2 * dp + 1], hi, b[2], b[3]);
-                Mma<T>::m16n8k16(o[2 * dp + 1], lo, b[2], b[3]);
-            }
-        }
-        // every read of this stage has fed an instruction above: release it
+    if (warp == kProducerWarp) {
+        if (lane == 0) produce(kmap, vmap, p, s, kvh, L, ntiles, stages, b, &failed);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0)
+            issue_mmas<std::is_same<T, __nv_bfloat16>::value>(b, tmem, smem_addr(qsm), stages,
+                                                              ntiles, &failed);
+    } else {
+        softmax_rows<T>(p, b, tmem, stages, L, n, q0, kvh, r0, nrows, ntiles, warp, lane,
+                        &failed);
+    }
+    if (failed) report_error(p.dev_error, PKV_DEVERR_TIMEOUT, s);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == kProducerWarp) {
         __syncwarp();
-        if (lane == 0) mbar_arrive_one(&empty[st]);
-    }
-    if (failed) {
-        // wait (bounded) for this CTA's loads still in flight, then leave
-        for (int k = j; k < ntiles && k < j + kStages; ++k)
-            mbar_wait_bounded(&full[k % kStages], (k / kStages) & 1);
-        if (lane == 0) report_error(p.dev_error, PKV_DEVERR_TIMEOUT, s);
-        return;
-    }
-    // rows' sums over the quad, then normalised 16-bit output
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l[h] += __shfl_xor_sync(kFull, l[h], 1);
-        l[h] += __shfl_xor_sync(kFull, l[h], 2);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (!ok[h]) continue;
-        const int row = r0 + 16 * warp + (lane >> 2) + 8 * h;
-        const int tok = row / G, g = row - tok * G;
-        T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD;
-        const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
-#pragma unroll
-        for (int nt = 0; nt < kD / 8; ++nt)
-            *reinterpret_cast<uint32_t*>(dst + nt * 8 + 2 * (lane & 3)) =
-                pack2<T>(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -392,10 +448,10 @@ extern "C" int pkv_prefill_attention(void* out, const void* query, const void* k
                 (long long)ctas);
     CUtensorMap kmap, vmap;
     int st = encode_paged_map_16bit(&kmap, key_cache, dtype, head_dim, num_kv_heads, block_size,
-                                    num_blocks, block_stride);
+                                    num_blocks, block_stride, 1);
     if (st != PKV_OK) return st;
     st = encode_paged_map_16bit(&vmap, value_cache, dtype, head_dim, num_kv_heads, block_size,
-                                num_blocks, block_stride);
+                                num_blocks, block_stride, 1);
     if (st != PKV_OK) return st;
     DeviceGuard guard(stream, key_cache);
     auto kern = dtype == PKV_BF16 ? paged_prefill_kernel<__nv_bfloat16>
