@@ -7,20 +7,23 @@
 // last n_s of its L_s cached tokens: row i is token p = L_s - n_s + i and
 // attends causally to tokens 0 .. p.
 //
-// One CTA takes 128 rows of one (sequence, KV head): (query token, head of
-// the GQA group) pairs, so each K/V tile is streamed once for the group.
+// One CTA takes 256 rows of one (sequence, KV head) as two 128-row Q tiles:
+// (query token, head of the GQA group) pairs, so each K/V tile is streamed
+// once for the group and both tiles.
 // The work runs on the 5th-generation tensor cores with the accumulators in
 // tensor memory:
 //   - a producer warp brings 128-key K and V tiles through a 2-stage ring
 //     (one TMA box per 16 slots of a block and per 64-dim half);
-//   - an MMA warp issues S = Q K^T (M 128, N 128, K 16 steps; Q and K from
-//     shared memory) into tensor memory, then O += P V with P read from
-//     tensor memory and V from shared memory (B operand MN-major);
-//   - four softmax warps (one tensor-memory lane quarter each, one row per
-//     thread) read S, apply the causal mask, keep the running max and sum,
-//     write P (a 16-bit high part and its 16-bit remainder, two MMAs) and
-//     rescale O when the running max grows by more than 2^8, then write the
-//     normalised output.
+//   - an MMA warp issues, per key tile, S = Q K^T for both Q tiles (M 128,
+//     N 128, K 16 steps; Q and K from shared memory) into tensor memory,
+//     then O += P V for each tile as its P is ready (P read from tensor
+//     memory, V from shared memory as an MN-major B operand), so that the
+//     tensor cores work on one tile while the other tile's softmax runs;
+//   - eight softmax warps, four per Q tile (one tensor-memory lane quarter
+//     each, one row per thread), read S, apply the causal mask, keep the
+//     running max and sum, write P over S (a 16-bit high part and its
+//     16-bit remainder, two MMAs) and rescale O when the running max grows
+//     by more than 2^8, then write the normalised output.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -31,20 +34,23 @@ namespace pkv {
 namespace {
 
 constexpr int kD = 128;                 // head_dim (built)
-constexpr int kRows = 128;              // (token, head) rows per CTA = UMMA M
+constexpr int kRows = 128;              // rows per Q tile = UMMA M
+constexpr int kQTiles = 2;              // Q tiles per CTA
 constexpr int kKeys = 128;              // keys per tile = UMMA N of S, K of P V
 constexpr int kStages = 2;
 constexpr int kHalfBytes = kKeys * 128; // one 64-dim half of a K (or V) tile: 16 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;          // 32 KiB
 constexpr int kStageBytes = 2 * kTileBytes;         // K + V
 constexpr int kQHalfBytes = kRows * 128;            // 16 KiB
-constexpr int kQBytes = 2 * kQHalfBytes;
+constexpr int kQTileBytes = 2 * kQHalfBytes;      // one Q tile, both halves
+constexpr int kQBytes = kQTiles * kQTileBytes;
 constexpr int kBoxKeys = 16;                        // slots per TMA box
-constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4;
+constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4 * kQTiles;
 constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;
-// tensor-memory columns: S | P high | P low | O
-constexpr uint32_t kColS = 0, kColPh = 128, kColPl = 192, kColO = 256, kTmemCols = 512;
-constexpr int kNumBars = 2 * kStages + 4;  // kv_full, kv_empty, s_full, p_full, o_done, drain
+// tensor-memory columns per Q tile t: S (P high | P low written over it
+// once S is read) at 256 t, O at 256 t + 128
+constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = 64, kTmemCols = 512;
+constexpr int kNumBars = 2 * kStages + 3 * kQTiles + 1;  // kv_full/empty, s_full/p_full/o_done per tile, drain
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the max grows by more than 2^8
@@ -80,9 +86,9 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
 struct Bars {
     uint64_t* kv_full;   // [kStages]: TMA bytes landed
     uint64_t* kv_empty;  // [kStages]: the P V MMAs reading the stage completed
-    uint64_t* s_full;    // S in tensor memory
-    uint64_t* p_full;    // P written (and O rescaled) by the softmax warps
-    uint64_t* o_done;    // the P V MMAs of the tile completed
+    uint64_t* s_full;    // [kQTiles]: S in tensor memory
+    uint64_t* p_full;    // [kQTiles]: P written (and O rescaled) by the softmax warps
+    uint64_t* o_done;    // [kQTiles]: the P V MMAs of the tile completed
     uint64_t* drain;     // every MMA issued completed (exit)
 };
 
@@ -142,31 +148,46 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
         tc::fence_after_sync();
         const uint32_t kaddr = smem_addr(stages + st * kStageBytes);
         const uint32_t vaddr = kaddr + kTileBytes;
-        // S = Q K^T: 8 steps of 16 dims (4 per 128-byte swizzle atom)
+        // S = Q K^T of both Q tiles: 8 steps of 16 dims (4 per 128-byte
+        // swizzle atom).  In issue order, S of tile t follows P V of tile t
+        // for the previous key tile, which reads the P written over S.
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * kQHalfBytes + (uint32_t)(kk & 3) * 32;
-            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
-            tc::mma_ss(tmem + kColS, tc::sw128_desc(qaddr + off, 16, 1024),
-                       tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        for (int t = 0; t < kQTiles; ++t) {
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t off = (uint32_t)t * kQTileBytes + (uint32_t)(kk >> 2) * kQHalfBytes +
+                                     (uint32_t)(kk & 3) * 32;
+                const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
+                tc::mma_ss(tmem + kTileCols * t, tc::sw128_desc(qaddr + off, 16, 1024),
+                           tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+            }
+            tc::commit(smem_addr(&b.s_full[t]));
         }
-        tc::commit(smem_addr(b.s_full));
-        if (!mbar_wait_bounded(b.p_full, j & 1)) {
+        // O += P V per tile as its P is ready: 8 steps of 16 keys; V's 8-key
+        // groups 1 KiB apart (SBO), its 64-dim halves 16 KiB apart (LBO)
+        bool ok = true;
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+            if (!mbar_wait_bounded(&b.p_full[t], j & 1)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const uint32_t cs = kTileCols * t;
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk) {
+                const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
+                tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
+            }
+            tc::commit(smem_addr(&b.o_done[t]));
+        }
+        if (!ok) {
             *failed = true;
             break;
         }
-        tc::fence_after_sync();
-        // O += P V: 8 steps of 16 keys; V's 8-key groups 1 KiB apart (SBO),
-        // its 64-dim halves 16 KiB apart (LBO)
-#pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
-            tc::mma_ts(tmem + kColO, tmem + kColPh + kk * 8, vd, kIdPV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-            tc::mma_ts(tmem + kColO, tmem + kColPl + kk * 8, vd, kIdPV, 1u);
-        }
         tc::commit(smem_addr(&b.kv_empty[st]));
-        tc::commit(smem_addr(b.o_done));
     }
     // every MMA issued has completed before the tensor memory is freed
     tc::commit(smem_addr(b.drain));
@@ -184,23 +205,24 @@ template <typename T>
 __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tmem,
                              uint8_t* stages, int L, int n, int q0, int kvh, int r0, int nrows,
                              int ntiles, int warp, int lane, bool* failed) {
-    const int quarter = warp & 3;  // tensor-memory lanes 32 * quarter .. + 31
-    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16);
+    const int t = (warp - kSoftmaxWarp0) >> 2;  // Q tile of this warp
+    const int quarter = warp & 3;              // tensor-memory lanes 32 * quarter .. + 31
+    const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16) + kTileCols * t;
     const int r = 32 * quarter + lane;
-    const int R = r0 + r;
+    const int R = r0 + kRows * t + r;
     const bool ok = R < nrows;
     const int pos = L - n + (ok ? R / p.group : 0);
     const float sl = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     int j = 0;
     for (; j < ntiles; ++j) {
-        if (!warp_wait(b.s_full, j & 1)) break;
+        if (!warp_wait(&b.s_full[t], j & 1)) break;
         tc::fence_after_sync();
         float sv[kKeys];
         {
             uint32_t u[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::ld32(trow + kColS + 32 * c, u[c]);
+            for (int c = 0; c < 4; ++c) tc::ld32(trow + 32 * c, u[c]);
             tc::wait_ld();
             const int key0 = j * kKeys;
 #pragma unroll
@@ -221,7 +243,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         const float mu = m == -INFINITY ? 0.f : m;
         // the P V of the previous tile must be done before P and O change
         if (j > 0) {
-            if (!warp_wait(b.o_done, (j - 1) & 1)) break;
+            if (!warp_wait(&b.o_done[t], (j - 1) & 1)) break;
             tc::fence_after_sync();
             if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -248,19 +270,19 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                 const float2 back = Storage<T>::to_float2(hi[e]);
                 lo[e] = Storage<T>::from_float2(a - back.x, d - back.y);
             }
-            tc::st16(trow + kColPh + 16 * c, hi);
+            tc::st16(trow + 16 * c, hi);  // over S, already read
             tc::st16(trow + kColPl + 16 * c, lo);
         }
         // keys past the context in the last tile: zero their V rows (NaN
         // bit patterns there must not meet their zero weights)
         const int key0 = j * kKeys;
-        if (key0 + kKeys > L) {
+        if (t == 0 && key0 + kKeys > L) {
             const int st = j % kStages;
             if (!warp_wait(&b.kv_full[st], (j / kStages) & 1)) break;
             uint8_t* vt = stages + st * kStageBytes + kTileBytes;
             const int first = max(L - key0, 0);
-            const int t = (warp - kSoftmaxWarp0) * 32 + lane;
-            for (int c = t; c < (kKeys - first) * 16; c += kSoftmaxWarps * 32) {
+            const int tid = (warp - kSoftmaxWarp0) * 32 + lane;  // tile 0's 128 threads
+            for (int c = tid; c < (kKeys - first) * 16; c += 4 * 32) {
                 const int k = first + (c >> 4), ch = c & 15;
                 *reinterpret_cast<uint4*>(vt + (ch >> 3) * kHalfBytes + swz(k, ch)) =
                     make_uint4(0, 0, 0, 0);
@@ -270,9 +292,9 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         tc::wait_st();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive_one(b.p_full);
+        if (lane == 0) mbar_arrive_one(&b.p_full[t]);
     }
-    if (j < ntiles || !warp_wait(b.o_done, (ntiles - 1) & 1)) {
+    if (j < ntiles || !warp_wait(&b.o_done[t], (ntiles - 1) & 1)) {
         *failed = true;
         return;
     }
@@ -311,8 +333,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     uint8_t* stages = smem + kQBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
-    Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + 1,
-           bars + 2 * kStages + 2, bars + 2 * kStages + 3};
+    Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + kQTiles,
+           bars + 2 * kStages + 2 * kQTiles, bars + 2 * kStages + 3 * kQTiles};
 
     // flat grid: the heaviest row tile of every (sequence, KV head) first
     const int pairs = p.num_seqs * p.num_kv_heads;
@@ -324,7 +346,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     const int n = __ldg(p.query_start + s + 1) - q0;
     const int L = __ldg(p.context_lens + s);
     const int nrows = n * G;
-    const int r0 = tile * kRows;
+    const int r0 = tile * kRows * kQTiles;
     if (n < 0 || n > L || n > p.max_query_len ||
         (int64_t)L > (int64_t)p.max_blocks_per_seq * p.block_size) {
         if (tile == p.tiles_per_seq - 1 && kvh == 0 && threadIdx.x == 0)
@@ -332,7 +354,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         return;
     }
     if (r0 >= nrows) return;  // a row tile past this sequence's rows
-    const int last_row = min(nrows, r0 + kRows) - 1;
+    const int last_row = min(nrows, r0 + kRows * kQTiles) - 1;
     const int kv_end = L - n + last_row / G + 1;
     const int ntiles = (kv_end + kKeys - 1) / kKeys;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -346,9 +368,11 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&b.kv_full[i], 1);
             mbar_init(&b.kv_empty[i], 1);
         }
-        mbar_init(b.s_full, 1);
-        mbar_init(b.p_full, kSoftmaxWarps);
-        mbar_init(b.o_done, 1);
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(&b.s_full[t], 1);
+            mbar_init(&b.p_full[t], 4);  // the tile's four softmax warps
+            mbar_init(&b.o_done[t], 1);
+        }
         mbar_init(b.drain, 1);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
@@ -356,8 +380,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA reads them
     const int Hq = p.num_q_heads;
-    for (int c = threadIdx.x; c < kRows * (kD / 8); c += kThreads) {
-        const int r = c >> 4, ch = c & 15;
+    for (int c = threadIdx.x; c < kQTiles * kRows * (kD / 8); c += kThreads) {
+        const int r = c >> 4, ch = c & 15;  // r: row of the CTA's 256
         const int row = r0 + r;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row < nrows) {
@@ -366,7 +390,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                                                 ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD +
                                                 ch * 8);
         }
-        *reinterpret_cast<uint4*>(qsm + (ch >> 3) * kQHalfBytes + swz(r, ch)) = v;
+        *reinterpret_cast<uint4*>(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
+                                  swz(r % kRows, ch)) = v;
     }
     tc::fence_proxy_async_smem();  // the tensor cores read Q through the async proxy
     tc::fence_before_sync();
@@ -441,7 +466,8 @@ extern "C" int pkv_prefill_attention(void* out, const void* query, const void* k
     p.num_blocks = num_blocks;
     p.block_size = block_size;
     p.max_query_len = max_query_len;
-    p.tiles_per_seq = (int)(((int64_t)max_query_len * p.group + kRows - 1) / kRows);
+    p.tiles_per_seq =
+        (int)(((int64_t)max_query_len * p.group + kRows * kQTiles - 1) / (kRows * kQTiles));
     p.scale_log2 = scale * kLog2e;
     const int64_t ctas = (int64_t)p.tiles_per_seq * num_seqs * num_kv_heads;
     PKV_REQUIRE(ctas < (1ll << 31), PKV_ERR_UNSUPPORTED, "pkv_prefill_attention: %lld CTAs",
