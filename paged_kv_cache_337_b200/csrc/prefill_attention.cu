@@ -12,10 +12,10 @@
 // once for the group and both tiles.
 // The work runs on the 5th-generation tensor cores with the accumulators in
 // tensor memory:
-//   - a producer warp brings 128-key K and V tiles through a 2-stage ring
+//   - a producer warp brings 64-key K and V tiles through a 4-stage ring
 //     (one TMA box per 16 slots of a block and per 64-dim half);
 //   - an MMA warp issues, per key tile, S = Q K^T for both Q tiles (M 128,
-//     N 128, K 16 steps; Q and K from shared memory) into tensor memory,
+//     N 64, K 16 steps; Q and K from shared memory) into tensor memory,
 //     then O += P V for each tile as its P is ready (P read from tensor
 //     memory, V from shared memory as an MN-major B operand), so that the
 //     tensor cores work on one tile while the other tile's softmax runs;
@@ -36,9 +36,9 @@ namespace {
 constexpr int kD = 128;                 // head_dim (built)
 constexpr int kRows = 128;              // rows per Q tile = UMMA M
 constexpr int kQTiles = 2;              // Q tiles per CTA
-constexpr int kKeys = 128;              // keys per tile = UMMA N of S, K of P V
-constexpr int kStages = 2;
-constexpr int kHalfBytes = kKeys * 128; // one 64-dim half of a K (or V) tile: 16 KiB
+constexpr int kKeys = 64;               // keys per tile = UMMA N of S, K of P V
+constexpr int kStages = 4;
+constexpr int kHalfBytes = kKeys * 128; // one 64-dim half of a K (or V) tile: 8 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;          // 32 KiB
 constexpr int kStageBytes = 2 * kTileBytes;         // K + V
 constexpr int kQHalfBytes = kRows * 128;            // 16 KiB
@@ -47,9 +47,9 @@ constexpr int kQBytes = kQTiles * kQTileBytes;
 constexpr int kBoxKeys = 16;                        // slots per TMA box
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4 * kQTiles;
 constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;
-// tensor-memory columns per Q tile t: S (P high | P low written over it
-// once S is read) at 256 t, O at 256 t + 128
-constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = 64, kTmemCols = 512;
+// tensor-memory columns per Q tile t: S (64 columns; P high | P low, 32
+// each, written over it once S is read) at 256 t, O at 256 t + 128
+constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = kKeys / 2, kTmemCols = 512;
 constexpr int kNumBars = 2 * kStages + 3 * kQTiles + 1;  // kv_full/empty, s_full/p_full/o_done per tile, drain
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -139,55 +139,72 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
                            int ntiles, bool* failed) {
     constexpr uint32_t kIdS = tc::f16_idesc(BF16, false, kRows, kKeys);  // K: K-major B
     constexpr uint32_t kIdPV = tc::f16_idesc(BF16, true, kRows, kD);     // V: MN-major B
-    for (int j = 0; j < ntiles; ++j) {
+    // S = Q K^T of Q tile t for key tile j: 8 steps of 16 dims (4 per
+    // 128-byte swizzle atom).  In issue order it follows P V of tile t for
+    // key tile j - 1, which reads the P written over S.
+    auto issue_s = [&](int t, int j) {
+        const uint32_t kaddr = smem_addr(stages + (j % kStages) * kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (uint32_t)t * kQTileBytes + (uint32_t)(kk >> 2) * kQHalfBytes +
+                                 (uint32_t)(kk & 3) * 32;
+            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
+            tc::mma_ss(tmem + kTileCols * t, tc::sw128_desc(qaddr + off, 16, 1024),
+                       tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(smem_addr(&b.s_full[t]));
+    };
+    // O += P V of Q tile t for key tile j: 8 steps of 16 keys; V's 8-key
+    // groups 1 KiB apart (SBO), its 64-dim halves 16 KiB apart (LBO)
+    auto issue_pv = [&](int t, int j) {
+        const uint32_t vaddr = smem_addr(stages + (j % kStages) * kStageBytes) + kTileBytes;
+        const uint32_t cs = kTileCols * t;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+            const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
+            tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
+        }
+        tc::commit(smem_addr(&b.o_done[t]));
+    };
+    // Ping-pong: while one tile's softmax runs, the tensor cores run the
+    // other tile's P V and its next S.
+    //   S_A(0) S_B(0) | P_A(j): PV_A(j) S_A(j+1) | P_B(j): PV_B(j) S_B(j+1)
+    if (!mbar_wait_bounded(&b.kv_full[0], 0)) {
+        *failed = true;
+    } else {
+        tc::fence_after_sync();
+        issue_s(0, 0);
+        issue_s(1, 0);
+    }
+    for (int j = 0; j < ntiles && !*failed; ++j) {
         const int st = j % kStages;
-        if (!mbar_wait_bounded(&b.kv_full[st], (j / kStages) & 1)) {
+        const bool more = j + 1 < ntiles;
+        // tile A
+        if (!mbar_wait_bounded(&b.p_full[0], j & 1)) {
             *failed = true;
             break;
         }
         tc::fence_after_sync();
-        const uint32_t kaddr = smem_addr(stages + st * kStageBytes);
-        const uint32_t vaddr = kaddr + kTileBytes;
-        // S = Q K^T of both Q tiles: 8 steps of 16 dims (4 per 128-byte
-        // swizzle atom).  In issue order, S of tile t follows P V of tile t
-        // for the previous key tile, which reads the P written over S.
-#pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint32_t off = (uint32_t)t * kQTileBytes + (uint32_t)(kk >> 2) * kQHalfBytes +
-                                     (uint32_t)(kk & 3) * 32;
-                const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
-                tc::mma_ss(tmem + kTileCols * t, tc::sw128_desc(qaddr + off, 16, 1024),
-                           tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-            }
-            tc::commit(smem_addr(&b.s_full[t]));
-        }
-        // O += P V per tile as its P is ready: 8 steps of 16 keys; V's 8-key
-        // groups 1 KiB apart (SBO), its 64-dim halves 16 KiB apart (LBO)
-        bool ok = true;
-#pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-            if (!mbar_wait_bounded(&b.p_full[t], j & 1)) {
-                ok = false;
+        issue_pv(0, j);
+        if (more) {
+            if (!mbar_wait_bounded(&b.kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1)) {
+                *failed = true;
                 break;
             }
             tc::fence_after_sync();
-            const uint32_t cs = kTileCols * t;
-#pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk) {
-                const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
-                tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
-            }
-            tc::commit(smem_addr(&b.o_done[t]));
+            issue_s(0, j + 1);
         }
-        if (!ok) {
+        // tile B
+        if (!mbar_wait_bounded(&b.p_full[1], j & 1)) {
             *failed = true;
             break;
         }
-        tc::commit(smem_addr(&b.kv_empty[st]));
+        tc::fence_after_sync();
+        issue_pv(1, j);
+        tc::commit(smem_addr(&b.kv_empty[st]));  // both tiles' P V of this stage
+        if (more) issue_s(1, j + 1);
     }
     // every MMA issued has completed before the tensor memory is freed
     tc::commit(smem_addr(b.drain));
@@ -220,13 +237,13 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         tc::fence_after_sync();
         float sv[kKeys];
         {
-            uint32_t u[4][32];
+            uint32_t u[kKeys / 32][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::ld32(trow + 32 * c, u[c]);
+            for (int c = 0; c < kKeys / 32; ++c) tc::ld32(trow + 32 * c, u[c]);
             tc::wait_ld();
             const int key0 = j * kKeys;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < kKeys / 32; ++c)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int key = key0 + 32 * c + e;
@@ -259,7 +276,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         }
         // P = 2^(s - m) as a 16-bit high part and the 16-bit remainder
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kKeys / 32; ++c) {
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
