@@ -586,6 +586,86 @@ def run_pkv(args, spec, world, rank, local):
 
 
 SWAP_WORKLOAD = "swap_7b_s256_q64_h32_d128_bs16_bf16"
+COW_LAYERS_WORKLOAD = "cow_layers_l32_p112_h32_d128_bs16_bf16"
+
+
+def run_cow_layers(args, world, rank, local):
+    """Copy-on-write over a 32-layer cache: the shared-prefix fork step's 112
+    (src, dst) pairs copied in every layer by one pkv_copy_blocks_layers
+    launch, against 32 pkv_copy_blocks launches.  `value` is the bytes
+    moved (each pair's K and V block read and written, every layer) over
+    the device time of the one-launch copy; the roofline peak is HBM."""
+    from paged_kv_cache_337_b200 import _abi
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _abi.lib()
+    layers, pairs_n, nb, bs, hkv, d = 32, 112, 2048, 16, 32, 128
+    dt = torch.bfloat16
+    g = torch.Generator(dev).manual_seed(4000 + rank)
+    ks = [torch.empty((nb, bs, hkv, d), dtype=dt, device=dev) for _ in range(layers)]
+    vs = [torch.empty((nb, bs, hkv, d), dtype=dt, device=dev) for _ in range(layers)]
+    for t in ks + vs:
+        t.view(-1)[:: 4096].normal_(generator=g)
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(4100 + rank))
+    pairs = torch.stack([perm[:pairs_n], perm[pairs_n:2 * pairs_n]], 1).to(torch.int32).to(dev)
+    kp, vp = _abi.layer_pointers(ks, dev), _abi.layer_pointers(vs, dev)
+    err = torch.zeros(2, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    step_bytes = pairs_n * layers * 2 * 2 * bs * hkv * d * 2
+
+    def one_launch():
+        _abi.pkv_copy_blocks_layers(ks, vs, pairs, dev_error=err, stream=stream, key_ptrs=kp,
+                                    value_ptrs=vp)
+
+    def per_layer():
+        for l in range(layers):
+            _abi.pkv_copy_blocks(ks[l], vs[l], pairs, dev_error=err, stream=stream)
+
+    def timed(fn, K):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs) / K
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    K = args.steps
+    ms = timed(one_launch, K)
+    ms_layers = timed(per_layer, K)
+    barrier(world)
+    clock_info = clocks.stop() if clocks else None
+    t_max = max_over_ranks(ms, world, dev)
+    value = sum_over_ranks(step_bytes, world, dev) / (t_max * 1e-3) / 1e9
+    peak, peak_kind = measured_peak()
+    if err.tolist() != [0, 0]:
+        raise RuntimeError("device error %s" % err.tolist())
+    if rank == 0:
+        line = {
+            "metric": "multi-layer copy-on-write GB/s (read + write)", "value": round(value, 2),
+            "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": round(t_max, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": COW_LAYERS_WORKLOAD, "layers": layers, "pairs": pairs_n,
+                       "block_bytes_kv": 2 * bs * hkv * d * 2, "step_gb": step_bytes / 1e9,
+                       "per_layer_launches_ms": round(ms_layers, 4)},
+            "roofline": {"bound": "hbm", "achieved": round(value, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(value / peak, 4), "traffic": None,
+                         "kernel": "copy_blocks_layers_kernel", "peak_source": peak_kind},
+            "e2e": None, "cpu_baseline": None, "gpu_launches": K * (1 + layers),
+            "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
 
 
 def host_link_peak(dev, nbytes=1 << 30):
@@ -988,6 +1068,14 @@ def main():
     args = parse_args()
     from paged_kv_cache_337_b200 import workloads as W
 
+    if args.workload == COW_LAYERS_WORKLOAD:
+        world, rank, local = dist_setup()
+        try:
+            run_cow_layers(args, world, rank, local)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+        return
     if args.workload == PREFILL_WORKLOAD:
         world, rank, local = dist_setup()
         try:

@@ -217,6 +217,7 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
  *   context_lens     device int32 [num_seqs]: L, the chunk's tokens included
  *   query_start      device int32 [num_seqs + 1], non-decreasing from 0
  *   max_query_len    host bound on every n_s: it sizes the grid
+ *   scale            > 0 (PKV_ERR_INVALID otherwise)
  * A sequence with n_s > L, n_s > max_query_len or L > max_blocks_per_seq *
  * block_size is reported (PKV_DEVERR_CONTEXT_LEN) and its rows are left
  * unwritten.  Built for head_dim 128 and block_size a multiple of 16;
@@ -406,6 +407,8 @@ PKV_API int pkv_pool_block_tables(const pkv_pool* pool, int n, const int64_t* se
                           int32_t* out, int max_blocks_per_seq, int32_t fill,
                           int32_t* context_lens, int32_t* max_context_len);
 
+/* Free blocks, total blocks and block size of the pool (negative status on
+ * a NULL pool). */
 PKV_API int pkv_pool_num_free(const pkv_pool* pool);
 PKV_API int pkv_pool_num_blocks(const pkv_pool* pool);
 PKV_API int pkv_pool_block_size(const pkv_pool* pool);
@@ -452,7 +455,10 @@ PKV_API int pkv_seq_swap_out(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int
 PKV_API int pkv_seq_swap_in(pkv_pool* pool, int64_t seq_id, int32_t* pairs, int cap,
                             int* num_pairs);
 
+/* *swapped = 1 while the sequence's blocks are on the host, else 0. */
 PKV_API int pkv_seq_is_swapped(const pkv_pool* pool, int64_t seq_id, int* swapped);
+
+/* Free host blocks (negative status on a NULL pool; 0 without a host pool). */
 PKV_API int pkv_pool_num_free_host(const pkv_pool* pool);
 
 /* The host free stack from bottom to top (the next block taken is the last). */

@@ -235,6 +235,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
     for (; j < ntiles; ++j) {
         if (!warp_wait(&b.s_full[t], j & 1)) break;
         tc::fence_after_sync();
+        // raw scores; the scale (positive) is applied with the max subtraction
         float sv[kKeys];
         {
             uint32_t u[kKeys / 32][32];
@@ -242,17 +243,27 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
             for (int c = 0; c < kKeys / 32; ++c) tc::ld32(trow + 32 * c, u[c]);
             tc::wait_ld();
             const int key0 = j * kKeys;
+            // the causal mask only where some row of the warp stops inside
+            // this tile (or a row is past the sequence's rows)
+            if (__all_sync(0xffffffffu, ok && key0 + kKeys - 1 <= pos)) {
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c)
+                for (int c = 0; c < kKeys / 32; ++c)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int key = key0 + 32 * c + e;
-                    sv[32 * c + e] = (ok && key <= pos) ? __uint_as_float(u[c][e]) * sl : -INFINITY;
-                }
+                    for (int e = 0; e < 32; ++e) sv[32 * c + e] = __uint_as_float(u[c][e]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kKeys / 32; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = key0 + 32 * c + e;
+                        sv[32 * c + e] = (ok && key <= pos) ? __uint_as_float(u[c][e]) : -INFINITY;
+                    }
+            }
         }
-        float mt = -INFINITY;
+        float raw_max = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < kKeys; ++e) mt = fmaxf(mt, sv[e]);
+        for (int e = 0; e < kKeys; ++e) raw_max = fmaxf(raw_max, sv[e]);
+        const float mt = raw_max * sl;            // the tile's max in base-2 units
         const bool resc = mt > m + kRescaleLog2;  // also the first finite max
         const float alpha = resc ? exp2f(m - mt) : 1.f;
         if (resc) m = mt;
@@ -280,8 +291,8 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const float a = exp2f(sv[32 * c + 2 * e] - mu);
-                const float d = exp2f(sv[32 * c + 2 * e + 1] - mu);
+                const float a = exp2f(fmaf(sv[32 * c + 2 * e], sl, -mu));
+                const float d = exp2f(fmaf(sv[32 * c + 2 * e + 1], sl, -mu));
                 l += a + d;
                 hi[e] = Storage<T>::from_float2(a, d);
                 const float2 back = Storage<T>::to_float2(hi[e]);
@@ -453,6 +464,8 @@ extern "C" int pkv_prefill_attention(void* out, const void* query, const void* k
                 "pkv_prefill_attention: dtype %d", (int)dtype);
     PKV_REQUIRE(head_dim == kD, PKV_ERR_UNSUPPORTED,
                 "pkv_prefill_attention: head_dim %d (built: 128)", head_dim);
+    PKV_REQUIRE(scale > 0.f, PKV_ERR_INVALID, "pkv_prefill_attention: scale %g (must be > 0)",
+                (double)scale);
     PKV_REQUIRE(num_seqs >= 0 && max_query_len >= 0 && num_q_heads > 0 && num_kv_heads > 0 &&
                     num_q_heads % num_kv_heads == 0 && max_blocks_per_seq >= 0,
                 PKV_ERR_INVALID, "pkv_prefill_attention: bad sizes");
