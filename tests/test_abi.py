@@ -72,3 +72,12 @@ def test_argument_errors_are_reported_before_any_launch(lib):
                                   16 * 8 * 64, 1.0, 24, None, 0, 1, None, None)
     assert st == _abi.PKV_ERR_INVALID  # partition of 24 tokens is not a multiple of 16
     assert C.sizeof(C.c_void_p) == 8
+
+
+def test_prefill_rejects_a_non_positive_scale_before_any_device_work():
+    # the check precedes every pointer or device access, so it runs on CPU
+    L = _abi.lib()
+    st = L.pkv_prefill_attention(None, None, None, None, None, 1, None, None, 1, 1, 4, 4, 128,
+                                 8, 16, 16 * 4 * 128, 0.0, _abi.PKV_BF16, None, None)
+    assert st == _abi.PKV_ERR_INVALID
+    assert b"scale" in L.pkv_last_error()
