@@ -505,38 +505,56 @@ def run_pkv(args, spec, world, rank, local):
     # ---- end to end through the public step API from pinned host memory ----
     # Per step: the step's q, k and v go up in one copy from pinned memory,
     # the host pool reserves the slots and the metadata goes up in one copy,
-    # the kernels run, and the attention output comes back to the host.  The
-    # pool's work for step i+1 runs while step i is on the GPU (it does not
-    # depend on step i's output; the next q, k, v would).
+    # the kernels run, and the attention output comes back to the host; the
+    # host waits for it before the step ends.  The pool's work and the input
+    # upload for step i+1 (on a second stream, into the other of two input
+    # buffers) run while step i is on the GPU: neither depends on step i's
+    # output.
     e2e = None
     if e2e_steps:
         nq, nk = S * Hq * D, S * Hkv * D
         h_in = [torch.randn(nq + 2 * nk).to(dt).pin_memory() for _ in range(2)]
-        d_in = torch.empty(nq + 2 * nk, dtype=dt, device=dev)
-        dq = d_in[:nq].view(S, Hq, D)
-        dk = d_in[nq:nq + nk].view(S, Hkv, D)
-        dv = d_in[nq + nk:].view(S, Hkv, D)
+        d_in = [torch.empty(nq + 2 * nk, dtype=dt, device=dev) for _ in range(2)]
+        views = [(b[:nq].view(S, Hq, D), b[nq:nq + nk].view(S, Hkv, D),
+                  b[nq + nk:].view(S, Hkv, D)) for b in d_in]
         hout = torch.empty((S, Hq, D), dtype=dt).pin_memory()
+        copy_stream = torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
+        ev_used = [torch.cuda.Event() for _ in range(2)]  # step using buffer b done
+        ev_out = torch.cuda.Event()                       # step result on the host
         e2e_bytes = 0
         h2d = d2h = 0
         barrier(world)
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            prep = cache.prepare_step(ids)
-            for i in range(e2e_steps):
-                d_in.copy_(h_in[i % 2], non_blocking=True)
+        with torch.cuda.stream(copy_stream):
+            d_in[0].copy_(h_in[0], non_blocking=True)
+            ev_in[0].record(copy_stream)
+        prep = cache.prepare_step(ids)
+        for i in range(e2e_steps):
+            b = i % 2
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev_in[b])
                 cache.upload_step(prep, stream)
+                dq, dk, dv = views[b]
                 cache.launch_step(prep, dq, dk, dv, out, stream=stream)
+                ev_used[b].record(stream)
                 hout.copy_(out, non_blocking=True)
-                lens = prep["st"]["h_lens"].tolist()
-                e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
-                              copy_bytes(spec, prep["num_pairs"], fp8))
-                h2d = d_in.numel() * 2 + prep["st"]["h"].numel() * 4
-                d2h = hout.numel() * 2
-                if i + 1 < e2e_steps:
-                    prep = cache.prepare_step(ids)  # overlaps the GPU work of step i
-                stream.synchronize()
+                ev_out.record(stream)
+            lens = prep["st"]["h_lens"].tolist()
+            e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
+                          copy_bytes(spec, prep["num_pairs"], fp8))
+            h2d = d_in[b].numel() * 2 + prep["st"]["h"].numel() * 4
+            d2h = hout.numel() * 2
+            if i + 1 < e2e_steps:
+                nb_ = 1 - b
+                with torch.cuda.stream(copy_stream):
+                    if i >= 1:
+                        copy_stream.wait_event(ev_used[nb_])  # step i-1 done with it
+                    d_in[nb_].copy_(h_in[(i + 1) % 2], non_blocking=True)
+                    ev_in[nb_].record(copy_stream)
+                prep = cache.prepare_step(ids)  # overlaps the GPU work of step i
+            ev_out.synchronize()
         e2e_s = time.perf_counter() - t0
         barrier(world)
         e2e_s = max_over_ranks(e2e_s, world, dev)
