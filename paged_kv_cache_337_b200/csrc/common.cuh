@@ -178,33 +178,6 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
     return r;
 }
 
-// c + a.lo * b.lo + a.hi * b.hi for two f16x2 words, by the mixed-precision
-// fma (f16 operands widened exactly, the product and sum in fp32).
-__device__ __forceinline__ float dot2_f16_f32(uint32_t a, uint32_t b, float c) {
-    float d;
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\t"
-        "mov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.f16 %0, al, bl, %3;\n\t"
-        "fma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
-        : "=f"(d)
-        : "r"(a), "r"(b), "f"(c));
-    return d;
-}
-
-// Four e4m3 codes (one 32-bit word, lowest byte first) to four floats.
-__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float (&v)[4]) {
-    const uint32_t a = e4m3x2_to_f16x2((uint16_t)(w & 0xffffu));
-    const uint32_t b = e4m3x2_to_f16x2((uint16_t)(w >> 16));
-    __half2 ha, hb;
-    memcpy(&ha, &a, 4);
-    memcpy(&hb, &b, 4);
-    const float2 fa = __half22float2(ha), fb = __half22float2(hb);
-    v[0] = fa.x;
-    v[1] = fa.y;
-    v[2] = fb.x;
-    v[3] = fb.y;
-}
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

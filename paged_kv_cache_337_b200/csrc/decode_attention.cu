@@ -129,38 +129,17 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int s, bool* b
 // ---------------------------------------------------------------------------
 // Per-warp arithmetic, G == 1: FFMA + shuffles
 // ---------------------------------------------------------------------------
-// FP8 (e4m3 caches): the lane's query dims are also kept as f16 pairs,
-// scaled by a power of two into f16 range, so that the K dot products run
-// on the mixed-precision fma straight from the widened codes.
-template <typename T, int D, bool FP8 = false>
+// (16-bit caches; e4m3 caches take the tensor-core path for every group)
+template <typename T, int D>
 struct GemvWarp {
     static constexpr int DV = D / 32;  // dims per lane
     static constexpr int GP = 1;       // heads held (padded)
     static constexpr bool kMma = false;
     float q[DV], o[DV], m, l;
-    uint32_t qh[DV / 2];               // e4m3 caches: q * 2^sh as f16x2
-    float qinv;                        // 2^-sh
 
     __device__ __forceinline__ void init(const DecodeParams& p, int s, int kvh, int lane) {
         const T* qrow = static_cast<const T*>(p.query) + ((int64_t)s * p.num_q_heads + kvh) * D;
         load(reinterpret_cast<const uint8_t*>(qrow + lane * DV), q);
-        qinv = 1.f;
-        if constexpr (FP8) {
-            float mx = 0.f;
-#pragma unroll
-            for (int j = 0; j < DV; ++j) mx = fmaxf(mx, fabsf(q[j]));
-#pragma unroll
-            for (int x = 1; x < 32; x <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, x));
-            // largest |q| into [2^14, 2^15)
-            int ex = 0;
-            frexpf(mx, &ex);
-            const int sh = mx > 0.f ? max(-120, min(120, 15 - ex)) : 0;
-            const float qs = ldexpf(1.f, sh);
-            qinv = ldexpf(1.f, -sh);
-#pragma unroll
-            for (int j = 0; j < DV / 2; ++j)
-                qh[j] = Storage<__half>::from_float2(q[2 * j] * qs, q[2 * j + 1] * qs);
-        }
 #pragma unroll
         for (int j = 0; j < DV; ++j) o[j] = 0.f;
         m = -INFINITY;
@@ -182,47 +161,22 @@ struct GemvWarp {
     // lane's DV elements of row r of a swizzled tile
     __device__ __forceinline__ static const uint8_t* at(const uint8_t* tile, int r, int lane) {
         const int d0 = lane * DV;
-        if constexpr (FP8) {
-            // e4m3 tile: one 128-byte row per token, 16-byte chunks swizzled
-            return tile + r * 128 + ((((d0 >> 4) ^ (r & 7))) << 4) + (d0 & 15);
-        } else {
-            return tile + swz(r, d0 >> 3) + (d0 & 7) * 2;
-        }
+        return tile + swz(r, d0 >> 3) + (d0 & 7) * 2;
     }
 
-    // lane's DV cache elements of row r as floats (codes, before the scale)
-    __device__ __forceinline__ static void load_kv(const uint8_t* tile, int r, int lane,
-                                                   float (&v)[DV]) {
-        if constexpr (FP8) {
-            static_assert(DV == 4, "e4m3 caches are built for head_dim 128");
-            e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(at(tile, r, lane)), v);
-        } else {
-            load(at(tile, r, lane), v);
-        }
-    }
-
-    // One tile.  scale_log2 multiplies q.k (with any K dequantisation scale
-    // folded in); vscale multiplies the V rows (1 for 16-bit caches).
+    // One tile.  scale_log2 multiplies q.k; vscale multiplies the V rows.
     __device__ __forceinline__ void tile(const uint8_t* kt, const uint8_t* vt, int valid,
                                          float scale_log2, int lane, float vscale = 1.f) {
         float part[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            if constexpr (FP8) {
-                static_assert(DV == 4, "e4m3 caches are built for head_dim 128");
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(at(kt, r, lane));
-                const float acc = dot2_f16_f32(e4m3x2_to_f16x2((uint16_t)w), qh[0], 0.f);
-                part[r] = dot2_f16_f32(e4m3x2_to_f16x2((uint16_t)(w >> 16)), qh[1], acc);
-            } else {
-                float k[DV];
-                load_kv(kt, r, lane, k);
-                float acc = 0.f;
+            float k[DV];
+            load(at(kt, r, lane), k);
+            float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
-                part[r] = acc;
-            }
+            for (int j = 0; j < DV; ++j) acc = fmaf(q[j], k[j], acc);
+            part[r] = acc;
         }
-        if constexpr (FP8) scale_log2 *= qinv;
         // reduce-scatter the 16 partial sums over the 32 lanes: after the
         // rounds with masks 16, 8, 4, 2 and a final pairwise add, lane l
         // holds the full dot product of token l / 2
@@ -273,7 +227,7 @@ struct GemvWarp {
         for (int rr = 0; rr < 16; ++rr) {
             const float pb = __shfl_sync(kFull, prv, rr * 2);
             float v[DV];
-            load_kv(vt, rr, lane, v);
+            load(at(vt, rr, lane), v);
 #pragma unroll
             for (int j = 0; j < DV; ++j) o[j] = fmaf(pb, v[j], o[j]);
         }
@@ -609,7 +563,8 @@ struct MmaWarp {
 template <int D, bool FP8, bool MMA>
 struct Plan {
     static_assert(!FP8 || D == 128, "e4m3 caches are built for head_dim 128");
-    static constexpr int kStages = FP8 ? (MMA ? 3 : 4) : Geom<D>::kStages;
+    static_assert(!FP8 || MMA, "e4m3 caches run on the tensor-core path");
+    static constexpr int kStages = FP8 ? 3 : Geom<D>::kStages;
     static constexpr int kTileBytes = FP8 ? kTile * D : Geom<D>::kKBytes;  // K (or V) as stored
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr size_t kRing = (size_t)kWarps * kStages * kStageBytes;
@@ -1016,8 +971,13 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
 template <typename T, int D, bool FP8>
 int dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
                    int num_kv_heads, cudaStream_t stream) {
-    if (p.group == 1)
-        return launch_decode<T, D, GemvWarp<T, D, FP8>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+    // e4m3 caches take the tensor-core path for every group size: its
+    // conversions are cheaper per tile than the GEMV's, and the tensor pipe
+    // is otherwise idle (G = 1 uses one of the eight MMA columns)
+    if constexpr (!FP8) {
+        if (p.group == 1)
+            return launch_decode<T, D, GemvWarp<T, D>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+    }
     if (p.group <= 8)
         return launch_decode<T, D, MmaWarp<T, D, 1, FP8>, FP8>(kmap, vmap, p, num_kv_heads,
                                                                stream);
