@@ -50,7 +50,7 @@ constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;
 // tensor-memory columns per Q tile t: S (64 columns; P high | P low, 32
 // each, written over it once S is read) at 256 t, O at 256 t + 128
 constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = kKeys / 2, kTmemCols = 512;
-constexpr int kNumBars = 2 * kStages + 3 * kQTiles + 1;  // kv_full/empty, s_full/p_full/o_done per tile, drain
+constexpr int kNumBars = 2 * kStages + 3 * kQTiles + 2;  // kv_full/empty, s_full/p_full/o_done per tile, drain, q_ready
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the max grows by more than 2^8
@@ -90,6 +90,7 @@ struct Bars {
     uint64_t* p_full;    // [kQTiles]: P written (and O rescaled) by the softmax warps
     uint64_t* o_done;    // [kQTiles]: the P V MMAs of the tile completed
     uint64_t* drain;     // every MMA issued completed (exit)
+    uint64_t* q_ready;   // the Q tiles are staged (every staging warp arrived)
 };
 
 // Producer: lane 0 of warp 0.  A box past the context still loads a block
@@ -362,7 +363,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + kQTiles,
-           bars + 2 * kStages + 2 * kQTiles, bars + 2 * kStages + 3 * kQTiles};
+           bars + 2 * kStages + 2 * kQTiles, bars + 2 * kStages + 3 * kQTiles,
+           bars + 2 * kStages + 3 * kQTiles + 1};
 
     // flat grid: the heaviest row tile of every (sequence, KV head) first
     const int pairs = p.num_seqs * p.num_kv_heads;
@@ -402,41 +404,55 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&b.o_done[t], 1);
         }
         mbar_init(b.drain, 1);
+        mbar_init(b.q_ready, kThreads / 32 - 1);  // every warp but the producer
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
-    // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA reads them
-    const int Hq = p.num_q_heads;
-    for (int c = threadIdx.x; c < kQTiles * kRows * (kD / 8); c += kThreads) {
-        const int r = c >> 4, ch = c & 15;  // r: row of the CTA's 256
-        const int row = r0 + r;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < nrows) {
-            const int tok = row / G, g = row - tok * G;
-            v = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.query) +
-                                                ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD +
-                                                ch * 8);
-        }
-        *reinterpret_cast<uint4*>(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
-                                  swz(r % kRows, ch)) = v;
-    }
-    tc::fence_proxy_async_smem();  // the tensor cores read Q through the async proxy
     tc::fence_before_sync();
-    __syncthreads();
+    __syncthreads();  // barriers initialised, tensor memory allocated
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
     bool failed = false;
     if (warp == kProducerWarp) {
+        // K/V do not depend on Q: stream them while the other warps stage it
         if (lane == 0) produce(kmap, vmap, p, s, kvh, L, ntiles, stages, b, &failed);
-    } else if (warp == kMmaWarp) {
-        if (lane == 0)
-            issue_mmas<std::is_same<T, __nv_bfloat16>::value>(b, tmem, smem_addr(qsm), stages,
-                                                              ntiles, &failed);
     } else {
-        softmax_rows<T>(p, b, tmem, stages, L, n, q0, kvh, r0, nrows, ntiles, warp, lane,
-                        &failed);
+        // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA
+        // reads them, staged by every warp but the producer
+        const int Hq = p.num_q_heads;
+        for (int c = threadIdx.x - 32; c < kQTiles * kRows * (kD / 8); c += kThreads - 32) {
+            const int r = c >> 4, ch = c & 15;  // r: row of the CTA's 256
+            const int row = r0 + r;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (row < nrows) {
+                const int tok = row / G, g = row - tok * G;
+                v = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.query) +
+                                                    ((int64_t)(q0 + tok) * Hq + kvh * G + g) *
+                                                        kD +
+                                                    ch * 8);
+            }
+            *reinterpret_cast<uint4*>(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
+                                      swz(r % kRows, ch)) = v;
+        }
+        tc::fence_proxy_async_smem();  // the tensor cores read Q through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive_one(b.q_ready);
+        if (warp == kMmaWarp) {
+            if (lane == 0) {
+                if (!mbar_wait_bounded(b.q_ready, 0)) {
+                    failed = true;
+                } else {
+                    tc::fence_after_sync();
+                    issue_mmas<std::is_same<T, __nv_bfloat16>::value>(b, tmem, smem_addr(qsm),
+                                                                      stages, ntiles, &failed);
+                }
+            }
+        } else {
+            softmax_rows<T>(p, b, tmem, stages, L, n, q0, kvh, r0, nrows, ntiles, warp, lane,
+                            &failed);
+        }
     }
     if (failed) report_error(p.dev_error, PKV_DEVERR_TIMEOUT, s);
     tc::fence_before_sync();
