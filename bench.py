@@ -41,9 +41,12 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "paged decode attention effective KV GB/s (% of HBM peak); decode tok/s"
+# the committed ncu summaries that give a decode workload's DRAM bytes per
+# launch, by workload name; other workloads report traffic null
 PROFILE_TRAFFIC = {
-    False: os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md"),
-    True: os.path.join(ROOT, "profiles", "decode_attention_fp8_7b_s256.md"),
+    "7b_s256_h32_d128_bs16_bf16": os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md"),
+    "7b_s256_h32_d128_bs16_bf16_kv_e4m3": os.path.join(ROOT, "profiles",
+                                                        "decode_attention_fp8_7b_s256.md"),
 }
 
 
@@ -213,14 +216,14 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def profiled_traffic(source_digest, fp8=False):
+def profiled_traffic(source_digest, workload):
     """DRAM bytes per launch of the decode kernel from the committed ncu
-    summary, or None when that summary is missing or was taken on other
-    kernel source."""
+    summary of this workload, or None when there is none or it was taken on
+    other kernel source."""
     try:
-        with open(PROFILE_TRAFFIC[fp8]) as f:
+        with open(PROFILE_TRAFFIC[workload]) as f:
             text = f.read()
-    except OSError:
+    except (KeyError, OSError):
         return None
     vals = {}
     for line in text.splitlines():
@@ -572,7 +575,7 @@ def run_pkv(args, spec, world, rank, local):
                          "repeated %d times, %.1f s" % (n, S, Hq, reps, secs)}
 
     if rank == 0:
-        traffic = profiled_traffic(kernel_source_digest(), fp8)
+        traffic = profiled_traffic(kernel_source_digest(), workload_name(spec, fp8))
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),

@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "packed_f32.cuh"
 #include "tcgen05.cuh"
 #include "tensor_maps.h"
 
@@ -261,12 +262,9 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                     }
             }
         }
-        float raw_max = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < kKeys; ++e) raw_max = fmaxf(raw_max, sv[e]);
-        const float mt = raw_max * sl;            // the tile's max in base-2 units
-        const bool resc = mt > m + kRescaleLog2;  // also the first finite max
-        const float alpha = resc ? exp2f(m - mt) : 1.f;
+        const float mt = max_tree<kKeys>(sv) * sl;  // the tile's max in base-2 units
+        const bool resc = mt > m + kRescaleLog2;    // also the first finite max
+        const float alpha = resc ? ex2_approx(m - mt) : 1.f;
         if (resc) m = mt;
         l *= alpha;
         const float mu = m == -INFINITY ? 0.f : m;
@@ -286,22 +284,29 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                 }
             }
         }
-        // P = 2^(s - m) as a 16-bit high part and the 16-bit remainder
+        // P = 2^(s - m) as a 16-bit high part and the 16-bit remainder, on
+        // key pairs (packed fp32 FMA, add and subtract); the row sum in four
+        // independent packed partial sums
+        const float2 sl2 = make_float2(sl, sl), nmu2 = make_float2(-mu, -mu);
+        float2 ls[4] = {};
 #pragma unroll
         for (int c = 0; c < kKeys / 32; ++c) {
             uint32_t hi[16], lo[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const float a = exp2f(fmaf(sv[32 * c + 2 * e], sl, -mu));
-                const float d = exp2f(fmaf(sv[32 * c + 2 * e + 1], sl, -mu));
-                l += a + d;
-                hi[e] = Storage<T>::from_float2(a, d);
-                const float2 back = Storage<T>::to_float2(hi[e]);
-                lo[e] = Storage<T>::from_float2(a - back.x, d - back.y);
+                const float2 x =
+                    ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), sl2, nmu2);
+                const float2 w = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                ls[e & 3] = fadd2(ls[e & 3], w);
+                hi[e] = Storage<T>::from_float2(w.x, w.y);
+                const float2 rem = fsub2(w, Storage<T>::to_float2(hi[e]));
+                lo[e] = Storage<T>::from_float2(rem.x, rem.y);
             }
             tc::st16(trow + 16 * c, hi);  // over S, already read
             tc::st16(trow + kColPl + 16 * c, lo);
         }
+        ls[0] = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+        l += ls[0].x + ls[0].y;
         // keys past the context in the last tile: zero their V rows (NaN
         // bit patterns there must not meet their zero weights)
         const int key0 = j * kKeys;
