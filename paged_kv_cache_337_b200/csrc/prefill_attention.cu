@@ -94,51 +94,73 @@ struct Bars {
     uint64_t* q_ready;   // the Q tiles are staged (every staging warp arrived)
 };
 
-// Producer: lane 0 of warp 0.  A box past the context still loads a block
-// (the last one) so that every stage receives its full byte count; those
-// rows are masked (K) or zeroed (V) downstream.
+// Producer: warp 0.  A box past the context still loads a block (the last
+// one) so that every stage receives its full byte count; those rows are
+// masked (K) or zeroed (V) downstream.  The block ids come from the Block
+// Table one warp-wide load per eight key tiles (lane i: the id of box i of
+// the window), handed to lane 0, which issues the TMA loads, by shuffles.
 __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const PrefillParams& p,
                         int s, int kvh, int L, int ntiles, uint8_t* stages, const Bars& b,
-                        bool* failed) {
+                        int lane, bool* failed) {
+    constexpr int kBoxes = kKeys / kBoxKeys;       // TMA boxes per key tile and 64-dim half
+    constexpr int kWindowTiles = 32 / kBoxes;      // key tiles per warp-wide block-id load
     const int bs = p.block_size;
     const int32_t* row = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
     const int last_block = L > 0 ? (L - 1) / bs : 0;
+    int phys_lane = 0;
     int issued = 0;
     for (int j = 0; j < ntiles; ++j) {
+        if (j % kWindowTiles == 0) {
+            const int box = j * kBoxes + lane;  // box of this lane in the window
+            phys_lane = __ldg(row + min(box * kBoxKeys / bs, last_block));
+            if (box < ntiles * kBoxes && (phys_lane < 0 || phys_lane >= p.num_blocks))
+                report_error(p.dev_error, PKV_DEVERR_BLOCK_ID, s);
+        }
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait_bounded(&b.kv_empty[st], ((j / kStages) - 1) & 1)) {
+        if (j >= kStages &&
+            !__all_sync(0xffffffffu,
+                        mbar_wait_bounded(&b.kv_empty[st], ((j / kStages) - 1) & 1))) {
             *failed = true;
             break;
         }
-        uint8_t* kdst = stages + st * kStageBytes;
-        uint8_t* vdst = kdst + kTileBytes;
-        mbar_arrive_expect_tx(&b.kv_full[st], kStageBytes);
-#pragma unroll 1
-        for (int bx = 0; bx < kKeys / kBoxKeys; ++bx) {
-            const int key0 = j * kKeys + bx * kBoxKeys;
-            const int lb = min(key0 / bs, last_block);
-            const int off = key0 < L ? key0 % bs : 0;
-            const int32_t phys = __ldg(row + lb);
-            if (phys < 0 || phys >= p.num_blocks) report_error(p.dev_error, PKV_DEVERR_BLOCK_ID, s);
+        int phys[kBoxes];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap, &b.kv_full[st], 0,
-                            kvh, off, h, phys);
-                tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap, &b.kv_full[st], 0,
-                            kvh, off, h, phys);
+        for (int bx = 0; bx < kBoxes; ++bx)
+            phys[bx] = __shfl_sync(0xffffffffu, phys_lane, (j % kWindowTiles) * kBoxes + bx);
+        if (lane == 0) {
+            uint8_t* kdst = stages + st * kStageBytes;
+            uint8_t* vdst = kdst + kTileBytes;
+            mbar_arrive_expect_tx(&b.kv_full[st], kStageBytes);
+#pragma unroll
+            for (int bx = 0; bx < kBoxes; ++bx) {
+                const int key0 = j * kKeys + bx * kBoxKeys;
+                const int off = key0 < L ? key0 % bs : 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap,
+                                &b.kv_full[st], 0, kvh, off, h, phys[bx]);
+                    tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap,
+                                &b.kv_full[st], 0, kvh, off, h, phys[bx]);
+                }
             }
         }
+        __syncwarp();
         ++issued;
     }
     // before leaving, every issued load has landed (bounded)
-    for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait_bounded(&b.kv_full[j % kStages], (j / kStages) & 1);
+    if (lane == 0)
+        for (int j = max(0, issued - kStages); j < issued; ++j)
+            mbar_wait_bounded(&b.kv_full[j % kStages], (j / kStages) & 1);
 }
 
-// MMA issuer: lane 0 of warp 1.
+// MMA issuer: warp 1, in step; one elected lane issues each MMA and commit,
+// the descriptors stay warp-uniform.
 template <bool BF16>
 __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t* stages,
                            int ntiles, bool* failed) {
+    // one lane issues every MMA and every commit (a commit tracks the MMAs
+    // of the thread that executes it)
+    const bool leader = tc::elect_one();
     constexpr uint32_t kIdS = tc::f16_idesc(BF16, false, kRows, kKeys);  // K: K-major B
     constexpr uint32_t kIdPV = tc::f16_idesc(BF16, true, kRows, kD);     // V: MN-major B
     // S = Q K^T of Q tile t for key tile j: 8 steps of 16 dims (4 per
@@ -151,10 +173,11 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
             const uint32_t off = (uint32_t)t * kQTileBytes + (uint32_t)(kk >> 2) * kQHalfBytes +
                                  (uint32_t)(kk & 3) * 32;
             const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
-            tc::mma_ss(tmem + kTileCols * t, tc::sw128_desc(qaddr + off, 16, 1024),
-                       tc::sw128_desc(kaddr + koff, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+            const uint64_t qd = tc::sw128_desc(qaddr + off, 16, 1024);
+            const uint64_t kd = tc::sw128_desc(kaddr + koff, 16, 1024);
+            if (leader) tc::mma_ss(tmem + kTileCols * t, qd, kd, kIdS, kk > 0 ? 1u : 0u);
         }
-        tc::commit(smem_addr(&b.s_full[t]));
+        if (leader) tc::commit(smem_addr(&b.s_full[t]));
     };
     // O += P V of Q tile t for key tile j: 8 steps of 16 keys; V's 8-key
     // groups 1 KiB apart (SBO), its 64-dim halves 16 KiB apart (LBO)
@@ -164,16 +187,18 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
             const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
-            tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-            tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
+            if (leader) {
+                tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
+            }
         }
-        tc::commit(smem_addr(&b.o_done[t]));
+        if (leader) tc::commit(smem_addr(&b.o_done[t]));
     };
     // Ping-pong: while one tile's softmax runs, the tensor cores run the
     // other tile's P V and its next S.
     //   S_A(0) S_B(0) | P_A(j): PV_A(j) S_A(j+1) | P_B(j): PV_B(j) S_B(j+1)
-    if (!mbar_wait_bounded(&b.kv_full[0], 0)) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[0], 0))) {
         *failed = true;
     } else {
         tc::fence_after_sync();
@@ -184,14 +209,15 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
         const int st = j % kStages;
         const bool more = j + 1 < ntiles;
         // tile A
-        if (!mbar_wait_bounded(&b.p_full[0], j & 1)) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[0], j & 1))) {
             *failed = true;
             break;
         }
         tc::fence_after_sync();
         issue_pv(0, j);
         if (more) {
-            if (!mbar_wait_bounded(&b.kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1)) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[(j + 1) % kStages],
+                                                           ((j + 1) / kStages) & 1))) {
                 *failed = true;
                 break;
             }
@@ -199,17 +225,17 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
             issue_s(0, j + 1);
         }
         // tile B
-        if (!mbar_wait_bounded(&b.p_full[1], j & 1)) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[1], j & 1))) {
             *failed = true;
             break;
         }
         tc::fence_after_sync();
         issue_pv(1, j);
-        tc::commit(smem_addr(&b.kv_empty[st]));  // both tiles' P V of this stage
+        if (leader) tc::commit(smem_addr(&b.kv_empty[st]));  // both tiles' P V of this stage
         if (more) issue_s(1, j + 1);
     }
     // every MMA issued has completed before the tensor memory is freed
-    tc::commit(smem_addr(b.drain));
+    if (leader) tc::commit(smem_addr(b.drain));
     mbar_wait_bounded(b.drain, 0);
 }
 
@@ -422,7 +448,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     bool failed = false;
     if (warp == kProducerWarp) {
         // K/V do not depend on Q: stream them while the other warps stage it
-        if (lane == 0) produce(kmap, vmap, p, s, kvh, L, ntiles, stages, b, &failed);
+        produce(kmap, vmap, p, s, kvh, L, ntiles, stages, b, lane, &failed);
     } else {
         // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA
         // reads them, staged by every warp but the producer
@@ -445,14 +471,12 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         __syncwarp();
         if (lane == 0) mbar_arrive_one(b.q_ready);
         if (warp == kMmaWarp) {
-            if (lane == 0) {
-                if (!mbar_wait_bounded(b.q_ready, 0)) {
-                    failed = true;
-                } else {
-                    tc::fence_after_sync();
-                    issue_mmas<std::is_same<T, __nv_bfloat16>::value>(b, tmem, smem_addr(qsm),
-                                                                      stages, ntiles, &failed);
-                }
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(b.q_ready, 0))) {
+                failed = true;
+            } else {
+                tc::fence_after_sync();
+                issue_mmas<std::is_same<T, __nv_bfloat16>::value>(b, tmem, smem_addr(qsm), stages,
+                                                                  ntiles, &failed);
             }
         } else {
             softmax_rows<T>(p, b, tmem, stages, L, n, q0, kvh, r0, nrows, ntiles, warp, lane,
