@@ -48,10 +48,11 @@ constexpr int kQBytes = kQTiles * kQTileBytes;
 constexpr int kBoxKeys = 16;                        // slots per TMA box
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4 * kQTiles;
 constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;
-// tensor-memory columns per Q tile t: S (64 columns; P high | P low, 32
-// each, written over it once S is read) at 256 t, O at 256 t + 128
+// tensor-memory columns per Q tile t: two S buffers (64 columns each; P
+// high | P low, 32 each, written over S once it is read) at 256 t and
+// 256 t + 64, O at 256 t + 128; key tile j uses S buffer j % 2
 constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = kKeys / 2, kTmemCols = 512;
-constexpr int kNumBars = 2 * kStages + 3 * kQTiles + 2;  // kv_full/empty, s_full/p_full/o_done per tile, drain, q_ready
+constexpr int kNumBars = 2 * kStages + 5 * kQTiles + 2;  // kv_full/empty, s_full/p_full per (tile, buffer), o_done per tile, drain, q_ready
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the max grows by more than 2^8
@@ -87,8 +88,8 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
 struct Bars {
     uint64_t* kv_full;   // [kStages]: TMA bytes landed
     uint64_t* kv_empty;  // [kStages]: the P V MMAs reading the stage completed
-    uint64_t* s_full;    // [kQTiles]: S in tensor memory
-    uint64_t* p_full;    // [kQTiles]: P written (and O rescaled) by the softmax warps
+    uint64_t* s_full;    // [kQTiles][2]: S of the buffer in tensor memory
+    uint64_t* p_full;    // [kQTiles][2]: P of the buffer written (and O rescaled)
     uint64_t* o_done;    // [kQTiles]: the P V MMAs of the tile completed
     uint64_t* drain;     // every MMA issued completed (exit)
     uint64_t* q_ready;   // the Q tiles are staged (every staging warp arrived)
@@ -163,76 +164,85 @@ __device__ void issue_mmas(const Bars& b, uint32_t tmem, uint32_t qaddr, uint8_t
     const bool leader = tc::elect_one();
     constexpr uint32_t kIdS = tc::f16_idesc(BF16, false, kRows, kKeys);  // K: K-major B
     constexpr uint32_t kIdPV = tc::f16_idesc(BF16, true, kRows, kD);     // V: MN-major B
-    // S = Q K^T of Q tile t for key tile j: 8 steps of 16 dims (4 per
-    // 128-byte swizzle atom).  In issue order it follows P V of tile t for
-    // key tile j - 1, which reads the P written over S.
+    // S = Q K^T of Q tile t for key tile j into S buffer j % 2: 8 steps of
+    // 16 dims (4 per 128-byte swizzle atom).  In issue order it follows P V
+    // of tile t for key tile j - 2, which reads the P written over that
+    // buffer.
+    // descriptor bases; a step's byte offset enters the start-address
+    // field (16-byte units, no carry: shared addresses stay below 256 KiB)
+    const uint64_t qd0 = tc::sw128_desc(qaddr, 16, 1024);
+    const uint64_t sd0 = tc::sw128_desc(smem_addr(stages), 16, 1024);
+    const uint64_t vd0 = tc::sw128_desc(smem_addr(stages) + kTileBytes, kHalfBytes, 1024);
     auto issue_s = [&](int t, int j) {
-        const uint32_t kaddr = smem_addr(stages + (j % kStages) * kStageBytes);
+        const uint64_t kd = sd0 + (uint64_t)(((j % kStages) * kStageBytes) >> 4);
+        const uint64_t qd = qd0 + (uint64_t)((t * kQTileBytes) >> 4);
+        const uint32_t dst = tmem + kTileCols * t + kKeys * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (uint32_t)t * kQTileBytes + (uint32_t)(kk >> 2) * kQHalfBytes +
-                                 (uint32_t)(kk & 3) * 32;
-            const uint32_t koff = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
-            const uint64_t qd = tc::sw128_desc(qaddr + off, 16, 1024);
-            const uint64_t kd = tc::sw128_desc(kaddr + koff, 16, 1024);
-            if (leader) tc::mma_ss(tmem + kTileCols * t, qd, kd, kIdS, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * kQHalfBytes + (kk & 3) * 32) >> 4;
+            const uint32_t koff = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            if (leader) tc::mma_ss(dst, qd + off, kd + koff, kIdS, kk > 0 ? 1u : 0u);
         }
-        if (leader) tc::commit(smem_addr(&b.s_full[t]));
+        if (leader) tc::commit(smem_addr(&b.s_full[2 * t + (j & 1)]));
     };
     // O += P V of Q tile t for key tile j: 8 steps of 16 keys; V's 8-key
     // groups 1 KiB apart (SBO), its 64-dim halves 16 KiB apart (LBO)
     auto issue_pv = [&](int t, int j) {
-        const uint32_t vaddr = smem_addr(stages + (j % kStages) * kStageBytes) + kTileBytes;
-        const uint32_t cs = kTileCols * t;
+        const uint64_t vd = vd0 + (uint64_t)(((j % kStages) * kStageBytes) >> 4);
+        const uint32_t cs = kTileCols * t, cp = cs + kKeys * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint64_t vd = tc::sw128_desc(vaddr + (uint32_t)kk * 2048, kHalfBytes, 1024);
             if (leader) {
-                tc::mma_ts(tmem + cs + kColO, tmem + cs + kk * 8, vd, kIdPV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_ts(tmem + cs + kColO, tmem + cs + kColPl + kk * 8, vd, kIdPV, 1u);
+                tc::mma_ts(tmem + cs + kColO, tmem + cp + kk * 8, vd + kk * (2048 >> 4),
+                               kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_ts(tmem + cs + kColO, tmem + cp + kColPl + kk * 8,
+                               vd + kk * (2048 >> 4), kIdPV, 1u);
             }
         }
         if (leader) tc::commit(smem_addr(&b.o_done[t]));
     };
-    // Ping-pong: while one tile's softmax runs, the tensor cores run the
-    // other tile's P V and its next S.
-    //   S_A(0) S_B(0) | P_A(j): PV_A(j) S_A(j+1) | P_B(j): PV_B(j) S_B(j+1)
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[0], 0))) {
-        *failed = true;
-    } else {
+    // S runs two key tiles ahead of P V, so that a tile's softmax finds its
+    // next S ready, and the tensor cores take one tile's P V and S while the
+    // other tile's softmax runs:
+    //   S_A(0) S_B(0) S_A(1) S_B(1) | P_A(j): PV_A(j) S_A(j+2) | P_B(j): PV_B(j) S_B(j+2)
+    for (int j = 0; j < min(ntiles, 2) && !*failed; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[j], 0))) {
+            *failed = true;
+            break;
+        }
         tc::fence_after_sync();
-        issue_s(0, 0);
-        issue_s(1, 0);
+        issue_s(0, j);
+        issue_s(1, j);
     }
     for (int j = 0; j < ntiles && !*failed; ++j) {
-        const int st = j % kStages;
-        const bool more = j + 1 < ntiles;
+        const int st = j % kStages, buf = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const bool more = j + 2 < ntiles;
         // tile A
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[0], j & 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[buf], ph))) {
             *failed = true;
             break;
         }
         tc::fence_after_sync();
         issue_pv(0, j);
         if (more) {
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[(j + 1) % kStages],
-                                                           ((j + 1) / kStages) & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.kv_full[(j + 2) % kStages],
+                                                           ((j + 2) / kStages) & 1))) {
                 *failed = true;
                 break;
             }
             tc::fence_after_sync();
-            issue_s(0, j + 1);
+            issue_s(0, j + 2);
         }
         // tile B
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[1], j & 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&b.p_full[2 + buf], ph))) {
             *failed = true;
             break;
         }
         tc::fence_after_sync();
         issue_pv(1, j);
         if (leader) tc::commit(smem_addr(&b.kv_empty[st]));  // both tiles' P V of this stage
-        if (more) issue_s(1, j + 1);
+        if (more) issue_s(1, j + 2);
     }
     // every MMA issued has completed before the tensor memory is freed
     if (leader) tc::commit(smem_addr(b.drain));
@@ -261,14 +271,16 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
     float m = -INFINITY, l = 0.f;
     int j = 0;
     for (; j < ntiles; ++j) {
-        if (!warp_wait(&b.s_full[t], j & 1)) break;
+        const int buf = j & 1;
+        const uint32_t srow = trow + kKeys * buf;  // this key tile's S buffer
+        if (!warp_wait(&b.s_full[2 * t + buf], (j >> 1) & 1)) break;
         tc::fence_after_sync();
         // raw scores; the scale (positive) is applied with the max subtraction
         float sv[kKeys];
         {
             uint32_t u[kKeys / 32][32];
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) tc::ld32(trow + 32 * c, u[c]);
+            for (int c = 0; c < kKeys / 32; ++c) tc::ld32(srow + 32 * c, u[c]);
             tc::wait_ld();
             const int key0 = j * kKeys;
             // the causal mask only where some row of the warp stops inside
@@ -294,11 +306,13 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         if (resc) m = mt;
         l *= alpha;
         const float mu = m == -INFINITY ? 0.f : m;
-        // the P V of the previous tile must be done before P and O change
-        if (j > 0) {
+        // O changes only after the P V of the previous key tile is done
+        // (S of this tile was issued after the P V of tile j - 2, so at
+        // most that one P V is outstanding)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
             if (!warp_wait(&b.o_done[t], (j - 1) & 1)) break;
             tc::fence_after_sync();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            {
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -328,8 +342,8 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                 const float2 rem = fsub2(w, Storage<T>::to_float2(hi[e]));
                 lo[e] = Storage<T>::from_float2(rem.x, rem.y);
             }
-            tc::st16(trow + 16 * c, hi);  // over S, already read
-            tc::st16(trow + kColPl + 16 * c, lo);
+            tc::st16(srow + 16 * c, hi);  // over S, already read
+            tc::st16(srow + kColPl + 16 * c, lo);
         }
         ls[0] = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
         l += ls[0].x + ls[0].y;
@@ -352,9 +366,11 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         tc::wait_st();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive_one(&b.p_full[t]);
+        if (lane == 0) mbar_arrive_one(&b.p_full[2 * t + buf]);
     }
-    if (j < ntiles || !warp_wait(&b.o_done[t], (ntiles - 1) & 1)) {
+    // the last two P V (phases ntiles - 2 and ntiles - 1 of o_done), in order
+    if (j < ntiles || (ntiles >= 2 && !warp_wait(&b.o_done[t], (ntiles - 2) & 1)) ||
+        !warp_wait(&b.o_done[t], (ntiles - 1) & 1)) {
         *failed = true;
         return;
     }
@@ -393,9 +409,9 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     uint8_t* stages = smem + kQBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
-    Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + kQTiles,
-           bars + 2 * kStages + 2 * kQTiles, bars + 2 * kStages + 3 * kQTiles,
-           bars + 2 * kStages + 3 * kQTiles + 1};
+    Bars b{bars, bars + kStages, bars + 2 * kStages, bars + 2 * kStages + 2 * kQTiles,
+           bars + 2 * kStages + 4 * kQTiles, bars + 2 * kStages + 5 * kQTiles,
+           bars + 2 * kStages + 5 * kQTiles + 1};
 
     // flat grid: the heaviest row tile of every (sequence, KV head) first
     const int pairs = p.num_seqs * p.num_kv_heads;
@@ -430,8 +446,10 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&b.kv_empty[i], 1);
         }
         for (int t = 0; t < kQTiles; ++t) {
-            mbar_init(&b.s_full[t], 1);
-            mbar_init(&b.p_full[t], 4);  // the tile's four softmax warps
+            for (int u = 0; u < 2; ++u) {
+                mbar_init(&b.s_full[2 * t + u], 1);
+                mbar_init(&b.p_full[2 * t + u], 4);  // the tile's four softmax warps
+            }
             mbar_init(&b.o_done[t], 1);
         }
         mbar_init(b.drain, 1);
