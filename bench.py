@@ -41,12 +41,20 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "paged decode attention effective KV GB/s (% of HBM peak); decode tok/s"
-# the committed ncu summaries that give a decode workload's DRAM bytes per
-# launch, by workload name; other workloads report traffic null
+# the committed ncu summaries that give a workload's DRAM bytes per launch of
+# its dominant kernel, by workload name; other workloads report traffic null
 PROFILE_TRAFFIC = {
     "7b_s256_h32_d128_bs16_bf16": os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md"),
     "7b_s256_h32_d128_bs16_bf16_kv_e4m3": os.path.join(ROOT, "profiles",
                                                         "decode_attention_fp8_7b_s256.md"),
+    "prefill_s8_l2048_hq32_hkv8_d128_bs16_bf16": os.path.join(ROOT, "profiles",
+                                                               "prefill_attention_s8_l2048.md"),
+}
+# the sources whose digest a summary records: the kernel's file and the
+# headers it includes
+KERNEL_SOURCES = {
+    "decode": ("decode_attention.cu", "common.cuh"),
+    "prefill": ("prefill_attention.cu", "common.cuh", "packed_f32.cuh", "tcgen05.cuh"),
 }
 
 
@@ -217,8 +225,8 @@ def measured_peak():
 
 
 def profiled_traffic(source_digest, workload):
-    """DRAM bytes per launch of the decode kernel from the committed ncu
-    summary of this workload, or None when there is none or it was taken on
+    """DRAM bytes per launch of the workload's dominant kernel from its
+    committed ncu summary, or None when there is none or it was taken on
     other kernel source."""
     try:
         with open(PROFILE_TRAFFIC[workload]) as f:
@@ -239,11 +247,11 @@ def profiled_traffic(source_digest, workload):
         return None
 
 
-def kernel_source_digest():
+def kernel_source_digest(kernel="decode"):
     import hashlib
 
     h = hashlib.sha256()
-    for name in ("decode_attention.cu", "common.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "paged_kv_cache_337_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -951,7 +959,9 @@ def run_prefill(args, world, rank, local):
                            2 * T * Hkv * D * 2 / 1e9, T * Hq * D * 2 / 1e9)},
             "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
                          "peak": peak[0], "unit": "TFLOP/s",
-                         "frac": round(attn_tflops / peak[0], 4), "traffic": None,
+                         "frac": round(attn_tflops / peak[0], 4),
+                         "traffic": profiled_traffic(kernel_source_digest("prefill"),
+                                                     PREFILL_WORKLOAD),
                          "kernel": "paged_prefill_kernel", "peak_source": peak[1]},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "clocks": clock_info,
         }

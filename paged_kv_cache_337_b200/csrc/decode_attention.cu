@@ -564,11 +564,14 @@ template <int D, bool FP8, bool MMA>
 struct Plan {
     static_assert(!FP8 || D == 128, "e4m3 caches are built for head_dim 128");
     static_assert(!FP8 || MMA, "e4m3 caches run on the tensor-core path");
-    static constexpr int kStages = FP8 ? 3 : Geom<D>::kStages;
+    static constexpr int kStages = FP8 ? 2 : Geom<D>::kStages;
     static constexpr int kTileBytes = FP8 ? kTile * D : Geom<D>::kKBytes;  // K (or V) as stored
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr size_t kRing = (size_t)kWarps * kStages * kStageBytes;
-    static constexpr size_t kEpilogue = kRing;
+    // the warps' merge reuses the ring: per warp m and l of up to 16 (padded)
+    // heads, the common max, and per warp G x D partial outputs (G <= 16)
+    static constexpr size_t kMerge = ((size_t)kWarps * 2 * 16 + 16 + (size_t)kWarps * 16 * D) * 4;
+    static constexpr size_t kEpilogue = kRing > kMerge ? kRing : kMerge;
     static constexpr size_t kBarOff = kEpilogue;
     static constexpr size_t kScaleOff = kBarOff + (size_t)kWarps * kStages * 8;
     static constexpr size_t kTableOff = kScaleOff + (FP8 ? (size_t)kWarps * kStages * 32 : 0);
