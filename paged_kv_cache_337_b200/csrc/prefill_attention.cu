@@ -85,6 +85,19 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// 16-byte copy global -> shared that does not wait (cp.async, L2 only);
+// when copy is false, the destination is zero-filled and nothing is read
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src, bool copy) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
+                 "l"(src), "r"(copy ? 16 : 0)
+                 : "memory");
+}
+
+// waits for every cp.async this thread issued
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 struct Bars {
     uint64_t* kv_full;   // [kStages]: TMA bytes landed
     uint64_t* kv_empty;  // [kStages]: the P V MMAs reading the stage completed
@@ -469,22 +482,22 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         produce(kmap, vmap, p, s, kvh, L, ntiles, stages, b, lane, &failed);
     } else {
         // Q rows (token r / G, head kvh * G + r % G), swizzled as the MMA
-        // reads them, staged by every warp but the producer
+        // reads them, staged by every warp but the producer: each thread
+        // issues all its 16-byte copies (zero-filled past the sequence's
+        // rows) before waiting, so the CTA pays one memory latency
         const int Hq = p.num_q_heads;
+        const T* qbase = static_cast<const T*>(p.query);
         for (int c = threadIdx.x - 32; c < kQTiles * kRows * (kD / 8); c += kThreads - 32) {
             const int r = c >> 4, ch = c & 15;  // r: row of the CTA's 256
             const int row = r0 + r;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (row < nrows) {
-                const int tok = row / G, g = row - tok * G;
-                v = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.query) +
-                                                    ((int64_t)(q0 + tok) * Hq + kvh * G + g) *
-                                                        kD +
-                                                    ch * 8);
-            }
-            *reinterpret_cast<uint4*>(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
-                                      swz(r % kRows, ch)) = v;
+            const bool in = row < nrows;
+            const int tok = in ? row / G : 0, g = in ? row - tok * G : 0;
+            const T* src = qbase + ((int64_t)(q0 + tok) * Hq + kvh * G + g) * kD + ch * 8;
+            cp_async_16(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
+                            swz(r % kRows, ch),
+                        src, in);
         }
+        cp_async_wait_all();
         tc::fence_proxy_async_smem();  // the tensor cores read Q through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive_one(b.q_ready);
