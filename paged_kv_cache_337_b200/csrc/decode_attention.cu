@@ -75,7 +75,6 @@ template <int D>
 struct Geom {
     static constexpr int kBoxes = D / kBoxD;             // boxes per K (or V) tile
     static constexpr int kKBytes = kBoxes * kSubTileBytes;
-    static constexpr int kStageBytes = 2 * kKBytes;      // K + V of one tile
     static constexpr int kStages = D == 128 ? PKV_DECODE_STAGES_D128 : PKV_DECODE_STAGES_D64;
 };
 
@@ -581,10 +580,10 @@ struct Plan {
 // ---------------------------------------------------------------------------
 // The attention kernel (single pass or one partition of split-K)
 // ---------------------------------------------------------------------------
+// The body of one CTA; the kernels below differ only in their launch bounds.
 template <typename T, int D, typename Warp, bool FP8>
-__global__ void __launch_bounds__(kWarps * 32)
-paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
-                    const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+__device__ __forceinline__ void decode_cta(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                           const DecodeParams& p) {
     using Gm = Geom<D>;
     using Pl = Plan<D, FP8, Warp::kMma>;
     constexpr int STAGES = Pl::kStages;
@@ -858,6 +857,23 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
     if (threadIdx.x == 0) *count = 0;  // ready for the next launch
 }
 
+template <typename T, int D, typename Warp, bool FP8>
+__global__ void __launch_bounds__(kWarps * 32)
+paged_decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+    decode_cta<T, D, Warp, FP8>(kmap, vmap, p);
+}
+
+// e4m3 caches with up to 8 query heads per KV head: registers capped so
+// that 5 CTAs fit per SM (35 KB of shared memory each), which hides more of
+// the conversion and fragment-load latency this path is bound by.
+template <typename T, typename Warp>
+__global__ void __launch_bounds__(kWarps * 32, 5)
+paged_decode_kernel_e4m3(const __grid_constant__ CUtensorMap kmap,
+                         const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+    decode_cta<T, 128, Warp, true>(kmap, vmap, p);
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -952,7 +968,11 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
                     "pkv_decode_attention: %d partitions of %d query heads are too many to "
                     "merge in one CTA; use a larger partition_size",
                     p.num_partitions, p.group);
-    auto kern = paged_decode_kernel<T, D, Warp, FP8>;
+    void (*kern)(CUtensorMap, CUtensorMap, DecodeParams) = nullptr;
+    if constexpr (FP8 && Warp::GP <= 8)
+        kern = paged_decode_kernel_e4m3<T, Warp>;
+    else
+        kern = paged_decode_kernel<T, D, Warp, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess)
