@@ -216,7 +216,8 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
  *   block_tables     device int32 [num_seqs, max_blocks_per_seq]
  *   context_lens     device int32 [num_seqs]: L, the chunk's tokens included
  *   query_start      device int32 [num_seqs + 1], non-decreasing from 0
- *   max_query_len    host bound on every n_s: it sizes the grid
+ *   max_query_len    host bound on every n_s: it sizes the list of 256-row
+ *                    tiles that the kernel's persistent CTAs (one per SM) walk
  *   scale            > 0 (PKV_ERR_INVALID otherwise)
  * A sequence with n_s > L, n_s > max_query_len or L > max_blocks_per_seq *
  * block_size is reported (PKV_DEVERR_CONTEXT_LEN) and its rows are left
