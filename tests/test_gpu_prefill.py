@@ -130,3 +130,58 @@ def test_prompt_write_then_prefill_through_the_pool(cuda_device):
     got_v = ref.bits(cache.value_cache.cpu()).reshape(nb * bs, Hkv, D)[slots]
     assert np.array_equal(got_k, wk.reshape(nb * bs, Hkv, D)[slots])
     assert np.array_equal(got_v, wv.reshape(nb * bs, Hkv, D)[slots])
+
+
+def row_tiles(chunks, group):
+    """The kernel's work items: 256-row tiles x sequences x KV heads."""
+    return -(-max(chunks) * group // 256)
+
+
+@pytest.mark.parametrize("kind", ["whole", "chunked"])
+def test_prefill_many_row_tiles_per_cta(kind, cuda_device):
+    """More 256-row tiles than SMs, of uneven weight, with the tiles past
+    short sequences' rows skipped: each persistent CTA walks several items,
+    so its ring stages, S buffers and barrier phases carry across items."""
+    lens = [600, 3, 450, 257, 64, 1, 520, 333, 130, 47, 40, 300]
+    chunks = lens if kind == "whole" else [600, 3, 100, 257, 17, 1, 520, 64, 130, 47, 1, 299]
+    Hq, Hkv = 32, 8
+    items = row_tiles(chunks, Hq // Hkv) * len(lens) * Hkv
+    assert items > 2 * torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    p, q, qs = case(31 if kind == "whole" else 32, Hq, Hkv, 16, lens, chunks, "bf16")
+    scale = 1.0 / np.sqrt(128)
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    got = run_prefill(p, q, qs, scale, cuda_device, err)
+    want = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                 Hkv, 16)
+    assert err.tolist() == [0, 0]
+    assert torch.isfinite(got).all()
+    assert tolerance_violation(got, want, ATOL, RTOL) <= 0
+
+
+def test_prefill_full_size_sampled_rows(cuda_device):
+    """The benchmark's launch: 8 prompts of 2048 tokens, 32 query / 8 KV
+    heads, block size 16, bf16: 2048 row tiles, about 14 per persistent CTA.
+    Checked on sampled rows: row p of a prompt is attention over its tokens
+    0 .. p, which the oracle computes as a one-row sequence of context p + 1."""
+    S, L, Hq, Hkv, D, bs = 8, 2048, 32, 8, 128, 16
+    p = paged_problem(77, Hq, Hkv, D, bs, [L] * S, "bf16")
+    g = torch.Generator().manual_seed(78)
+    q = torch.randn(S * L, Hq, D, generator=g).to(torch.bfloat16)
+    qs = np.arange(0, S * L + 1, L, dtype=np.int32)
+    scale = 1.0 / np.sqrt(D)
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    got = run_prefill(p, q, qs, scale, cuda_device, err)
+    assert err.tolist() == [0, 0]
+    assert torch.isfinite(got).all()
+    rng = np.random.default_rng(79)
+    edges = [0, 1, 15, 16, 63, 64, 255, 256, 1023, 1024, 2046, 2047]
+    seqs, pos = [], []
+    for s in range(S):
+        for t in edges + list(rng.integers(0, L, 4)):
+            seqs.append(s)
+            pos.append(int(t))
+    rows = np.asarray(seqs) * L + np.asarray(pos)
+    want = ref.prefill_attention(q[rows], p["kc"], p["vc"], p["tables"][seqs],
+                                 np.asarray(pos, np.int32) + 1,
+                                 np.arange(len(rows) + 1, dtype=np.int32), scale, "bf16", Hkv, bs)
+    assert tolerance_violation(got[rows], want, ATOL, RTOL) <= 0
