@@ -277,8 +277,9 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
             if (leader) {
                 tc::mma_ts(tmem + cs + kColO, tmem + cp + kk * 8, vd + kk * (2048 >> 4), kIdPV,
                            (!first || kk > 0) ? 1u : 0u);
-                tc::mma_ts(tmem + cs + kColO, tmem + cp + kColPl + kk * 8,
-                           vd + kk * (2048 >> 4), kIdPV, 1u);
+                if constexpr (BF16)  // the remainder of a bf16 P
+                    tc::mma_ts(tmem + cs + kColO, tmem + cp + kColPl + kk * 8,
+                               vd + kk * (2048 >> 4), kIdPV, 1u);
             }
         }
         if (leader) tc::commit(smem_addr(&b.o_done[t]));
@@ -474,9 +475,12 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                     tc::st32(trow + kColO + 32 * c, o);
                 }
             }
-            // P = 2^(s - m) as a 16-bit high part and the 16-bit remainder, on
-            // key pairs (packed fp32 FMA, add and subtract); the row sum in
-            // four independent packed partial sums
+            // P = 2^(s - m) on key pairs (packed fp32 FMA, add and subtract);
+            // the row sum in four independent packed partial sums.  A bf16 P
+            // is written as a 16-bit high part and the 16-bit remainder (two
+            // MMAs): one bf16 value carries up to 2^-9 relative error per
+            // weight.  An f16 P (2^-11, P <= 2^8, row sum >= 1) is one part.
+            constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
             const float2 sl2 = make_float2(sl, sl), nmu2 = make_float2(-mu, -mu);
             float2 ls[4] = {};
 #pragma unroll
@@ -489,11 +493,13 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                     const float2 w = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     ls[e & 3] = fadd2(ls[e & 3], w);
                     hi[e] = Storage<T>::from_float2(w.x, w.y);
-                    const float2 rem = fsub2(w, Storage<T>::to_float2(hi[e]));
-                    lo[e] = Storage<T>::from_float2(rem.x, rem.y);
+                    if constexpr (kSplit) {
+                        const float2 rem = fsub2(w, Storage<T>::to_float2(hi[e]));
+                        lo[e] = Storage<T>::from_float2(rem.x, rem.y);
+                    }
                 }
                 tc::st16(srow + 16 * c, hi);  // over S, already read
-                tc::st16(srow + kColPl + 16 * c, lo);
+                if constexpr (kSplit) tc::st16(srow + kColPl + 16 * c, lo);
             }
             ls[0] = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
             l += ls[0].x + ls[0].y;
