@@ -71,8 +71,15 @@ def parse_args():
                     help="profiling only: run the workload's first N sequences")
     ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
                     help="fp8: e4m3 cache with a scale per (block, KV head)")
+    ap.add_argument("--work-list", choices=["longest_first", "grid", "none"],
+                    default="longest_first",
+                    help="decode over the library's work list (items longest first, or in "
+                         "grid order) or over the full grid (none)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", choices=["all", "none"], default="all",
+                    help="with the default workload: also measure the other decode "
+                         "workloads, e4m3 caches, the shared prefix and prefill")
     return ap.parse_args()
 
 
@@ -165,55 +172,123 @@ def copy_bytes(spec, num_pairs, fp8=False):
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
+# A child process polls NVML (read-only queries) every millisecond and
+# stamps each sample with CLOCK_MONOTONIC, which the parent shares, so the
+# samples taken while the timed region ran can be picked out afterwards.
+# It runs apart from the benchmark's interpreter so that the GIL never
+# delays a sample or a launch.
+_NVML_SAMPLER = r"""
+import signal, sys, time
+import pynvml
+pynvml.nvmlInit()
+path, dt, keys = sys.argv[1], float(sys.argv[2]), sys.argv[3:]
+h = None
+for key in keys:  # the device's UUID first, then its NVML index
+    try:
+        if key.startswith(("GPU-", "MIG-")):
+            h = pynvml.nvmlDeviceGetHandleByUUID(key)
+        else:
+            h = pynvml.nvmlDeviceGetHandleByIndex(int(key))
+        break
+    except pynvml.NVMLError:
+        pass
+if h is None:
+    sys.exit(1)
+stop = []
+signal.signal(signal.SIGTERM, lambda *a: stop.append(1))
+with open(path, "w") as f:
+    f.write("max %d\n" % pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+    f.flush()
+    while not stop:
+        t = time.monotonic()
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        why = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        f.write("%.6f %d %d\n" % (t, sm, why))
+        time.sleep(dt)
+"""
+# NVML clock-event reason bits, by the names the clocks record uses
+_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled during a timed region.
+
+    start() launches the sampler, mark() brackets each timed region with
+    host monotonic times (taken just before the first launch and just after
+    the closing synchronize, so the device work lies inside), stop() returns
+    the summary of the samples inside the marked windows."""
+
+    INTERVAL_S = 0.001
 
     def __init__(self, local_rank):
         vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-        self.index = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.keys = [vis.split(",")[local_rank].strip() if vis else str(local_rank)]
+        try:
+            uuid = str(torch.cuda.get_device_properties(local_rank).uuid)
+            self.keys.insert(0, uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except (AttributeError, RuntimeError, AssertionError):
+            pass
         self.proc = None
         self.path = None
+        self.windows = []
 
     def start(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            fd, self.path = tempfile.mkstemp(suffix=".clk")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.index, "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+                [sys.executable, "-c", _NVML_SAMPLER, self.path, str(self.INTERVAL_S)] +
+                self.keys, stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+            return
+        # wait (bounded) until the sampler has its handle and is polling
+        t0 = time.monotonic()
+        while time.monotonic() - t0 < 10.0 and self.proc.poll() is None:
+            try:
+                with open(self.path) as f:
+                    if len(f.read().splitlines()) >= 3:
+                        break
+            except OSError:
+                pass
+            time.sleep(0.02)
+
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
 
     def stop(self):
         if self.proc is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
+        if self.proc.poll() is None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.proc.wait()
+        smax, rows = None, []
         try:
             with open(self.path) as f:
                 for line in f:
-                    parts = [x.strip() for x in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
+                    parts = line.split()
+                    if parts[:1] == ["max"] and len(parts) == 2:
+                        smax = float(parts[1])
+                    elif len(parts) == 3:
+                        rows.append((float(parts[0]), float(parts[1]), int(parts[2])))
             os.unlink(self.path)
-        except OSError:
+        except (OSError, ValueError):
             return None
-        if not rows:
+        inside = [r for r in rows if any(a <= r[0] <= b for a, b in self.windows)]
+        use = inside or rows
+        if not use:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted(n for n, bit in _REASON_BITS.items() if any(r[2] & bit for r in use))
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(inside), "samples_total": len(rows),
+                "interval_ms": 1e3 * self.INTERVAL_S,
+                "source": "NVML, samples inside the timed region" if inside else
+                          "NVML, no sample inside the timed region: all samples"}
 
 
 def measured_peak():
@@ -380,7 +455,50 @@ def run_reference(args, spec, world, rank):
 # ---------------------------------------------------------------------------
 # the product arm
 # ---------------------------------------------------------------------------
-def run_pkv(args, spec, world, rank, local):
+def cache_work_list(args):
+    return {"none": False, "longest_first": "longest_first", "grid": "grid"}[args.work_list]
+
+
+def allocator_latency(spec, lens, order, rank):
+    """Block-allocation latency of the host pool (the metric the "PagedAttention
+    动态内存分页" page lists under 性能监控要点): microseconds per batched append
+    (one token for every sequence of the batch, new blocks taken from the
+    pool as they fill) and per single-sequence append, both through the
+    Python binding, on a pool in the workload's state."""
+    from paged_kv_cache_337_b200 import _abi
+
+    S, bs = spec.num_seqs, spec.block_size
+    nb = len(order)
+    pool = _abi.BlockPool(nb, bs, order)
+    for s in range(S):
+        pool.add(s, int(lens[s]) - 1)
+    ids = torch.arange(S, dtype=torch.int64)
+    slots = torch.empty(S, dtype=torch.int64)
+    pairs = torch.empty((S, 2), dtype=torch.int32)
+    # stay within the pool's spare blocks: each round may take one per sequence
+    spare = pool.num_free() // max(1, S)
+    rounds = max(1, min(64, spare * bs // 2))
+    for _ in range(2):
+        pool.append_batch(ids, slots, pairs)
+    t0 = time.perf_counter()
+    for _ in range(rounds):
+        pool.append_batch(ids, slots, pairs)
+    batch_us = 1e6 * (time.perf_counter() - t0) / rounds
+    singles = min(S * 4, max(1, (pool.num_free() // 2) * bs))
+    t0 = time.perf_counter()
+    for i in range(singles):
+        pool.append(i % S)
+    single_us = 1e6 * (time.perf_counter() - t0) / singles
+    pool.close()
+    return {"append_batch_us": round(batch_us, 2), "batch": S,
+            "per_sequence_us": round(batch_us / S, 4), "append_single_us": round(single_us, 3),
+            "batches_timed": rounds, "singles_timed": singles,
+            "what": "host pool, Python binding included: one slot per sequence, a new block "
+                    "from the pool when the last one is full"}
+
+
+def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc=True):
+    """One decode workload: returns its JSON line (rank 0) or None."""
     from paged_kv_cache_337_b200 import _abi
     from paged_kv_cache_337_b200 import workloads as W
     from paged_kv_cache_337_b200.cache import PagedKVCache
@@ -400,10 +518,10 @@ def run_pkv(args, spec, world, rank, local):
     n_states = 16  # decode steps whose metadata is prepared (one block's worth)
     e2e_steps = 0 if args.no_e2e else min(args.steps, 48)
     mb = spec.max_blocks_per_seq + -(-(n_states + e2e_steps + 2) // bs)
-    fp8 = args.kv_dtype == "fp8"
     cache = PagedKVCache(nb, bs, Hq, Hkv, D, spec.torch_dtype, dev, mb, P,
                          free_order=order.tolist(), scale=spec.scale,
-                         kv_dtype=torch.uint8 if fp8 else None)
+                         kv_dtype=torch.uint8 if fp8 else None,
+                         work_list=cache_work_list(args))
     if fp8:
         W.fill_device_scales_(cache.k_scale, spec.seed * 10 + 2 * rank + 5)
         W.fill_device_scales_(cache.v_scale, spec.seed * 10 + 2 * rank + 6)
@@ -428,9 +546,11 @@ def run_pkv(args, spec, world, rank, local):
         st = prep["st"]
         npairs = prep["num_pairs"]
         lens = st["h_lens"].tolist()
+        n_items = prep["num_items"]
         states.append(dict(
             slots=st["h_slots"].to(dev), pairs=st["h_pairs"][:npairs].to(dev),
             tables=st["h_tables"].to(dev), lens=st["h_lens"].to(dev), max_len=max(lens),
+            items=st["h_items"][:n_items].to(dev) if n_items >= 0 else None,
             q=torch.randn((S, Hq, D), generator=dgen, device=dev).to(dt),
             k=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
             v=torch.randn((S, Hkv, D), generator=dgen, device=dev).to(dt),
@@ -464,11 +584,12 @@ def run_pkv(args, spec, world, rank, local):
         if fp8:
             _abi.pkv_decode_attention_fp8(out, state["q"], kc, vc, ks, vs, state["tables"],
                                           state["lens"], state["max_len"], spec.scale, P, ws,
-                                          dev_error=err, stream=stream)
+                                          dev_error=err, stream=stream,
+                                          work_items=state["items"])
         else:
             _abi.pkv_decode_attention(out, state["q"], kc, vc, state["tables"], state["lens"],
                                       state["max_len"], spec.scale, P, ws, dev_error=err,
-                                      stream=stream)
+                                      stream=stream, work_items=state["items"])
         if ev is not None:
             ev[1].record(stream)
         # copy-on-write: a bytes kernel, plus a scale kernel for e4m3 caches
@@ -481,7 +602,6 @@ def run_pkv(args, spec, world, rank, local):
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
     K = args.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
@@ -491,6 +611,7 @@ def run_pkv(args, spec, world, rank, local):
     bytes_step = bytes_decode = 0
     barrier(world)
     torch.cuda.synchronize(dev)
+    h0 = time.monotonic()
     t_start.record(stream)
     for i in range(K):
         stt = states[(args.warmup + i) % n_states]
@@ -499,6 +620,8 @@ def run_pkv(args, spec, world, rank, local):
         bytes_decode += stt["bytes_decode"]
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.window(h0, time.monotonic())
     barrier(world)
     clock_info = clocks.stop() if clocks else None
     elapsed_ms = t_start.elapsed_time(t_end)
@@ -520,7 +643,7 @@ def run_pkv(args, spec, world, rank, local):
     # host waits for it before the step ends.  The pool's work and the input
     # upload for step i+1 (on a second stream, into the other of two input
     # buffers) run while step i is on the GPU: neither depends on step i's
-    # output.
+    # output.  The host time of each part is recorded.
     e2e = None
     if e2e_steps:
         nq, nk = S * Hq * D, S * Hkv * D
@@ -535,6 +658,7 @@ def run_pkv(args, spec, world, rank, local):
         ev_out = torch.cuda.Event()                       # step result on the host
         e2e_bytes = 0
         h2d = d2h = 0
+        host = {"prepare": 0.0, "enqueue": 0.0, "input_upload_enqueue": 0.0, "wait": 0.0}
         barrier(world)
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
@@ -542,8 +666,10 @@ def run_pkv(args, spec, world, rank, local):
             d_in[0].copy_(h_in[0], non_blocking=True)
             ev_in[0].record(copy_stream)
         prep = cache.prepare_step(ids)
+        host["prepare"] += time.perf_counter() - t0
         for i in range(e2e_steps):
             b = i % 2
+            ta = time.perf_counter()
             with torch.cuda.stream(stream):
                 stream.wait_event(ev_in[b])
                 cache.upload_step(prep, stream)
@@ -552,11 +678,14 @@ def run_pkv(args, spec, world, rank, local):
                 ev_used[b].record(stream)
                 hout.copy_(out, non_blocking=True)
                 ev_out.record(stream)
+            tb = time.perf_counter()
+            host["enqueue"] += tb - ta
             lens = prep["st"]["h_lens"].tolist()
             e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
                           copy_bytes(spec, prep["num_pairs"], fp8))
             h2d = d_in[b].numel() * 2 + prep["st"]["h"].numel() * 4
             d2h = hout.numel() * 2
+            tc = time.perf_counter()
             if i + 1 < e2e_steps:
                 nb_ = 1 - b
                 with torch.cuda.stream(copy_stream):
@@ -564,54 +693,75 @@ def run_pkv(args, spec, world, rank, local):
                         copy_stream.wait_event(ev_used[nb_])  # step i-1 done with it
                     d_in[nb_].copy_(h_in[(i + 1) % 2], non_blocking=True)
                     ev_in[nb_].record(copy_stream)
+                td = time.perf_counter()
+                host["input_upload_enqueue"] += td - tc
                 prep = cache.prepare_step(ids)  # overlaps the GPU work of step i
+                tc = time.perf_counter()
+                host["prepare"] += tc - td
             ev_out.synchronize()
+            host["wait"] += time.perf_counter() - tc
         e2e_s = time.perf_counter() - t0
         barrier(world)
         e2e_s = max_over_ranks(e2e_s, world, dev)
         e2e_total = sum_over_ranks(e2e_bytes, world, dev)
         e2e = {"value": round(e2e_total / e2e_s / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": e2e_steps, "ms_per_step": round(1e3 * e2e_s / e2e_steps, 4)}
+               "steps": e2e_steps, "ms_per_step": round(1e3 * e2e_s / e2e_steps, 4),
+               "host_ms_per_step": {
+                   "pool_append_and_tables": round(1e3 * host["prepare"] / e2e_steps, 4),
+                   "metadata_upload_and_launches": round(1e3 * host["enqueue"] / e2e_steps, 4),
+                   "input_upload_enqueue": round(
+                       1e3 * host["input_upload_enqueue"] / e2e_steps, 4),
+                   "readback_wait": round(1e3 * host["wait"] / e2e_steps, 4)},
+               "device_ms_per_step": round(ms_per_step, 4)}
         cache.check_errors()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and with_cpu and not args.no_cpu_baseline:
         gbs, secs, n, reps, cores = time_oracle(spec, lens0, 10.0, fp8)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": "first %d of %d sequences (all %d query heads), decode step "
                          "repeated %d times, %.1f s" % (n, S, Hq, reps, secs)}
+    alloc = allocator_latency(spec, lens0, order.tolist(), rank) if with_alloc else None
 
-    if rank == 0:
-        traffic = profiled_traffic(kernel_source_digest(), workload_name(spec, fp8))
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if fp8 else "bf16" if dt == torch.bfloat16 else "f16",
-            "data": "synthetic",
-            "config": {
-                "workload": workload_name(spec, fp8), "num_seqs": S, "num_q_heads": Hq, "num_kv_heads": Hkv,
-                "head_dim": D, "block_size": bs, "context_lens": "U[%d,%d]" % (spec.len_lo,
-                                                                             spec.len_hi),
-                "pool_blocks": nb, "partition_size": P,
-                "kv_cache": ("e4m3, fp32 scale per (block, KV head)" if fp8 else
-                             "bf16" if dt == torch.bfloat16 else "f16"),
-                "step": "host slot append + slot write + paged decode attention"
-                        " (+ copy-on-write copies; split-K partitions merged in-kernel)",
-                "l2": "inputs larger than L2 (%.2f GB of K/V read per step)" % (
-                    states[0]["lens_sum"] * Hkv * D * (2 if fp8 else 4) / 1e9),
-                "states": "%d consecutive decode steps prepared by the host pool, replayed "
-                          "cyclically" % n_states},
-            "pct_hbm_peak": round(100 * value / (world * peak), 2),
-            "decode_tok_s": round(tok_s, 1),
-            "roofline": {"bound": "hbm", "achieved": round(decode_gbs, 2), "peak": peak,
-                         "unit": "GB/s", "frac": round(decode_gbs / peak, 4),
-                         "traffic": traffic, "kernel": "paged_decode_kernel",
-                         "peak_source": peak_kind},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clock_info,
-        }
-        print(json.dumps(line), flush=True)
+    if rank != 0:
+        return None
+    traffic = profiled_traffic(kernel_source_digest(), workload_name(spec, fp8))
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if fp8 else "bf16" if dt == torch.bfloat16 else "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": workload_name(spec, fp8), "num_seqs": S, "num_q_heads": Hq,
+            "num_kv_heads": Hkv, "head_dim": D, "block_size": bs,
+            "context_lens": "U[%d,%d]" % (spec.len_lo, spec.len_hi),
+            "pool_blocks": nb, "partition_size": P,
+            "grid": {"none": "full grid", "longest_first": "work list: (sequence, KV head, "
+                     "partition) items holding tokens, longest first",
+                     "grid": "work list: (sequence, KV head, partition) items holding tokens, "
+                     "in grid order"}[args.work_list],
+            "kv_cache": ("e4m3, fp32 scale per (block, KV head)" if fp8 else
+                         "bf16" if dt == torch.bfloat16 else "f16"),
+            "step": "slot write + paged decode attention (+ copy-on-write copies; split-K "
+                    "partitions merged in-kernel); the host pool's slot appends are done "
+                    "before timing, so value holds device work only and e2e holds the pool",
+            "l2": "inputs larger than L2 (%.2f GB of K/V read per step)" % (
+                states[0]["lens_sum"] * Hkv * D * (2 if fp8 else 4) / 1e9),
+            "states": "%d consecutive decode steps prepared by the host pool, replayed "
+                      "cyclically" % n_states},
+        "pct_hbm_peak": round(100 * value / (world * peak), 2),
+        "decode_tok_s": round(tok_s, 1),
+        "roofline": {"bound": "hbm", "achieved": round(decode_gbs, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(decode_gbs / peak, 4),
+                     "traffic": traffic, "kernel": "paged_decode_kernel",
+                     "peak_source": peak_kind},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clock_info,
+    }
+    if alloc is not None:
+        line["allocator"] = alloc
+    return line
 
 
 SWAP_WORKLOAD = "swap_7b_s256_q64_h32_d128_bs16_bf16"
@@ -667,11 +817,13 @@ def run_cow_layers(args, world, rank, local):
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
     barrier(world)
     K = args.steps
+    h0 = time.monotonic()
     ms = timed(one_launch, K)
     ms_layers = timed(per_layer, K)
+    if clocks:
+        clocks.window(h0, time.monotonic())
     barrier(world)
     clock_info = clocks.stop() if clocks else None
     t_max = max_over_ranks(ms, world, dev)
@@ -776,15 +928,17 @@ def run_swap(args, world, rank, local):
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize(dev)
+    h0 = time.monotonic()
     total = 0
     for i in range(K):
         total += step(evs[i])
     torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.window(h0, time.monotonic())
     barrier(world)
     clock_info = clocks.stop() if clocks else None
     out_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
@@ -850,7 +1004,7 @@ def prefill_flops(lens, n, Hq, D):
     return f
 
 
-def run_prefill(args, world, rank, local):
+def run_prefill(args, world, rank, local, with_cpu=True):
     """Paged prefill of 8 prompts of 2048 tokens (Hq 32 / Hkv 8, head_dim
     128, block size 16, bf16) over scattered blocks: each step writes the
     prompts' K/V into their slots (pkv_write_slots) and runs causal paged
@@ -904,18 +1058,20 @@ def run_prefill(args, world, rank, local):
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
     K = args.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
+    h0 = time.monotonic()
     t0.record(stream)
     for i in range(K):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.window(h0, time.monotonic())
     barrier(world)
     clock_info = clocks.stop() if clocks else None
     cache.check_errors()
@@ -926,7 +1082,7 @@ def run_prefill(args, world, rank, local):
     peak = measured_tensor_peak()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and with_cpu and not args.no_cpu_baseline:
         from oracle import reference as ref
 
         n_rows = 64  # the last 64 rows of one prompt: the heaviest rows
@@ -965,7 +1121,8 @@ def run_prefill(args, world, rank, local):
                          "kernel": "paged_prefill_kernel", "peak_source": peak[1]},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": 2 * K, "clocks": clock_info,
         }
-        print(json.dumps(line), flush=True)
+        return line
+    return None
 
 
 def measured_tensor_peak():
@@ -999,7 +1156,8 @@ def run_shared_prefix(args, world, rank, local):
     ids = list(range(S))
     mb = -(-(int(inp.prompt_lens.max()) + int(inp.diverge.max()) + 4) // bs)
     cache = PagedKVCache(inp.num_blocks, bs, Hq, Hkv, D, dt, dev, mb, 0,
-                         free_order=inp.free_order.tolist(), scale=spec.scale)
+                         free_order=inp.free_order.tolist(), scale=spec.scale,
+                         work_list=cache_work_list(args))
     W.fill_device_cache_(cache.key_cache, inp.seed_values + rank)
     W.fill_device_cache_(cache.value_cache, inp.seed_values + rank + 1)
     for p in range(Pn):
@@ -1020,8 +1178,10 @@ def run_shared_prefix(args, world, rank, local):
         for i in range(S):
             nblk = -(-lens[i] // bs)
             used.update(tables[i, :nblk].tolist())
+        ni = prep["num_items"]
         return dict(slots=st["h_slots"].to(dev), pairs=st["h_pairs"][:n].to(dev), npairs=n,
                     tables=tables.to(dev), lens=st["h_lens"].to(dev), max_len=max(lens),
+                    items=st["h_items"][:ni].to(dev) if ni >= 0 else None,
                     logical=decode_bytes(spec_like(spec), lens, 0) + write_bytes(spec, S) +
                     copy_bytes(spec, n),
                     unique=len(used) * bs * Hkv * D * 4,
@@ -1039,7 +1199,7 @@ def run_shared_prefix(args, world, rank, local):
                                  stream=stream)
             _abi.pkv_decode_attention(out, stt["q"], kc, vc, stt["tables"], stt["lens"],
                                       stt["max_len"], spec.scale, 0, None, dev_error=err,
-                                      stream=stream)
+                                      stream=stream, work_items=stt["items"])
             return (1 if stt["npairs"] else 0) + 2
 
         for _ in range(args.warmup):
@@ -1048,10 +1208,13 @@ def run_shared_prefix(args, world, rank, local):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize(dev)
+        h0 = time.monotonic()
         e0.record(stream)
         launches = sum(step() for _ in range(args.steps))
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        if clocks:
+            clocks.window(h0, time.monotonic())
         barrier(world)
         cache.check_errors()
         ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.steps
@@ -1060,6 +1223,9 @@ def run_shared_prefix(args, world, rank, local):
                 "unique_kv_gb": round(stt["unique"] / 1e9, 3), "cow_copies": stt["npairs"],
                 "logical_gb": round(stt["logical"] / 1e9, 3)}, launches
 
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
     fork = snapshot()
     fork_res, launches = time_state(fork)
     # every sample advances by its private tokens (host pool only; values
@@ -1069,6 +1235,7 @@ def run_shared_prefix(args, world, rank, local):
             cache.pool.append(s)
     steady = snapshot()
     steady_res, _ = time_state(steady)
+    clock_info = clocks.stop() if clocks else None
     peak, peak_kind = measured_peak()
     if rank == 0:
         line = {
@@ -1083,8 +1250,10 @@ def run_shared_prefix(args, world, rank, local):
             "fork_step": fork_res, "steady_step": steady_res,
             "decode_tok_s": round(world * S / (fork_res["ms_per_step"] * 1e-3), 1),
             "peak_gbs": peak, "peak_source": peak_kind, "gpu_launches": launches,
+            "clocks": clock_info,
         }
-        print(json.dumps(line), flush=True)
+        return line
+    return None
 
 
 def spec_like(spec):
@@ -1095,38 +1264,70 @@ def spec_like(spec):
                         spec.num_kv_heads, spec.head_dim, spec.block_size, 1, 1, spec.dtype)
 
 
+# The decode workloads measured beside the headline in the same process, with
+# the same --steps / --warmup and the same device timing: the 70B-shaped GQA
+# batch, the long split-K contexts at block sizes 32 and 64, both decode
+# shapes over e4m3 caches, the shared-prefix fork and steady steps, and
+# paged prefill.
+EXTRA_DECODE = (("70b_gqa_s64_hq64_hkv8_d128_bs16_bf16", False),
+                ("long_s8_l32768_hq32_hkv8_d128_bs32_bf16", False),
+                ("long_s8_l32768_hq32_hkv8_d128_bs64_bf16", False),
+                ("7b_s256_h32_d128_bs16_bf16", True),
+                ("70b_gqa_s64_hq64_hkv8_d128_bs16_bf16", True))
+
+
+def summary(line):
+    """The fields of a workload's line kept under the headline's workloads."""
+    keep = ("value", "unit", "ms_per_step", "roofline", "clocks", "e2e", "gpu_launches",
+            "decode_tok_s", "pct_hbm_peak", "fork_step", "steady_step", "dtype")
+    out = {k: line[k] for k in keep if k in line}
+    cfg = line.get("config", {})
+    out["config"] = {k: cfg[k] for k in ("workload", "partition_size", "grid", "step", "bytes")
+                     if k in cfg}
+    return out
+
+
+def run_extra_workloads(args, world, rank, local):
+    from paged_kv_cache_337_b200 import workloads as W
+
+    sub = argparse.Namespace(**vars(args))
+    sub.partition_size = -1
+    out = {}
+    runs = [(workload_name(W.SPECS[n], fp8),
+             lambda n=n, fp8=fp8: run_pkv(sub, W.SPECS[n], world, rank, local, fp8=fp8,
+                                          with_cpu=False, with_alloc=False))
+            for n, fp8 in EXTRA_DECODE]
+    runs.append((W.SHARED_PREFIX.name, lambda: run_shared_prefix(sub, world, rank, local)))
+    runs.append((PREFILL_WORKLOAD, lambda: run_prefill(sub, world, rank, local, with_cpu=False)))
+    for name, fn in runs:
+        try:
+            line = fn()
+            if line is not None:
+                out[name] = summary(line)
+        except Exception as e:  # recorded; the headline line still prints
+            if world > 1:
+                raise
+            out[name] = {"error": "%s: %s" % (type(e).__name__, e)}
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse_args()
     from paged_kv_cache_337_b200 import workloads as W
 
-    if args.workload == COW_LAYERS_WORKLOAD:
+    special = {COW_LAYERS_WORKLOAD: run_cow_layers, SWAP_WORKLOAD: run_swap}
+    returning = {PREFILL_WORKLOAD: run_prefill, W.SHARED_PREFIX.name: run_shared_prefix}
+    if args.workload in special or args.workload in returning:
         world, rank, local = dist_setup()
         try:
-            run_cow_layers(args, world, rank, local)
-        finally:
-            if world > 1:
-                torch.distributed.destroy_process_group()
-        return
-    if args.workload == PREFILL_WORKLOAD:
-        world, rank, local = dist_setup()
-        try:
-            run_prefill(args, world, rank, local)
-        finally:
-            if world > 1:
-                torch.distributed.destroy_process_group()
-        return
-    if args.workload == SWAP_WORKLOAD:
-        world, rank, local = dist_setup()
-        try:
-            run_swap(args, world, rank, local)
-        finally:
-            if world > 1:
-                torch.distributed.destroy_process_group()
-        return
-    if args.workload == W.SHARED_PREFIX.name:
-        world, rank, local = dist_setup()
-        try:
-            run_shared_prefix(args, world, rank, local)
+            if args.workload in special:
+                special[args.workload](args, world, rank, local)
+            else:
+                line = returning[args.workload](args, world, rank, local)
+                if line is not None:
+                    print(json.dumps(line), flush=True)
         finally:
             if world > 1:
                 torch.distributed.destroy_process_group()
@@ -1141,8 +1342,16 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, spec, world, rank)
-        else:
-            run_pkv(args, spec, world, rank, local)
+            return
+        fp8 = args.kv_dtype == "fp8"
+        line = run_pkv(args, spec, world, rank, local, fp8=fp8)
+        if (args.extra == "all" and args.workload == W.DECODE_7B.name and not fp8 and
+                not args.num_seqs):
+            extra = run_extra_workloads(args, world, rank, local)
+            if line is not None:
+                line["workloads"] = extra
+        if line is not None:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

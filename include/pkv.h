@@ -71,6 +71,7 @@ typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 #define PKV_DEVERR_SLOT 3        /* index: token; slot >= num_blocks * block_size */
 #define PKV_DEVERR_PAIR 4        /* index: pair; a block id outside [0, num_blocks) */
 #define PKV_DEVERR_TIMEOUT 5     /* index: 0; a bounded wait on a copy ran out */
+#define PKV_DEVERR_WORK_ITEM 6   /* index: CTA; a work-list entry outside the grid */
 
 /* ---------------------------------------------------------------------- */
 /* Slot write                                                              */
@@ -199,6 +200,73 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
                          int32_t* dev_error, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
+/* Decode work list: per-sequence partitions, longest first                */
+/* ---------------------------------------------------------------------- */
+/*
+ * The pages note that sequences of very different lengths are what makes a
+ * batch costly to schedule ("PagedAttention 动态内存分页" page, 技术边界与取舍).
+ * pkv_decode_attention's grid has num_seqs * num_kv_heads * NP slots (NP =
+ * partitions of the longest sequence), and slots past a shorter sequence's
+ * end exit at once, in grid order.  This host-side planner lists instead
+ * the work items that hold tokens: one per (sequence s, KV head, partition
+ * p) with p < max(1, ceil(L_s / P)), so a short sequence runs one pass and
+ * a long one is split.  order:
+ *   PKV_ITEMS_LONGEST_FIRST  by the 16-token tiles each item holds, most
+ *                            first (ties in grid order): the long items
+ *                            start first and the short ones fill the end
+ *                            of the launch
+ *   PKV_ITEMS_GRID           grid order (the empty slots left out): the
+ *                            items of one sequence, and of sequences next
+ *                            to each other in the batch, run side by side
+ *
+ *   context_lens     HOST int32 [num_seqs]: the same lengths the device
+ *                    copy passed to the attention call holds
+ *   max_context_len, partition_size
+ *                    exactly as they will be passed to the attention call
+ *                    (they fix P and NP as pkv_decode_attention does)
+ *   items            HOST int32 [capacity]: receives the items, each the
+ *                    flat index (s * num_kv_heads + kv_head) * NP + p
+ *   num_items        receives the number of items.  When it exceeds
+ *                    capacity, nothing is written to items and
+ *                    PKV_ERR_INVALID is returned (num_items still set);
+ *                    num_kv_heads * sum_s max(1, ceil(L_s / P)) is the count
+ *                    and num_seqs * num_kv_heads * NP always suffices.
+ * A length outside [0, max_context_len] or an unknown order returns
+ * PKV_ERR_INVALID.  O(items + P / 16): a counting sort on the host, no
+ * device work.
+ */
+#define PKV_ITEMS_LONGEST_FIRST 0
+#define PKV_ITEMS_GRID 1
+PKV_API int pkv_decode_work_items(const int32_t* context_lens, int num_seqs, int num_kv_heads,
+                                  int max_context_len, int partition_size, int order,
+                                  int32_t* items, int capacity, int* num_items);
+
+/*
+ * pkv_decode_attention over a work list from pkv_decode_work_items: one
+ * CTA per item, in list order.  Every other argument, the result and the
+ * errors are those of pkv_decode_attention.
+ *   work_items       DEVICE int32 [num_items]: the planner's list for the
+ *                    same context lengths, max_context_len and
+ *                    partition_size.  An entry outside the grid is reported
+ *                    (PKV_DEVERR_WORK_ITEM) and skipped; a list that misses
+ *                    an item of a sequence leaves that sequence's output
+ *                    unwritten, and one that repeats an item gives an
+ *                    unspecified result for that sequence (no access leaves
+ *                    the buffers either way).
+ *   num_items        0 launches nothing
+ */
+PKV_API int pkv_decode_attention_items(void* out, const void* query, const void* key_cache,
+                                       const void* value_cache, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       int num_seqs, int max_context_len, int num_q_heads,
+                                       int num_kv_heads, int head_dim, int num_blocks,
+                                       int block_size, int64_t block_stride, float scale,
+                                       int partition_size, void* workspace,
+                                       size_t workspace_bytes, const int32_t* work_items,
+                                       int num_items, pkv_dtype dtype, int32_t* dev_error,
+                                       cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* Paged prefill attention                                                 */
 /* ---------------------------------------------------------------------- */
 /*
@@ -252,12 +320,16 @@ PKV_API int pkv_prefill_attention(void* out, const void* query, const void* key_
  * from a device array built into the library.
  *
  *   - The array is PKV_NOALLOC_WORKSPACE_BYTES long and lives on every GPU
- *     where this entry point has been called, until the process exits.  A
- *     call whose sizes need more (see pkv_decode_workspace_bytes) returns
- *     PKV_ERR_WORKSPACE and launches nothing.
- *   - The first call on a device looks up that device's copy of the array
- *     (cudaGetSymbolAddress) and keeps the address; make that first call
- *     before any stream capture.
+ *     where this entry point has been called, until the process exits.
+ *     With CUDA_MODULE_LOADING=EAGER it lives on every GPU whose context
+ *     loads the library, called or not.  A call whose sizes need more (see
+ *     pkv_decode_workspace_bytes) returns PKV_ERR_WORKSPACE and launches
+ *     nothing.
+ *   - The first call on a device with num_seqs > 0 (split-K or not) looks
+ *     up that device's copy of the array (cudaGetSymbolAddress) and keeps
+ *     the address, keyed by the device's CUDA context; make that first
+ *     call before any stream capture.  A context made anew on the device
+ *     (after cudaDeviceReset, say) is looked up again at its first call.
  *   - Nothing here allocates: no cudaMalloc, no cudaFree, no allocating
  *     library routine.
  *   - Every call on a device shares the one array, which keeps whatever the
@@ -336,6 +408,22 @@ PKV_API int pkv_decode_attention_fp8(void* out, const void* query, const void* k
                                      int partition_size, void* workspace,
                                      size_t workspace_bytes, pkv_dtype dtype,
                                      int32_t* dev_error, cudaStream_t stream);
+
+/*
+ * pkv_decode_attention_fp8 over a work list from pkv_decode_work_items
+ * (work_items and num_items as in pkv_decode_attention_items).
+ */
+PKV_API int pkv_decode_attention_fp8_items(void* out, const void* query, const void* key_cache,
+                                           const void* value_cache, const float* k_scale,
+                                           const float* v_scale, const int32_t* block_tables,
+                                           int max_blocks_per_seq, const int32_t* context_lens,
+                                           int num_seqs, int max_context_len, int num_q_heads,
+                                           int num_kv_heads, int head_dim, int num_blocks,
+                                           int block_size, int64_t block_stride, float scale,
+                                           int partition_size, void* workspace,
+                                           size_t workspace_bytes, const int32_t* work_items,
+                                           int num_items, pkv_dtype dtype, int32_t* dev_error,
+                                           cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
 /* Host block pool (allocator)                                             */

@@ -28,6 +28,10 @@ PKV_DEVERR_BLOCK_ID = 2
 PKV_DEVERR_SLOT = 3
 PKV_DEVERR_PAIR = 4
 PKV_DEVERR_TIMEOUT = 5
+PKV_DEVERR_WORK_ITEM = 6
+
+PKV_ITEMS_LONGEST_FIRST = 0
+PKV_ITEMS_GRID = 1
 
 PKV_NOALLOC_WORKSPACE_BYTES = 64 << 20
 
@@ -42,6 +46,9 @@ SIGNATURES = {
     "pkv_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "pkv_decode_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i,
                                   _i64, _f, _i, _p, _sz, _i, _p, _p]),
+    "pkv_decode_attention_items": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
+                                        _i, _i64, _f, _i, _p, _sz, _p, _i, _i, _p, _p]),
+    "pkv_decode_work_items": (_i, [_p, _i, _i, _i, _i, _i, _p, _i, _p]),
     "pkv_decode_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i,
                                           _i, _i64, _f, _i, _i, _p, _p]),
     "pkv_prefill_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i,
@@ -51,6 +58,9 @@ SIGNATURES = {
     "pkv_copy_blocks_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i64, _p, _p]),
     "pkv_decode_attention_fp8": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i,
                                       _i, _i, _i64, _f, _i, _p, _sz, _i, _p, _p]),
+    "pkv_decode_attention_fp8_items": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i,
+                                            _i, _i, _i, _i, _i64, _f, _i, _p, _sz, _p, _i, _i,
+                                            _p, _p]),
     "pkv_pool_create": (_i, [_i, _i, _p, C.POINTER(_p)]),
     "pkv_pool_destroy": (None, [_p]),
     "pkv_seq_add": (_i, [_p, _i64, _i]),
@@ -245,14 +255,48 @@ def pkv_decode_workspace_bytes(num_seqs, num_q_heads, max_context_len, partition
                                                 partition_size, head_dim))
 
 
+def pkv_decode_work_items(context_lens, num_kv_heads, max_context_len, partition_size,
+                          out=None, order=PKV_ITEMS_LONGEST_FIRST):
+    """The decode work list for these lengths (a host int32 tensor or
+    sequence): every (sequence, KV head, partition) that holds tokens, as
+    flat grid indices, the items holding the most tokens first
+    (PKV_ITEMS_LONGEST_FIRST) or in grid order (PKV_ITEMS_GRID).  Returns an
+    int32 CPU tensor (a view of `out` when given, e.g. pinned staging)."""
+    lens = torch.as_tensor(context_lens, dtype=torch.int32)
+    if lens.device.type != "cpu":
+        raise ValueError("pkv_decode_work_items: context_lens must be on the host")
+    lens = lens.contiguous()
+    S = lens.numel()
+    n = C.c_int()
+    cap = out.numel() if out is not None else 0
+    if out is None:
+        lib().pkv_decode_work_items(_ptr(lens), S, num_kv_heads, int(max_context_len),
+                                    int(partition_size), int(order), None, 0, C.byref(n))
+        if n.value == 0 and S > 0:  # a size error: report it
+            _check(lib().pkv_decode_work_items(_ptr(lens), S, num_kv_heads,
+                                               int(max_context_len), int(partition_size),
+                                               int(order), None, 0, C.byref(n)),
+                   "pkv_decode_work_items")
+        out = torch.empty(max(n.value, 1), dtype=torch.int32)
+        cap = out.numel()
+    elif out.dtype != torch.int32 or out.device.type != "cpu" or not out.is_contiguous():
+        raise ValueError("pkv_decode_work_items: out must be a contiguous host int32 tensor")
+    _check(lib().pkv_decode_work_items(_ptr(lens), S, num_kv_heads, int(max_context_len),
+                                       int(partition_size), int(order), _ptr(out), cap,
+                                       C.byref(n)), "pkv_decode_work_items")
+    return out[:n.value]
+
+
 def pkv_decode_attention(out, query, key_cache, value_cache, block_tables, context_lens,
                          max_context_len, scale, partition_size=0, workspace=None,
-                         dev_error=None, stream=None):
+                         dev_error=None, stream=None, work_items=None):
     """Paged decode attention: out/query [S, Hq, D]; block_tables int32
     [S, MB]; context_lens int32 [S]; workspace a uint8 device tensor of at
-    least pkv_decode_workspace_bytes(...) bytes when partitions are used."""
+    least pkv_decode_workspace_bytes(...) bytes when partitions are used.
+    work_items: a device int32 list from pkv_decode_work_items for the same
+    lengths (pkv_decode_attention_items), or None for the full grid."""
     _on_device("pkv_decode_attention", out, query, key_cache, value_cache, block_tables,
-               context_lens, workspace, dev_error)
+               context_lens, workspace, dev_error, work_items)
     nb, bs, hkv, d, bstride = _cache_geometry(key_cache)
     if _cache_geometry(value_cache) != (nb, bs, hkv, d, bstride):
         raise ValueError("key_cache and value_cache differ in geometry")
@@ -269,6 +313,15 @@ def pkv_decode_attention(out, query, key_cache, value_cache, block_tables, conte
         _need(dev_error, torch.int32, "dev_error")
     mb = block_tables.shape[1]
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if work_items is not None:
+        _need(work_items, torch.int32, "work_items")
+        st = lib().pkv_decode_attention_items(
+            _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), mb,
+            _ptr(context_lens), S, int(max_context_len), hq, hkv, d, nb, bs, bstride,
+            float(scale), int(partition_size), _ptr(workspace), ws_bytes, _ptr(work_items),
+            work_items.numel(), _dtype(query), _ptr(dev_error), _stream(stream, query.device))
+        _check(st, "pkv_decode_attention_items")
+        return
     st = lib().pkv_decode_attention(
         _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), mb,
         _ptr(context_lens), S, int(max_context_len), hq, hkv, d, nb, bs, bstride,
@@ -407,11 +460,13 @@ def pkv_copy_blocks_fp8(key_cache, value_cache, k_scale, v_scale, block_pairs, d
 
 def pkv_decode_attention_fp8(out, query, key_cache, value_cache, k_scale, v_scale,
                              block_tables, context_lens, max_context_len, scale,
-                             partition_size=0, workspace=None, dev_error=None, stream=None):
+                             partition_size=0, workspace=None, dev_error=None, stream=None,
+                             work_items=None):
     """pkv_decode_attention over e4m3 caches with per-(block, KV head)
-    scales; query/out stay f16 or bf16."""
+    scales; query/out stay f16 or bf16.  work_items as in
+    pkv_decode_attention (pkv_decode_attention_fp8_items)."""
     _on_device("pkv_decode_attention_fp8", out, query, key_cache, value_cache, k_scale, v_scale,
-               block_tables, context_lens, workspace, dev_error)
+               block_tables, context_lens, workspace, dev_error, work_items)
     nb, bs, hkv, d, bstride = _fp8_geometry("pkv_decode_attention_fp8", key_cache, value_cache,
                                             k_scale, v_scale)
     S, hq, dq = query.shape
@@ -424,6 +479,16 @@ def pkv_decode_attention_fp8(out, query, key_cache, value_cache, k_scale, v_scal
     if block_tables.dim() != 2 or block_tables.shape[0] != S or context_lens.numel() != S:
         raise ValueError("block_tables must be [num_seqs, max_blocks] and context_lens [num_seqs]")
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if work_items is not None:
+        _need(work_items, torch.int32, "work_items")
+        st = lib().pkv_decode_attention_fp8_items(
+            _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+            _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,
+            int(max_context_len), hq, hkv, d, nb, bs, bstride, float(scale),
+            int(partition_size), _ptr(workspace), ws_bytes, _ptr(work_items),
+            work_items.numel(), _dtype(query), _ptr(dev_error), _stream(stream, query.device))
+        _check(st, "pkv_decode_attention_fp8_items")
+        return
     st = lib().pkv_decode_attention_fp8(
         _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
         _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S,

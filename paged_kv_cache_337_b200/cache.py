@@ -17,8 +17,16 @@ block) the three device calls are their ``_fp8`` forms, which also copy and
 read the per-(block, KV head) scales.
 
 Steps 2-4 are launched on one stream; the metadata of step 1 travels to the
-device through pinned host staging buffers.  All arithmetic is in the
-library; this module only moves arguments.
+device through pinned host staging buffers.  With ``work_list`` (the
+default) step 1 also asks the library for the decode work list
+(``pkv_decode_work_items``: every (sequence, KV head, partition) holding
+tokens, the longest first or in grid order) and step 4 runs over it
+(``pkv_decode_attention_items``).  All arithmetic is in the library; this
+module only moves arguments.
+
+``upload_step`` and ``launch_step`` may run on different streams: the
+launch waits for the upload's event, and the next upload into the same
+staging bank waits for the last launch that read it.
 """
 import torch
 
@@ -28,12 +36,16 @@ from . import _abi
 class PagedKVCache:
     def __init__(self, num_blocks, block_size, num_q_heads, num_kv_heads, head_dim, dtype,
                  device, max_blocks_per_seq, partition_size=0, free_order=None,
-                 key_cache=None, value_cache=None, scale=None, kv_dtype=None, kv_scale=1.0):
+                 key_cache=None, value_cache=None, scale=None, kv_dtype=None, kv_scale=1.0,
+                 work_list=True):
         """dtype is the type of queries, new K/V rows and outputs (f16 or
         bf16).  kv_dtype torch.uint8 (or torch.float8_e4m3fn) stores the
         cache as e4m3 codes with a scale per (block, KV head) in k_scale /
         v_scale ([num_blocks, num_kv_heads] fp32, every entry kv_scale until
-        the caller sets them); None stores it in dtype."""
+        the caller sets them); None stores it in dtype.  work_list: decode
+        over the library's work list instead of the full grid, its items
+        longest first (True or "longest_first") or in grid order ("grid");
+        False: the full grid."""
         self.num_blocks = num_blocks
         self.block_size = block_size
         self.num_q_heads = num_q_heads
@@ -43,6 +55,12 @@ class PagedKVCache:
         self.device = torch.device(device)
         self.max_blocks_per_seq = max_blocks_per_seq
         self.partition_size = partition_size
+        orders = {True: _abi.PKV_ITEMS_LONGEST_FIRST,
+                  "longest_first": _abi.PKV_ITEMS_LONGEST_FIRST, "grid": _abi.PKV_ITEMS_GRID}
+        if work_list is not False and work_list not in orders:
+            raise ValueError("work_list must be True, False, 'longest_first' or 'grid'")
+        self.work_list = work_list is not False
+        self._item_order = orders.get(work_list, _abi.PKV_ITEMS_LONGEST_FIRST)
         self.scale = scale if scale is not None else 1.0 / (head_dim ** 0.5)
         shape = (num_blocks, block_size, num_kv_heads, head_dim)
         kv_dtype = dtype if kv_dtype is None else kv_dtype
@@ -80,31 +98,47 @@ class PagedKVCache:
         self.pool.free(seq_id)
 
     # -- one decode step --------------------------------------------------
+    def _item_capacity(self, n):
+        """Work items a batch of n sequences can need: every (sequence, KV
+        head, partition) of the longest context the tables can hold."""
+        if not self.work_list:
+            return 0
+        longest = self.max_blocks_per_seq * self.block_size
+        P = self.partition_size
+        parts = 1 if P <= 0 or P >= longest else -(-longest // P)
+        return n * self.num_kv_heads * parts
+
     def _stage(self, n):
         """Staging for a batch of n sequences: two banks, each one pinned host
         buffer and one device buffer holding slots | lengths | copy pairs |
-        Block Tables, so a step's metadata travels in one copy and the next
-        step can be prepared while the previous upload is in flight."""
+        Block Tables | work items, so a step's metadata travels in one copy
+        (of the used prefix) and the next step can be prepared while the
+        previous upload is in flight."""
         banks = self._staging.get(n)
         if banks is None:
             pin = torch.cuda.is_available()
             mb = self.max_blocks_per_seq
-            words = 2 * n + n + 2 * n + n * mb  # int32 words
+            cap = self._item_capacity(n)
+            t0 = 5 * n
+            i0 = t0 + n * mb
+            words = i0 + cap  # int32 words
 
             def views(buf):
                 return dict(slots=buf[:2 * n].view(torch.int64), lens=buf[2 * n:3 * n],
-                            pairs=buf[3 * n:5 * n].view(n, 2), tables=buf[5 * n:].view(n, mb))
+                            pairs=buf[3 * n:5 * n].view(n, 2),
+                            tables=buf[t0:i0].view(n, mb), items=buf[i0:])
 
             banks = []
             for _ in range(2):
-                h = torch.empty(words, dtype=torch.int32, pin_memory=pin)
-                d = torch.empty(words, dtype=torch.int32, device=self.device)
+                h = torch.empty(max(words, 1), dtype=torch.int32, pin_memory=pin)
+                d = torch.empty(max(words, 1), dtype=torch.int32, device=self.device)
                 hv, dv = views(h), views(d)
                 banks.append(dict(ids=torch.empty(n, dtype=torch.int64), h=h, d=d,
                                   h_slots=hv["slots"], h_lens=hv["lens"], h_pairs=hv["pairs"],
-                                  h_tables=hv["tables"], d_slots=dv["slots"],
-                                  d_lens=dv["lens"], d_pairs=dv["pairs"],
-                                  d_tables=dv["tables"], uploaded=None))
+                                  h_tables=hv["tables"], h_items=hv["items"],
+                                  d_slots=dv["slots"], d_lens=dv["lens"], d_pairs=dv["pairs"],
+                                  d_tables=dv["tables"], d_items=dv["items"], items_off=i0,
+                                  uploaded=None, consumed=None))
             self._staging[n] = banks = [banks, 0]
         banks[1] ^= 1
         return banks[0][banks[1]]
@@ -122,14 +156,23 @@ class PagedKVCache:
         slots, pairs = self.pool.append_batch(st["ids"], st["h_slots"], st["h_pairs"])
         tables, lens, longest = self.pool.block_tables(
             st["ids"], self.max_blocks_per_seq, -1, st["h_tables"], st["h_lens"], with_max=True)
-        return dict(st=st, num_pairs=pairs.shape[0], max_len=longest)
+        n_items = -1  # the full grid
+        if self.work_list:
+            n_items = _abi.pkv_decode_work_items(lens, self.num_kv_heads, longest,
+                                                 self.partition_size, st["h_items"],
+                                                 self._item_order).numel()
+        return dict(st=st, num_pairs=pairs.shape[0], max_len=longest, num_items=n_items)
 
     def upload_step(self, prep, stream=None):
-        """One host-to-device copy of a prepared step's metadata."""
+        """One host-to-device copy of a prepared step's metadata (the work
+        items the step uses, not the whole capacity)."""
         st = prep["st"]
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        used = st["items_off"] + max(prep.get("num_items", 0), 0)
         with torch.cuda.stream(s):
-            st["d"].copy_(st["h"], non_blocking=True)
+            if st["consumed"] is not None:
+                s.wait_event(st["consumed"])  # the last launch that read this bank
+            st["d"][:used].copy_(st["h"][:used], non_blocking=True)
             if st["uploaded"] is None:
                 st["uploaded"] = torch.cuda.Event()
             st["uploaded"].record(s)
@@ -143,17 +186,33 @@ class PagedKVCache:
 
     def launch_step(self, prep, query, key, value, out, max_len=None, stream=None):
         """Device part of a decode step (copy, write, attention) with the
-        prepared metadata already uploaded."""
+        prepared metadata uploaded by upload_step (on this or another
+        stream: the launch waits for it)."""
         st = prep["st"]
         n = prep["num_pairs"]
+        items = prep.get("num_items", -1)
+        if max_len is not None and max_len != prep["max_len"]:
+            items = -1  # the work list was planned for the prepared bound
         max_len = prep["max_len"] if max_len is None else max_len
+        s_ = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if st["uploaded"] is not None:
+            s_.wait_event(st["uploaded"])
+        try:
+            return self._launch(st, n, items, max_len, query, key, value, out, stream)
+        finally:
+            if st["consumed"] is None:
+                st["consumed"] = torch.cuda.Event()
+            st["consumed"].record(s_)
+
+    def _launch(self, st, n, items, max_len, query, key, value, out, stream):
         if n:
             self._copy(st["d_pairs"][:n], stream)
         ws = self.workspace(len(st["ids"]), max_len)
+        wl = st["d_items"][:items] if items >= 0 else None
         if not self._checked(query, key, value, out):
             # first use of these tensor shapes: the binding's full checks
             self._write(key, value, st["d_slots"], stream)
-            self._attend(out, query, st["d_tables"], st["d_lens"], max_len, ws, stream)
+            self._attend(out, query, st["d_tables"], st["d_lens"], max_len, ws, stream, wl)
             self._seen.add(self._signature(query, key, value, out))
             return out
         # same shapes, dtypes and device as a call already checked: pass the
@@ -165,28 +224,28 @@ class PagedKVCache:
         S = query.shape[0]
         err = self.dev_error.data_ptr()
         wsp, wsn = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
+        args = (st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
+                int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
+                int(self.partition_size), wsp, wsn)
+        tail = (self._dtype_code, err, sp)
+        if wl is not None:
+            tail = (wl.data_ptr(), wl.numel()) + tail
         if self.fp8:
             ks, vs = self.k_scale.data_ptr(), self.v_scale.data_ptr()
             _abi._check(L.pkv_write_slots_fp8(
                 key.data_ptr(), value.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
                 st["d_slots"].data_ptr(), S, nb, bs, hkv, d, bstride, self._dtype_code, err, sp),
                 "pkv_write_slots_fp8")
-            _abi._check(L.pkv_decode_attention_fp8(
-                out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
-                st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
-                int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
-                int(self.partition_size), wsp, wsn, self._dtype_code, err, sp),
-                "pkv_decode_attention_fp8")
+            fn = L.pkv_decode_attention_fp8_items if wl is not None else L.pkv_decode_attention_fp8
+            _abi._check(fn(out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
+                           *args, *tail), "pkv_decode_attention_fp8")
             return out
         _abi._check(L.pkv_write_slots(key.data_ptr(), value.data_ptr(), kc.data_ptr(),
                                       vc.data_ptr(), st["d_slots"].data_ptr(), S, nb, bs, hkv,
                                       d, bstride, self._dtype_code, err, sp), "pkv_write_slots")
-        _abi._check(L.pkv_decode_attention(
-            out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(),
-            st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
-            int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
-            int(self.partition_size), wsp, wsn, self._dtype_code, err, sp),
-            "pkv_decode_attention")
+        fn = L.pkv_decode_attention_items if wl is not None else L.pkv_decode_attention
+        _abi._check(fn(out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), *args,
+                       *tail), "pkv_decode_attention")
         return out
 
     # -- the three device calls, for either cache type ---------------------
@@ -208,16 +267,18 @@ class PagedKVCache:
             _abi.pkv_write_slots(key, value, self.key_cache, self.value_cache, slots,
                                  dev_error=self.dev_error, stream=stream)
 
-    def _attend(self, out, query, tables, lens, max_len, ws, stream):
+    def _attend(self, out, query, tables, lens, max_len, ws, stream, work_items=None):
         if self.fp8:
             _abi.pkv_decode_attention_fp8(out, query, self.key_cache, self.value_cache,
                                           self.k_scale, self.v_scale, tables, lens, max_len,
                                           self.scale, self.partition_size, ws,
-                                          dev_error=self.dev_error, stream=stream)
+                                          dev_error=self.dev_error, stream=stream,
+                                          work_items=work_items)
         else:
             _abi.pkv_decode_attention(out, query, self.key_cache, self.value_cache, tables,
                                       lens, max_len, self.scale, self.partition_size, ws,
-                                      dev_error=self.dev_error, stream=stream)
+                                      dev_error=self.dev_error, stream=stream,
+                                      work_items=work_items)
 
     def _signature(self, query, key, value, out):
         return tuple((tuple(t.shape), t.dtype, t.device, t.is_contiguous())

@@ -56,6 +56,7 @@ extern "C" int pkv_copy_blocks(void* key_cache, void* value_cache, const int32_t
                                int num_pairs, int num_blocks, int block_size, int num_kv_heads,
                                int head_dim, int64_t block_stride, pkv_dtype dtype,
                                int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_copy_blocks");
     using namespace pkv;
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_copy_blocks: dtype %d", (int)dtype);
@@ -110,6 +111,7 @@ extern "C" int pkv_copy_blocks_fp8(void* key_cache, void* value_cache, float* k_
                                    int num_blocks, int block_size, int num_kv_heads,
                                    int head_dim, int64_t block_stride, int32_t* dev_error,
                                    cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_copy_blocks_fp8");
     using namespace pkv;
     PKV_REQUIRE(num_pairs >= 0 && num_blocks >= 0 && block_size > 0 && num_kv_heads > 0 &&
                     head_dim > 0,
@@ -195,6 +197,7 @@ extern "C" int pkv_copy_blocks_layers(void* const* key_caches, void* const* valu
                                       int num_blocks, int64_t block_bytes,
                                       int64_t block_stride_bytes, int32_t* dev_error,
                                       cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_copy_blocks_layers");
     using namespace pkv;
     PKV_REQUIRE(num_layers >= 0 && num_pairs >= 0 && num_blocks >= 0 && block_bytes > 0,
                 PKV_ERR_INVALID, "pkv_copy_blocks_layers: bad sizes");

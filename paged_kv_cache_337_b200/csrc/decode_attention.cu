@@ -44,9 +44,11 @@
 // fills such a tile with zeros, so no access leaves the cache.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <type_traits>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -66,6 +68,11 @@ constexpr int kSubTileBytes = kTile * kBoxD * 2;   // one swizzled box: 2 KiB
 #endif
 #ifndef PKV_DECODE_STAGES_D64
 #define PKV_DECODE_STAGES_D64 4
+#endif
+// Whether the e4m3 path (every product in f16) adds the f16 remainder of P
+// as a second P V product, as the 16-bit paths do.
+#ifndef PKV_DECODE_E4M3_P_REMAINDER
+#define PKV_DECODE_E4M3_P_REMAINDER 1
 #endif
 constexpr int kWarps = PKV_DECODE_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -90,6 +97,10 @@ struct DecodeParams {
     const float* k_scale;  // e4m3 caches: [num_blocks, Hkv] dequantisation scales
     const float* v_scale;
     int32_t* dev_error;
+    // Optional work list: CTA i handles item work_items[i], a flat index
+    // (s * num_kv_heads + kvh) * num_partitions + part; null means CTA i
+    // handles item i of the full grid.
+    const int32_t* work_items;
     int num_seqs;
     int num_kv_heads;
     int max_blocks_per_seq;
@@ -275,6 +286,8 @@ struct MmaWarp {
     static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
     static constexpr int GP = NT * 8;  // heads held (padded)
     static constexpr bool kMma = true;
+    // the remainder of P as a second product (always for 16-bit caches)
+    static constexpr bool kPRem = !E4 || PKV_DECODE_E4M3_P_REMAINDER;
     uint32_t qf[KS][NT][2];            // Q^T B-fragments
     float acc[KS][NT][4];              // O^T[d][head]
     float m[NT][2], l[NT][2];          // per lane: heads nt*8 + (lane&3)*2 + {0,1}
@@ -468,8 +481,10 @@ struct MmaWarp {
             const float2 b01 = Storage<MT>::to_float2(h01), b23 = Storage<MT>::to_float2(h23);
             pb[nt][0] = movmatrix_trans(h01);
             pb[nt][1] = movmatrix_trans(h23);
-            pl[nt][0] = movmatrix_trans(Storage<MT>::from_float2(p0 - b01.x, p1 - b01.y));
-            pl[nt][1] = movmatrix_trans(Storage<MT>::from_float2(p2 - b23.x, p3 - b23.y));
+            if constexpr (kPRem) {
+                pl[nt][0] = movmatrix_trans(Storage<MT>::from_float2(p0 - b01.x, p1 - b01.y));
+                pl[nt][1] = movmatrix_trans(Storage<MT>::from_float2(p2 - b23.x, p3 - b23.y));
+            }
         }
         // O^T[d][head] += V^T P^T over the 16 tokens
         if constexpr (E4) {
@@ -492,7 +507,8 @@ struct MmaWarp {
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
                         Mma<MT>::m16n8k16(acc[2 * mp + h][nt], a, pb[nt][0], pb[nt][1]);
-                        Mma<MT>::m16n8k16(acc[2 * mp + h][nt], a, pl[nt][0], pl[nt][1]);
+                        if constexpr (kPRem)
+                            Mma<MT>::m16n8k16(acc[2 * mp + h][nt], a, pl[nt][0], pl[nt][1]);
                     }
                 }
             }
@@ -596,9 +612,20 @@ __device__ __forceinline__ void decode_cta(const CUtensorMap& kmap, const CUtens
 
     // Flat grid, partition fastest: the partitions of one (sequence, KV
     // head) run side by side, so their merge happens early and in parallel
-    // with the other CTAs' streaming rather than all at the end.
-    const int part = (int)(blockIdx.x % (unsigned)p.num_partitions);
-    const int rest = (int)(blockIdx.x / (unsigned)p.num_partitions);
+    // with the other CTAs' streaming rather than all at the end.  With a
+    // work list the CTA takes its item from the list instead (the host
+    // orders the items longest first and leaves out empty partitions).
+    unsigned item = blockIdx.x;
+    if (p.work_items != nullptr) {
+        item = (unsigned)__ldg(p.work_items + blockIdx.x);
+        if (item >= (unsigned)p.num_seqs * (unsigned)p.num_kv_heads *
+                        (unsigned)p.num_partitions) {
+            if (threadIdx.x == 0) report_error(p.dev_error, PKV_DEVERR_WORK_ITEM, blockIdx.x);
+            return;
+        }
+    }
+    const int part = (int)(item % (unsigned)p.num_partitions);
+    const int rest = (int)(item / (unsigned)p.num_partitions);
     const int kvh = rest % p.num_kv_heads;
     const int s = rest / p.num_kv_heads;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -951,7 +978,7 @@ void plan_partitions(int max_context_len, int partition_size, int* P, int* NP) {
 
 template <typename T, int D, typename Warp, bool FP8>
 int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
-                  int num_kv_heads, cudaStream_t stream) {
+                  int num_kv_heads, int num_items, cudaStream_t stream) {
     using Pl = Plan<D, FP8, Warp::kMma>;
     const int table_cap = (p.partition_size + p.block_size - 1) / p.block_size + 1;
     const size_t smem = 1024 + Pl::kTableOff + (size_t)table_cap * sizeof(int32_t);
@@ -984,7 +1011,9 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
             return fail(PKV_ERR_CUDA, "pkv_decode_attention: clearing the partition counters: %s",
                         cudaGetErrorString(e));
     }
-    const int64_t ctas = (int64_t)p.num_seqs * num_kv_heads * p.num_partitions;
+    const int64_t ctas = p.work_items != nullptr
+                             ? (int64_t)num_items
+                             : (int64_t)p.num_seqs * num_kv_heads * p.num_partitions;
     if (ctas >= (1ll << 31))
         return fail(PKV_ERR_UNSUPPORTED, "pkv_decode_attention: %lld CTAs", (long long)ctas);
     kern<<<(unsigned)ctas, kWarps * 32, smem, stream>>>(kmap, vmap, p);
@@ -993,18 +1022,20 @@ int launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap, const Decode
 
 template <typename T, int D, bool FP8>
 int dispatch_group(const CUtensorMap& kmap, const CUtensorMap& vmap, const DecodeParams& p,
-                   int num_kv_heads, cudaStream_t stream) {
+                   int num_kv_heads, int num_items, cudaStream_t stream) {
     // e4m3 caches take the tensor-core path for every group size: its
     // conversions are cheaper per tile than the GEMV's, and the tensor pipe
     // is otherwise idle (G = 1 uses one of the eight MMA columns)
     if constexpr (!FP8) {
         if (p.group == 1)
-            return launch_decode<T, D, GemvWarp<T, D>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+            return launch_decode<T, D, GemvWarp<T, D>, FP8>(kmap, vmap, p, num_kv_heads,
+                                                            num_items, stream);
     }
     if (p.group <= 8)
         return launch_decode<T, D, MmaWarp<T, D, 1, FP8>, FP8>(kmap, vmap, p, num_kv_heads,
-                                                               stream);
-    return launch_decode<T, D, MmaWarp<T, D, 2, FP8>, FP8>(kmap, vmap, p, num_kv_heads, stream);
+                                                               num_items, stream);
+    return launch_decode<T, D, MmaWarp<T, D, 2, FP8>, FP8>(kmap, vmap, p, num_kv_heads,
+                                                           num_items, stream);
 }
 
 // 4-D view of one e4m3 cache: (head_dim codes, kv head, slot, block), boxes
@@ -1051,8 +1082,8 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
                 const int32_t* context_lens, int num_seqs, int max_context_len, int num_q_heads,
                 int num_kv_heads, int head_dim, int num_blocks, int block_size,
                 int64_t block_stride, float scale, int partition_size, void* workspace,
-                size_t workspace_bytes, pkv_dtype dtype, int32_t* dev_error,
-                cudaStream_t stream) {
+                size_t workspace_bytes, const int32_t* work_items, int num_items,
+                pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_decode_attention: dtype %d", (int)dtype);
     PKV_REQUIRE(head_dim == 128 || (head_dim == 64 && !fp8), PKV_ERR_UNSUPPORTED,
@@ -1083,7 +1114,9 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
                 PKV_ERR_INVALID, "pkv_decode_attention: block_stride %lld",
                 (long long)block_stride);
     PKV_REQUIRE(num_kv_heads <= 65535, PKV_ERR_UNSUPPORTED, "too many KV heads");
-    if (num_seqs == 0) return PKV_OK;
+    PKV_REQUIRE(num_items >= 0, PKV_ERR_INVALID, "pkv_decode_attention_items: %d items",
+                num_items);
+    if (num_seqs == 0 || (work_items != nullptr && num_items == 0)) return PKV_OK;
     PKV_REQUIRE(out && query && key_cache && value_cache && context_lens &&
                     (block_tables || max_blocks_per_seq == 0),
                 PKV_ERR_INVALID, "pkv_decode_attention: NULL pointer");
@@ -1112,9 +1145,15 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     p.scale_log2 = scale * kLog2e;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.work_items = work_items;
     plan_partitions(max_context_len, partition_size, &p.partition_size, &p.num_partitions);
     PKV_REQUIRE(p.num_partitions <= 65535, PKV_ERR_UNSUPPORTED,
                 "pkv_decode_attention: %d partitions (max 65535)", p.num_partitions);
+    PKV_REQUIRE(work_items == nullptr ||
+                    (int64_t)num_items <= (int64_t)num_seqs * num_kv_heads * p.num_partitions,
+                PKV_ERR_INVALID,
+                "pkv_decode_attention_items: %d items for a grid of %lld", num_items,
+                (long long)num_seqs * num_kv_heads * p.num_partitions);
     if (p.num_partitions > 1) {
         WorkspaceLayout w = workspace_layout(num_seqs, num_q_heads, p.num_partitions, head_dim);
         PKV_REQUIRE(workspace != nullptr && workspace_bytes >= w.total && aligned16(workspace),
@@ -1141,18 +1180,22 @@ int decode_impl(void* out, const void* query, const void* key_cache, const void*
     if (st != PKV_OK) return st;
 
     DeviceGuard guard(stream, key_cache);
+    const int n = num_items;
     if (fp8) {
         return dtype == PKV_BF16
-                   ? dispatch_group<__nv_bfloat16, 128, true>(kmap, vmap, p, num_kv_heads, stream)
-                   : dispatch_group<__half, 128, true>(kmap, vmap, p, num_kv_heads, stream);
+                   ? dispatch_group<__nv_bfloat16, 128, true>(kmap, vmap, p, num_kv_heads, n, stream)
+                   : dispatch_group<__half, 128, true>(kmap, vmap, p, num_kv_heads, n, stream);
     }
     if (dtype == PKV_BF16) {
         return head_dim == 128
-                   ? dispatch_group<__nv_bfloat16, 128, false>(kmap, vmap, p, num_kv_heads, stream)
-                   : dispatch_group<__nv_bfloat16, 64, false>(kmap, vmap, p, num_kv_heads, stream);
+                   ? dispatch_group<__nv_bfloat16, 128, false>(kmap, vmap, p, num_kv_heads, n,
+                                                               stream)
+                   : dispatch_group<__nv_bfloat16, 64, false>(kmap, vmap, p, num_kv_heads, n,
+                                                              stream);
     }
-    return head_dim == 128 ? dispatch_group<__half, 128, false>(kmap, vmap, p, num_kv_heads, stream)
-                           : dispatch_group<__half, 64, false>(kmap, vmap, p, num_kv_heads, stream);
+    return head_dim == 128
+               ? dispatch_group<__half, 128, false>(kmap, vmap, p, num_kv_heads, n, stream)
+               : dispatch_group<__half, 64, false>(kmap, vmap, p, num_kv_heads, n, stream);
 }
 
 }  // namespace
@@ -1166,11 +1209,12 @@ extern "C" int pkv_decode_attention(void* out, const void* query, const void* ke
                                     int block_size, int64_t block_stride, float scale,
                                     int partition_size, void* workspace, size_t workspace_bytes,
                                     pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_decode_attention");
     return pkv::decode_impl(out, query, key_cache, value_cache, nullptr, nullptr, false,
                             block_tables, max_blocks_per_seq, context_lens, num_seqs,
                             max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
                             block_size, block_stride, scale, partition_size, workspace,
-                            workspace_bytes, dtype, dev_error, stream);
+                            workspace_bytes, nullptr, 0, dtype, dev_error, stream);
 }
 
 extern "C" int pkv_decode_attention_fp8(void* out, const void* query, const void* key_cache,
@@ -1183,9 +1227,118 @@ extern "C" int pkv_decode_attention_fp8(void* out, const void* query, const void
                                         int partition_size, void* workspace,
                                         size_t workspace_bytes, pkv_dtype dtype,
                                         int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_decode_attention_fp8");
     return pkv::decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, true,
                             block_tables, max_blocks_per_seq, context_lens, num_seqs,
                             max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
                             block_size, block_stride, scale, partition_size, workspace,
-                            workspace_bytes, dtype, dev_error, stream);
+                            workspace_bytes, nullptr, 0, dtype, dev_error, stream);
+}
+
+extern "C" int pkv_decode_attention_items(void* out, const void* query, const void* key_cache,
+                                          const void* value_cache, const int32_t* block_tables,
+                                          int max_blocks_per_seq, const int32_t* context_lens,
+                                          int num_seqs, int max_context_len, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int num_blocks,
+                                          int block_size, int64_t block_stride, float scale,
+                                          int partition_size, void* workspace,
+                                          size_t workspace_bytes, const int32_t* work_items,
+                                          int num_items, pkv_dtype dtype, int32_t* dev_error,
+                                          cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_decode_attention_items");
+    PKV_REQUIRE(work_items != nullptr || num_items == 0, PKV_ERR_INVALID,
+                "pkv_decode_attention_items: NULL work list");
+    if (num_items == 0) return PKV_OK;
+    return pkv::decode_impl(out, query, key_cache, value_cache, nullptr, nullptr, false,
+                            block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                            block_size, block_stride, scale, partition_size, workspace,
+                            workspace_bytes, work_items, num_items, dtype, dev_error, stream);
+}
+
+extern "C" int pkv_decode_attention_fp8_items(
+    void* out, const void* query, const void* key_cache, const void* value_cache,
+    const float* k_scale, const float* v_scale, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int max_context_len,
+    int num_q_heads, int num_kv_heads, int head_dim, int num_blocks, int block_size,
+    int64_t block_stride, float scale, int partition_size, void* workspace,
+    size_t workspace_bytes, const int32_t* work_items, int num_items, pkv_dtype dtype,
+    int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_decode_attention_fp8_items");
+    PKV_REQUIRE(work_items != nullptr || num_items == 0, PKV_ERR_INVALID,
+                "pkv_decode_attention_fp8_items: NULL work list");
+    if (num_items == 0) return PKV_OK;
+    return pkv::decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, true,
+                            block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                            block_size, block_stride, scale, partition_size, workspace,
+                            workspace_bytes, work_items, num_items, dtype, dev_error, stream);
+}
+
+// The decode work list ("PagedAttention 动态内存分页" page, 技术边界与取舍: a
+// batch of very uneven lengths is what costs).  Items are the (sequence, KV
+// head, partition) triples that hold tokens; longest first, a counting sort
+// on the number of 16-token tiles each holds orders them largest first,
+// keeping grid order among equals, in O(items + P / 16).
+extern "C" int pkv_decode_work_items(const int32_t* context_lens, int num_seqs,
+                                     int num_kv_heads, int max_context_len, int partition_size,
+                                     int order, int32_t* items, int capacity, int* num_items) {
+    using namespace pkv;
+    PKV_REQUIRE(num_items != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL count");
+    *num_items = 0;
+    PKV_REQUIRE(num_seqs >= 0 && num_kv_heads > 0 && max_context_len >= 0 && capacity >= 0,
+                PKV_ERR_INVALID, "pkv_decode_work_items: bad sizes");
+    PKV_REQUIRE(partition_size >= 0 && partition_size % kTile == 0, PKV_ERR_INVALID,
+                "pkv_decode_work_items: partition_size %d is not a multiple of 16",
+                partition_size);
+    PKV_REQUIRE(order == PKV_ITEMS_LONGEST_FIRST || order == PKV_ITEMS_GRID, PKV_ERR_INVALID,
+                "pkv_decode_work_items: order %d", order);
+    if (num_seqs == 0) return PKV_OK;
+    PKV_REQUIRE(context_lens != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL lengths");
+    int P, NP;
+    plan_partitions(max_context_len, partition_size, &P, &NP);
+    PKV_REQUIRE((int64_t)num_seqs * num_kv_heads * NP < (1ll << 31), PKV_ERR_UNSUPPORTED,
+                "pkv_decode_work_items: grid too large");
+    const int nbuckets = P / kTile + 1;  // tiles per item: 0 .. P / 16
+    std::vector<int64_t> count(nbuckets + 1, 0);
+    int64_t total = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int L = context_lens[s];
+        PKV_REQUIRE(L >= 0 && L <= max_context_len, PKV_ERR_INVALID,
+                    "pkv_decode_work_items: context_lens[%d] = %d outside [0, %d]", s, L,
+                    max_context_len);
+        const int np = L > 0 ? (L + P - 1) / P : 1;
+        // full partitions, then the last one's tiles (0 for an empty context)
+        const int last = L - (np - 1) * P;
+        count[P / kTile] += (int64_t)(np - 1) * num_kv_heads;
+        count[(last + kTile - 1) / kTile] += num_kv_heads;
+        total += (int64_t)np * num_kv_heads;
+    }
+    *num_items = (int)total;
+    PKV_REQUIRE(total <= capacity, PKV_ERR_INVALID,
+                "pkv_decode_work_items: %lld items, capacity %d", (long long)total, capacity);
+    PKV_REQUIRE(items != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL items");
+    // start offset of each bucket, the largest bucket first; in grid order
+    // every item goes to one bucket, in the order of the loop below
+    std::vector<int64_t> start(nbuckets, 0);
+    int64_t at = 0;
+    for (int b = nbuckets - 1; b >= 0; --b) {
+        start[b] = at;
+        at += count[b];
+    }
+    const bool grid_order = order == PKV_ITEMS_GRID;
+    if (grid_order) start[0] = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int L = context_lens[s];
+        const int np = L > 0 ? (L + P - 1) / P : 1;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            const int64_t base = ((int64_t)s * num_kv_heads + h) * NP;
+            for (int part = 0; part < np; ++part) {
+                const int tok = std::min(P, L - part * P);
+                const int b = grid_order ? 0 : (tok + kTile - 1) / kTile;
+                items[start[b]++] = (int32_t)(base + part);
+            }
+        }
+    }
+    return PKV_OK;
 }

@@ -165,6 +165,7 @@ extern "C" int pkv_seq_append(pkv_pool* pool, int64_t seq_id, int64_t* slot,
 extern "C" int pkv_seq_append_batch(pkv_pool* pool, int n, const int64_t* seq_ids,
                                     int64_t* slots, int32_t* cow_pairs,
                                     int* num_cow, int* num_done) {
+    PKV_NVTX_RANGE("pkv_seq_append_batch");
     PKV_REQUIRE(pool && n >= 0 && (n == 0 || (seq_ids && slots && cow_pairs)) && num_cow,
                 PKV_ERR_INVALID, "pkv_seq_append_batch: bad argument");
     *num_cow = 0;

@@ -97,12 +97,27 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Cache policy of the L2: the streaming Q reads and output writes are
+// evicted first, so that the K/V of the sequences in flight, which every
+// row tile of a sequence re-reads, stay in L2 (PKV_PREFILL_L2_HINTS 0: no
+// hints).
+#ifndef PKV_PREFILL_L2_HINTS
+#define PKV_PREFILL_L2_HINTS 1
+#endif
+constexpr bool kL2Hints = PKV_PREFILL_L2_HINTS != 0;
+
 // 16-byte copy global -> shared that does not wait (cp.async, L2 only);
 // when copy is false, the destination is zero-filled and nothing is read
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, bool copy) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
-                 "l"(src), "r"(copy ? 16 : 0)
-                 : "memory");
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src, bool copy,
+                                            uint64_t policy) {
+    if constexpr (kL2Hints)
+        asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
+                     ::"r"(smem_addr(dst)), "l"(src), "r"(copy ? 16 : 0), "l"(policy)
+                     : "memory");
+    else
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
+                     "l"(src), "r"(copy ? 16 : 0)
+                     : "memory");
 }
 
 // waits for every cp.async this thread issued
@@ -180,6 +195,7 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
     constexpr int kBoxes = kKeys / kBoxKeys;       // TMA boxes per key tile and 64-dim half
     constexpr int kWindowTiles = 32 / kBoxes;      // key tiles per warp-wide block-id load
     const int bs = p.block_size;
+    const uint64_t keep = l2_policy_evict_last();  // K/V: re-read by later row tiles
     int gk = 0;  // key tiles issued over all items
     for (int k = 0; !*failed; ++k) {
         const int idx = item_index(k);
@@ -217,10 +233,19 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
                     const int off = key0 < it.L ? key0 % bs : 0;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap,
-                                    &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
-                        tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap,
-                                    &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
+                        if constexpr (kL2Hints) {
+                            tma_load_5d_hint(kdst + h * kHalfBytes + bx * kBoxKeys * 128,
+                                             &kmap, &b.kv_full[st], 0, it.kvh, off, h, phys[bx],
+                                             keep);
+                            tma_load_5d_hint(vdst + h * kHalfBytes + bx * kBoxKeys * 128,
+                                             &vmap, &b.kv_full[st], 0, it.kvh, off, h, phys[bx],
+                                             keep);
+                        } else {
+                            tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap,
+                                        &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
+                            tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap,
+                                        &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
+                        }
                     }
                 }
             }
@@ -368,6 +393,7 @@ __device__ void stage_q(const PrefillParams& p, const Bars& b, uint8_t* qsm, int
     const T* qbase = static_cast<const T*>(p.query);
     const int G = p.group, Hq = p.num_q_heads;
     const int ch = lane & 15;
+    const uint64_t stream_once = l2_policy_evict_first();  // Q is read once
     int nk = 0;
     for (int k = 0; !*failed; ++k) {
         const int idx = item_index(k);
@@ -387,7 +413,7 @@ __device__ void stage_q(const PrefillParams& p, const Bars& b, uint8_t* qsm, int
                                     (in ? g : 0)) * kD + ch * 8;
             cp_async_16(qsm + (r / kRows) * kQTileBytes + (ch >> 3) * kQHalfBytes +
                             swz(r % kRows, ch),
-                        src, in);
+                        src, in, stream_once);
             g += 2;  // next row of this lane: two rows on
             while (g >= G) {
                 g -= G;
@@ -539,6 +565,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         T* dst = static_cast<T*>(p.out) +
                  ((int64_t)(it.q0 + tok) * p.num_q_heads + it.kvh * p.group + gh) * kD;
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        const uint64_t write_once = l2_policy_evict_first();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
@@ -551,9 +578,15 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                                                 __uint_as_float(o[2 * e + 1]) * inv);
             if (ok) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    reinterpret_cast<uint4*>(dst + 32 * c)[v] =
-                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 w = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                               pk[4 * v + 3]);
+                    if constexpr (kL2Hints)
+                        st_global_v4_hint(reinterpret_cast<uint4*>(dst + 32 * c) + v, w,
+                                          write_once);
+                    else
+                        reinterpret_cast<uint4*>(dst + 32 * c)[v] = w;
+                }
             }
         }
         // O has been read: the next item's first P V may overwrite it
@@ -646,6 +679,7 @@ extern "C" int pkv_prefill_attention(void* out, const void* query, const void* k
                                      int head_dim, int num_blocks, int block_size,
                                      int64_t block_stride, float scale, pkv_dtype dtype,
                                      int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_prefill_attention");
     using namespace pkv;
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_prefill_attention: dtype %d", (int)dtype);

@@ -1,6 +1,9 @@
 // status.cpp — status strings, the thread-local last-error message, sizing.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "internal.h"
 
@@ -17,6 +20,22 @@ int fail(int status, const char* fmt, ...) {
 }
 
 void clear_error() { g_last_error[0] = '\0'; }
+
+static bool nvtx_enabled() {
+    static const bool on = [] {
+        const char* v = std::getenv("PKV_NVTX");
+        return v != nullptr && std::strcmp(v, "1") == 0;
+    }();
+    return on;
+}
+
+NvtxRange::NvtxRange(const char* name) : on_(nvtx_enabled()) {
+    if (on_) nvtxRangePushA(name);
+}
+
+NvtxRange::~NvtxRange() {
+    if (on_) nvtxRangePop();
+}
 
 }  // namespace pkv
 

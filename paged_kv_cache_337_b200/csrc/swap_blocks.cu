@@ -101,6 +101,7 @@ extern "C" int pkv_swap_blocks(const void* src_key, const void* src_value, void*
                                int src_num_blocks, int dst_num_blocks, int64_t block_bytes,
                                int64_t src_block_stride, int64_t dst_block_stride,
                                int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_swap_blocks");
     using namespace pkv;
     PKV_REQUIRE(num_pairs >= 0 && src_num_blocks >= 0 && dst_num_blocks >= 0 &&
                     block_bytes > 0 && block_bytes % 4 == 0,

@@ -54,6 +54,7 @@ extern "C" int pkv_write_slots(const void* key, const void* value, void* key_cac
                                int num_tokens, int num_blocks, int block_size,
                                int num_kv_heads, int head_dim, int64_t block_stride,
                                pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_write_slots");
     using namespace pkv;
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_write_slots: dtype %d", (int)dtype);
@@ -147,6 +148,7 @@ extern "C" int pkv_write_slots_fp8(const void* key, const void* value, void* key
                                    int num_tokens, int num_blocks, int block_size,
                                    int num_kv_heads, int head_dim, int64_t block_stride,
                                    pkv_dtype dtype, int32_t* dev_error, cudaStream_t stream) {
+    PKV_NVTX_RANGE("pkv_write_slots_fp8");
     using namespace pkv;
     PKV_REQUIRE(dtype == PKV_F16 || dtype == PKV_BF16, PKV_ERR_UNSUPPORTED,
                 "pkv_write_slots_fp8: dtype %d of the new rows", (int)dtype);
