@@ -19,13 +19,22 @@ and outputs keep the workload's 16-bit type.
 
 `value` is effective GB/s of algorithmic bytes (every context token's K and V
 read once, plus queries, outputs, table rows, the slot write and any
-workspace traffic) over device time, with all inputs resident in HBM.  `e2e`
-is the same metric through the public step API from pinned host buffers,
-host allocator and copies included.  Under torchrun each rank runs its own
+workspace traffic) over device time, with all inputs resident in HBM; the
+host pool's slot appends for the timed steps are made before timing.  `e2e`
+is the same metric through the public step API (PagedKVCache) from pinned
+host buffers, host pool and copies included, with the host time of each part
+and the loop's mode.  `allocator` is the host pool's append latency.  With
+the default workload the line also carries `workloads`: the 70B-shaped GQA
+batch, the long split-K contexts at block sizes 32 and 64, both decode
+shapes over e4m3 caches, the shared-prefix fork and steady steps and paged
+prefill, each timed the same way in the same process.  `clocks` holds the
+SM clock and clock-event reasons sampled every millisecond, from the
+samples inside the timed region.  Under torchrun each rank runs its own
 batch (weak scaling, no collective on the data path) and the time is the
 maximum over ranks.
 """
 import argparse
+import gc
 import json
 import math
 import os
@@ -71,11 +80,15 @@ def parse_args():
                     help="profiling only: run the workload's first N sequences")
     ap.add_argument("--kv-dtype", choices=["auto", "fp8"], default="auto",
                     help="fp8: e4m3 cache with a scale per (block, KV head)")
-    ap.add_argument("--work-list", choices=["longest_first", "grid", "none"],
-                    default="longest_first",
-                    help="decode over the library's work list (items longest first, or in "
-                         "grid order) or over the full grid (none)")
+    ap.add_argument("--work-list", default="auto",
+                    choices=["auto", "longest_first", "sequences_longest_first", "batch_order",
+                             "none"],
+                    help="the decode grid: PagedKVCache's work_list (auto: the full grid for "
+                         "one pass, a work list with split-K)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-mode", choices=["serial", "pipelined"], default="pipelined",
+                    help="e2e loop: wait for each step's output before enqueueing the next "
+                         "(serial) or after (pipelined)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra", choices=["all", "none"], default="all",
                     help="with the default workload: also measure the other decode "
@@ -456,7 +469,23 @@ def run_reference(args, spec, world, rank):
 # the product arm
 # ---------------------------------------------------------------------------
 def cache_work_list(args):
-    return {"none": False, "longest_first": "longest_first", "grid": "grid"}[args.work_list]
+    return False if args.work_list == "none" else args.work_list
+
+
+def grid_label(args, P, max_len, fp8):
+    """What the decode launch runs over, as PagedKVCache's work_list picks
+    it for this workload."""
+    wl = args.work_list
+    if wl == "auto":
+        if not 0 < P < max_len:
+            return "full grid (one pass per sequence)"
+        wl = "longest_first" if fp8 else "sequences_longest_first"
+    if wl == "none":
+        return "full grid"
+    return "work list of the (sequence, KV head, partition) items holding tokens, " + {
+        "longest_first": "longest first",
+        "sequences_longest_first": "sequences longest first",
+        "batch_order": "sequences in batch order"}[wl]
 
 
 def allocator_latency(spec, lens, order, rank):
@@ -495,6 +524,106 @@ def allocator_latency(spec, lens, order, rank):
             "batches_timed": rounds, "singles_timed": singles,
             "what": "host pool, Python binding included: one slot per sequence, a new block "
                     "from the pool when the last one is full"}
+
+
+def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
+    """The decode step end to end through the public step API, from pinned
+    host memory.  Per step: the step's q, k and v go up in one copy from
+    pinned memory (on a second stream, into one of two input buffers), the
+    host pool reserves the slots and plans the work list
+    (PagedKVCache.prepare_step), the metadata goes up in one copy
+    (upload_step), the kernels run (launch_step), and the attention output
+    comes back to pinned host memory; the host waits for it.
+
+    serial: the host waits for step i's output before it enqueues step i+1
+    (the pool's work for step i+1 and its input upload still overlap step
+    i on the GPU).  pipelined: step i+1 is enqueued before the host waits
+    for step i's output (two output buffers), so the GPU goes from step to
+    step without waiting for the host.  Returns the e2e record with the
+    host time of each part."""
+    S, Hq, Hkv, D = spec.num_seqs, spec.num_q_heads, spec.num_kv_heads, spec.head_dim
+    dt = spec.torch_dtype
+    pipelined = args.e2e_mode == "pipelined"
+    nq, nk = S * Hq * D, S * Hkv * D
+    h_in = [torch.randn(nq + 2 * nk).to(dt).pin_memory() for _ in range(2)]
+    d_in = [torch.empty(nq + 2 * nk, dtype=dt, device=dev) for _ in range(2)]
+    views = [(b[:nq].view(S, Hq, D), b[nq:nq + nk].view(S, Hkv, D),
+              b[nq + nk:].view(S, Hkv, D)) for b in d_in]
+    nout = 2 if pipelined else 1
+    outs = [torch.empty((S, Hq, D), dtype=dt, device=dev) for _ in range(nout)]
+    houts = [torch.empty((S, Hq, D), dtype=dt).pin_memory() for _ in range(nout)]
+    copy_stream = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b done
+    ev_out = [torch.cuda.Event() for _ in range(nout)]  # a step's result on the host
+    e2e_bytes = h2d = d2h = 0
+    host = {"prepare": 0.0, "enqueue": 0.0, "input_upload_enqueue": 0.0, "wait": 0.0}
+
+    def timed(key, fn, *a):
+        t = time.perf_counter()
+        r = fn(*a)
+        host[key] += time.perf_counter() - t
+        return r
+
+    def enqueue(i, prep):
+        b, o = i % 2, i % nout
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[b])
+            cache.upload_step(prep, stream)
+            dq, dk, dv = views[b]
+            cache.launch_step(prep, dq, dk, dv, outs[o], stream=stream)
+            ev_used[b].record(stream)
+            houts[o].copy_(outs[o], non_blocking=True)
+            ev_out[o].record(stream)
+
+    def upload_inputs(i):
+        b = i % 2
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(ev_used[b])  # step i - 2 done with the buffer
+            d_in[b].copy_(h_in[i % 2], non_blocking=True)
+            ev_in[b].record(copy_stream)
+
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    # Python's collector runs before the timed loop, not inside it: a full
+    # collection over this process's heap pauses the host for milliseconds
+    gc.collect()
+    gc.disable()
+    t0 = time.perf_counter()
+    timed("input_upload_enqueue", upload_inputs, 0)
+    prep = timed("prepare", cache.prepare_step, ids)
+    for i in range(steps):
+        timed("enqueue", enqueue, i, prep)
+        lens = prep["st"]["h_lens"].tolist()
+        e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
+                      copy_bytes(spec, prep["num_pairs"], fp8))
+        used = prep["st"]["items_off"] + max(prep["num_items"], 0)
+        h2d = d_in[i % 2].numel() * 2 + used * 4
+        d2h = houts[0].numel() * 2
+        if pipelined and i >= 1:
+            timed("wait", ev_out[(i - 1) % nout].synchronize)  # step i - 1's result
+        if i + 1 < steps:
+            timed("input_upload_enqueue", upload_inputs, i + 1)
+            prep = timed("prepare", cache.prepare_step, ids)  # overlaps step i on the GPU
+        if not pipelined:
+            timed("wait", ev_out[0].synchronize)
+    if pipelined:
+        timed("wait", ev_out[(steps - 1) % nout].synchronize)
+    e2e_s = time.perf_counter() - t0
+    gc.enable()
+    barrier(world)
+    e2e_s = max_over_ranks(e2e_s, world, dev)
+    e2e_total = sum_over_ranks(e2e_bytes, world, dev)
+    return {"value": round(e2e_total / e2e_s / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps, "ms_per_step": round(1e3 * e2e_s / steps, 4), "mode": args.e2e_mode,
+            "python_gc": "collected before the timed loop, paused during it",
+            "host_ms_per_step": {
+                "pool_append_tables_and_work_list": round(1e3 * host["prepare"] / steps, 4),
+                "metadata_upload_and_launches": round(1e3 * host["enqueue"] / steps, 4),
+                "input_upload_enqueue": round(1e3 * host["input_upload_enqueue"] / steps, 4),
+                "readback_wait": round(1e3 * host["wait"] / steps, 4)}}
 
 
 def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc=True):
@@ -637,83 +766,10 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
     tok_s = world * S * K / (t_max * 1e-3)
 
     # ---- end to end through the public step API from pinned host memory ----
-    # Per step: the step's q, k and v go up in one copy from pinned memory,
-    # the host pool reserves the slots and the metadata goes up in one copy,
-    # the kernels run, and the attention output comes back to the host; the
-    # host waits for it before the step ends.  The pool's work and the input
-    # upload for step i+1 (on a second stream, into the other of two input
-    # buffers) run while step i is on the GPU: neither depends on step i's
-    # output.  The host time of each part is recorded.
     e2e = None
     if e2e_steps:
-        nq, nk = S * Hq * D, S * Hkv * D
-        h_in = [torch.randn(nq + 2 * nk).to(dt).pin_memory() for _ in range(2)]
-        d_in = [torch.empty(nq + 2 * nk, dtype=dt, device=dev) for _ in range(2)]
-        views = [(b[:nq].view(S, Hq, D), b[nq:nq + nk].view(S, Hkv, D),
-                  b[nq + nk:].view(S, Hkv, D)) for b in d_in]
-        hout = torch.empty((S, Hq, D), dtype=dt).pin_memory()
-        copy_stream = torch.cuda.Stream(dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
-        ev_used = [torch.cuda.Event() for _ in range(2)]  # step using buffer b done
-        ev_out = torch.cuda.Event()                       # step result on the host
-        e2e_bytes = 0
-        h2d = d2h = 0
-        host = {"prepare": 0.0, "enqueue": 0.0, "input_upload_enqueue": 0.0, "wait": 0.0}
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        t0 = time.perf_counter()
-        with torch.cuda.stream(copy_stream):
-            d_in[0].copy_(h_in[0], non_blocking=True)
-            ev_in[0].record(copy_stream)
-        prep = cache.prepare_step(ids)
-        host["prepare"] += time.perf_counter() - t0
-        for i in range(e2e_steps):
-            b = i % 2
-            ta = time.perf_counter()
-            with torch.cuda.stream(stream):
-                stream.wait_event(ev_in[b])
-                cache.upload_step(prep, stream)
-                dq, dk, dv = views[b]
-                cache.launch_step(prep, dq, dk, dv, out, stream=stream)
-                ev_used[b].record(stream)
-                hout.copy_(out, non_blocking=True)
-                ev_out.record(stream)
-            tb = time.perf_counter()
-            host["enqueue"] += tb - ta
-            lens = prep["st"]["h_lens"].tolist()
-            e2e_bytes += (decode_bytes(spec, lens, P, fp8) + write_bytes(spec, S, fp8) +
-                          copy_bytes(spec, prep["num_pairs"], fp8))
-            h2d = d_in[b].numel() * 2 + prep["st"]["h"].numel() * 4
-            d2h = hout.numel() * 2
-            tc = time.perf_counter()
-            if i + 1 < e2e_steps:
-                nb_ = 1 - b
-                with torch.cuda.stream(copy_stream):
-                    if i >= 1:
-                        copy_stream.wait_event(ev_used[nb_])  # step i-1 done with it
-                    d_in[nb_].copy_(h_in[(i + 1) % 2], non_blocking=True)
-                    ev_in[nb_].record(copy_stream)
-                td = time.perf_counter()
-                host["input_upload_enqueue"] += td - tc
-                prep = cache.prepare_step(ids)  # overlaps the GPU work of step i
-                tc = time.perf_counter()
-                host["prepare"] += tc - td
-            ev_out.synchronize()
-            host["wait"] += time.perf_counter() - tc
-        e2e_s = time.perf_counter() - t0
-        barrier(world)
-        e2e_s = max_over_ranks(e2e_s, world, dev)
-        e2e_total = sum_over_ranks(e2e_bytes, world, dev)
-        e2e = {"value": round(e2e_total / e2e_s / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": e2e_steps, "ms_per_step": round(1e3 * e2e_s / e2e_steps, 4),
-               "host_ms_per_step": {
-                   "pool_append_and_tables": round(1e3 * host["prepare"] / e2e_steps, 4),
-                   "metadata_upload_and_launches": round(1e3 * host["enqueue"] / e2e_steps, 4),
-                   "input_upload_enqueue": round(
-                       1e3 * host["input_upload_enqueue"] / e2e_steps, 4),
-                   "readback_wait": round(1e3 * host["wait"] / e2e_steps, 4)},
-               "device_ms_per_step": round(ms_per_step, 4)}
+        e2e = run_e2e(args, spec, cache, ids, e2e_steps, stream, P, fp8, world, dev)
+        e2e["device_ms_per_step"] = round(ms_per_step, 4)
         cache.check_errors()
 
     cpu = None
@@ -738,10 +794,7 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
             "num_kv_heads": Hkv, "head_dim": D, "block_size": bs,
             "context_lens": "U[%d,%d]" % (spec.len_lo, spec.len_hi),
             "pool_blocks": nb, "partition_size": P,
-            "grid": {"none": "full grid", "longest_first": "work list: (sequence, KV head, "
-                     "partition) items holding tokens, longest first",
-                     "grid": "work list: (sequence, KV head, partition) items holding tokens, "
-                     "in grid order"}[args.work_list],
+            "grid": grid_label(args, P, max_len_all, fp8),
             "kv_cache": ("e4m3, fp32 scale per (block, KV head)" if fp8 else
                          "bf16" if dt == torch.bfloat16 else "f16"),
             "step": "slot write + paged decode attention (+ copy-on-write copies; split-K "

@@ -210,14 +210,21 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
  * end exit at once, in grid order.  This host-side planner lists instead
  * the work items that hold tokens: one per (sequence s, KV head, partition
  * p) with p < max(1, ceil(L_s / P)), so a short sequence runs one pass and
- * a long one is split.  order:
+ * a long one is split.  Within a sequence the items go partition by
+ * partition, the KV heads of a partition side by side (their slices of a
+ * block share its memory rows).  order:
  *   PKV_ITEMS_LONGEST_FIRST  by the 16-token tiles each item holds, most
- *                            first (ties in grid order): the long items
- *                            start first and the short ones fill the end
- *                            of the launch
- *   PKV_ITEMS_GRID           grid order (the empty slots left out): the
- *                            items of one sequence, and of sequences next
- *                            to each other in the batch, run side by side
+ *                            first (ties as above, sequences in batch
+ *                            order): the long items start first and the
+ *                            short ones fill the end of the launch
+ *   PKV_ITEMS_SEQUENCES_LONGEST_FIRST
+ *                            sequences by context length, longest first
+ *                            (ties in batch order), each sequence's items
+ *                            together
+ *   PKV_ITEMS_BATCH_ORDER    sequences in batch order, each sequence's
+ *                            items together (sequences next to each other
+ *                            in the batch, such as samples sharing a
+ *                            prefix, run side by side)
  *
  *   context_lens     HOST int32 [num_seqs]: the same lengths the device
  *                    copy passed to the attention call holds
@@ -232,11 +239,12 @@ PKV_API int pkv_decode_attention(void* out, const void* query, const void* key_c
  *                    num_kv_heads * sum_s max(1, ceil(L_s / P)) is the count
  *                    and num_seqs * num_kv_heads * NP always suffices.
  * A length outside [0, max_context_len] or an unknown order returns
- * PKV_ERR_INVALID.  O(items + P / 16): a counting sort on the host, no
- * device work.
+ * PKV_ERR_INVALID.  Host work only: O(items + P / 16), plus a sort of the
+ * sequences for PKV_ITEMS_SEQUENCES_LONGEST_FIRST.
  */
 #define PKV_ITEMS_LONGEST_FIRST 0
-#define PKV_ITEMS_GRID 1
+#define PKV_ITEMS_SEQUENCES_LONGEST_FIRST 1
+#define PKV_ITEMS_BATCH_ORDER 2
 PKV_API int pkv_decode_work_items(const int32_t* context_lens, int num_seqs, int num_kv_heads,
                                   int max_context_len, int partition_size, int order,
                                   int32_t* items, int capacity, int* num_items);

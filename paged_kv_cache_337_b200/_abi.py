@@ -31,7 +31,8 @@ PKV_DEVERR_TIMEOUT = 5
 PKV_DEVERR_WORK_ITEM = 6
 
 PKV_ITEMS_LONGEST_FIRST = 0
-PKV_ITEMS_GRID = 1
+PKV_ITEMS_SEQUENCES_LONGEST_FIRST = 1
+PKV_ITEMS_BATCH_ORDER = 2
 
 PKV_NOALLOC_WORKSPACE_BYTES = 64 << 20
 
@@ -259,9 +260,8 @@ def pkv_decode_work_items(context_lens, num_kv_heads, max_context_len, partition
                           out=None, order=PKV_ITEMS_LONGEST_FIRST):
     """The decode work list for these lengths (a host int32 tensor or
     sequence): every (sequence, KV head, partition) that holds tokens, as
-    flat grid indices, the items holding the most tokens first
-    (PKV_ITEMS_LONGEST_FIRST) or in grid order (PKV_ITEMS_GRID).  Returns an
-    int32 CPU tensor (a view of `out` when given, e.g. pinned staging)."""
+    flat grid indices, in one of the PKV_ITEMS_* orders.  Returns an int32
+    CPU tensor (a view of `out` when given, e.g. pinned staging)."""
     lens = torch.as_tensor(context_lens, dtype=torch.int32)
     if lens.device.type != "cpu":
         raise ValueError("pkv_decode_work_items: context_lens must be on the host")

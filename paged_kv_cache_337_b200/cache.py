@@ -17,12 +17,13 @@ block) the three device calls are their ``_fp8`` forms, which also copy and
 read the per-(block, KV head) scales.
 
 Steps 2-4 are launched on one stream; the metadata of step 1 travels to the
-device through pinned host staging buffers.  With ``work_list`` (the
-default) step 1 also asks the library for the decode work list
-(``pkv_decode_work_items``: every (sequence, KV head, partition) holding
-tokens, the longest first or in grid order) and step 4 runs over it
-(``pkv_decode_attention_items``).  All arithmetic is in the library; this
-module only moves arguments.
+device through pinned host staging buffers.  When the step splits
+sequences into partitions, step 1 also asks the library for the decode work
+list (``pkv_decode_work_items``: every (sequence, KV head, partition)
+holding tokens, in the order ``work_list`` picks) and step 4 runs over it
+(``pkv_decode_attention_items``) instead of the full grid, whose slots past
+the shorter sequences' ends would launch and exit.  All arithmetic is in
+the library; this module only moves arguments.
 
 ``upload_step`` and ``launch_step`` may run on different streams: the
 launch waits for the upload's event, and the next upload into the same
@@ -37,15 +38,20 @@ class PagedKVCache:
     def __init__(self, num_blocks, block_size, num_q_heads, num_kv_heads, head_dim, dtype,
                  device, max_blocks_per_seq, partition_size=0, free_order=None,
                  key_cache=None, value_cache=None, scale=None, kv_dtype=None, kv_scale=1.0,
-                 work_list=True):
+                 work_list="auto"):
         """dtype is the type of queries, new K/V rows and outputs (f16 or
         bf16).  kv_dtype torch.uint8 (or torch.float8_e4m3fn) stores the
         cache as e4m3 codes with a scale per (block, KV head) in k_scale /
         v_scale ([num_blocks, num_kv_heads] fp32, every entry kv_scale until
-        the caller sets them); None stores it in dtype.  work_list: decode
-        over the library's work list instead of the full grid, its items
-        longest first (True or "longest_first") or in grid order ("grid");
-        False: the full grid."""
+        the caller sets them); None stores it in dtype.
+
+        work_list: the decode grid.  "auto" (or True): the full grid when
+        every sequence fits one partition, else the library's work list,
+        items longest first for an e4m3 cache and sequences longest first
+        for a 16-bit cache (the orders measured fastest on B200 for the
+        GQA and long-context batches); "longest_first",
+        "sequences_longest_first", "batch_order": the work list in that
+        order on every step; False or "none": the full grid."""
         self.num_blocks = num_blocks
         self.block_size = block_size
         self.num_q_heads = num_q_heads
@@ -55,12 +61,18 @@ class PagedKVCache:
         self.device = torch.device(device)
         self.max_blocks_per_seq = max_blocks_per_seq
         self.partition_size = partition_size
-        orders = {True: _abi.PKV_ITEMS_LONGEST_FIRST,
-                  "longest_first": _abi.PKV_ITEMS_LONGEST_FIRST, "grid": _abi.PKV_ITEMS_GRID}
-        if work_list is not False and work_list not in orders:
-            raise ValueError("work_list must be True, False, 'longest_first' or 'grid'")
-        self.work_list = work_list is not False
-        self._item_order = orders.get(work_list, _abi.PKV_ITEMS_LONGEST_FIRST)
+        orders = {"longest_first": _abi.PKV_ITEMS_LONGEST_FIRST,
+                  "sequences_longest_first": _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST,
+                  "batch_order": _abi.PKV_ITEMS_BATCH_ORDER}
+        if work_list is True:
+            work_list = "auto"
+        if work_list in (False, "none"):
+            work_list = None
+        if work_list is not None and work_list != "auto" and work_list not in orders:
+            raise ValueError("work_list must be 'auto', 'longest_first', "
+                             "'sequences_longest_first', 'batch_order' or False")
+        self.work_list = work_list is not None
+        self._item_order = orders.get(work_list)  # None: "auto"
         self.scale = scale if scale is not None else 1.0 / (head_dim ** 0.5)
         shape = (num_blocks, block_size, num_kv_heads, head_dim)
         kv_dtype = dtype if kv_dtype is None else kv_dtype
@@ -157,10 +169,15 @@ class PagedKVCache:
         tables, lens, longest = self.pool.block_tables(
             st["ids"], self.max_blocks_per_seq, -1, st["h_tables"], st["h_lens"], with_max=True)
         n_items = -1  # the full grid
-        if self.work_list:
+        order = self._item_order
+        split = 0 < self.partition_size < longest
+        if self.work_list and order is None and split:
+            order = (_abi.PKV_ITEMS_LONGEST_FIRST if self.fp8 else
+                     _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST)
+        if self.work_list and order is not None:
             n_items = _abi.pkv_decode_work_items(lens, self.num_kv_heads, longest,
                                                  self.partition_size, st["h_items"],
-                                                 self._item_order).numel()
+                                                 order).numel()
         return dict(st=st, num_pairs=pairs.shape[0], max_len=longest, num_items=n_items)
 
     def upload_step(self, prep, stream=None):

@@ -34,9 +34,10 @@
 //   an m16n8k16 tensor-core product with the 16 tokens as M and up to 8
 //   heads as N (K tiles through ldmatrix, Q^T fragments in registers);
 //   O^T += V^T P^T takes V^T tiles through ldmatrix.trans and P^T from the
-//   score fragments by movmatrix, with head_dim as M; P enters as a 16-bit
-//   high part plus a 16-bit remainder (two products into one accumulator),
-//   so rounding the softmax weights costs no accuracy.
+//   score fragments by movmatrix, with head_dim as M.  Over 16-bit caches P
+//   enters as a 16-bit high part plus a 16-bit remainder (two products into
+//   one accumulator), so rounding the softmax weights costs no accuracy;
+//   over e4m3 caches, whose products all run in f16, P is one f16 rounding.
 //
 // Every wait on an mbarrier is bounded (1 s); on expiry the kernel records
 // PKV_DEVERR_TIMEOUT, waits (bounded) for its loads in flight and skips its
@@ -68,11 +69,6 @@ constexpr int kSubTileBytes = kTile * kBoxD * 2;   // one swizzled box: 2 KiB
 #endif
 #ifndef PKV_DECODE_STAGES_D64
 #define PKV_DECODE_STAGES_D64 4
-#endif
-// Whether the e4m3 path (every product in f16) adds the f16 remainder of P
-// as a second P V product, as the 16-bit paths do.
-#ifndef PKV_DECODE_E4M3_P_REMAINDER
-#define PKV_DECODE_E4M3_P_REMAINDER 1
 #endif
 constexpr int kWarps = PKV_DECODE_WARPS;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -286,8 +282,11 @@ struct MmaWarp {
     static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
     static constexpr int GP = NT * 8;  // heads held (padded)
     static constexpr bool kMma = true;
-    // the remainder of P as a second product (always for 16-bit caches)
-    static constexpr bool kPRem = !E4 || PKV_DECODE_E4M3_P_REMAINDER;
+    // Over e4m3 caches P enters the P V product as one f16 rounding
+    // (relative error <= 2^-11 per weight, so the output moves by at most
+    // 2^-11 * sum_t p_t |v_t| / l); over 16-bit caches it adds its rounded
+    // remainder as a second product (a bf16 P alone is off by up to 2^-8)
+    static constexpr bool kPRem = !E4;
     uint32_t qf[KS][NT][2];            // Q^T B-fragments
     float acc[KS][NT][4];              // O^T[d][head]
     float m[NT][2], l[NT][2];          // per lane: heads nt*8 + (lane&3)*2 + {0,1}
@@ -473,9 +472,9 @@ struct MmaWarp {
                 acc[mt][nt][3] *= c1;
             }
             // P[token][head] as 16-bit fragments, transposed to P^T
-            // B-fragments.  P is split into a rounded high part and the
-            // rounded remainder, so the PV product sees P to ~16 bits of
-            // mantissa instead of the 8 of one bf16 rounding.
+            // B-fragments.  Over 16-bit caches P is split into a rounded high
+            // part and the rounded remainder, so the PV product sees P to
+            // ~16 bits of mantissa instead of the 8 of one bf16 rounding.
             const uint32_t h01 = Storage<MT>::from_float2(p0, p1);
             const uint32_t h23 = Storage<MT>::from_float2(p2, p3);
             const float2 b01 = Storage<MT>::to_float2(h01), b23 = Storage<MT>::to_float2(h23);
@@ -1277,12 +1276,15 @@ extern "C" int pkv_decode_attention_fp8_items(
 
 // The decode work list ("PagedAttention 动态内存分页" page, 技术边界与取舍: a
 // batch of very uneven lengths is what costs).  Items are the (sequence, KV
-// head, partition) triples that hold tokens; longest first, a counting sort
-// on the number of 16-token tiles each holds orders them largest first,
-// keeping grid order among equals, in O(items + P / 16).
+// head, partition) triples that hold tokens.  Within a sequence they go
+// partition by partition with the KV heads of a partition side by side: the
+// heads' slices of one block share its memory rows.  Longest first, a
+// counting sort on the number of 16-token tiles each item holds orders them
+// largest first, keeping that order among equals, in O(items + P / 16).
 extern "C" int pkv_decode_work_items(const int32_t* context_lens, int num_seqs,
                                      int num_kv_heads, int max_context_len, int partition_size,
                                      int order, int32_t* items, int capacity, int* num_items) {
+    PKV_NVTX_RANGE("pkv_decode_work_items");
     using namespace pkv;
     PKV_REQUIRE(num_items != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL count");
     *num_items = 0;
@@ -1291,53 +1293,58 @@ extern "C" int pkv_decode_work_items(const int32_t* context_lens, int num_seqs,
     PKV_REQUIRE(partition_size >= 0 && partition_size % kTile == 0, PKV_ERR_INVALID,
                 "pkv_decode_work_items: partition_size %d is not a multiple of 16",
                 partition_size);
-    PKV_REQUIRE(order == PKV_ITEMS_LONGEST_FIRST || order == PKV_ITEMS_GRID, PKV_ERR_INVALID,
-                "pkv_decode_work_items: order %d", order);
+    PKV_REQUIRE(order == PKV_ITEMS_LONGEST_FIRST || order == PKV_ITEMS_SEQUENCES_LONGEST_FIRST ||
+                    order == PKV_ITEMS_BATCH_ORDER,
+                PKV_ERR_INVALID, "pkv_decode_work_items: order %d", order);
     if (num_seqs == 0) return PKV_OK;
     PKV_REQUIRE(context_lens != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL lengths");
     int P, NP;
     plan_partitions(max_context_len, partition_size, &P, &NP);
     PKV_REQUIRE((int64_t)num_seqs * num_kv_heads * NP < (1ll << 31), PKV_ERR_UNSUPPORTED,
                 "pkv_decode_work_items: grid too large");
-    const int nbuckets = P / kTile + 1;  // tiles per item: 0 .. P / 16
-    std::vector<int64_t> count(nbuckets + 1, 0);
     int64_t total = 0;
     for (int s = 0; s < num_seqs; ++s) {
         const int L = context_lens[s];
         PKV_REQUIRE(L >= 0 && L <= max_context_len, PKV_ERR_INVALID,
                     "pkv_decode_work_items: context_lens[%d] = %d outside [0, %d]", s, L,
                     max_context_len);
-        const int np = L > 0 ? (L + P - 1) / P : 1;
-        // full partitions, then the last one's tiles (0 for an empty context)
-        const int last = L - (np - 1) * P;
-        count[P / kTile] += (int64_t)(np - 1) * num_kv_heads;
-        count[(last + kTile - 1) / kTile] += num_kv_heads;
-        total += (int64_t)np * num_kv_heads;
+        total += (int64_t)(L > 0 ? (L + P - 1) / P : 1) * num_kv_heads;
     }
     *num_items = (int)total;
     PKV_REQUIRE(total <= capacity, PKV_ERR_INVALID,
                 "pkv_decode_work_items: %lld items, capacity %d", (long long)total, capacity);
     PKV_REQUIRE(items != nullptr, PKV_ERR_INVALID, "pkv_decode_work_items: NULL items");
-    // start offset of each bucket, the largest bucket first; in grid order
-    // every item goes to one bucket, in the order of the loop below
-    std::vector<int64_t> start(nbuckets, 0);
-    int64_t at = 0;
-    for (int b = nbuckets - 1; b >= 0; --b) {
-        start[b] = at;
-        at += count[b];
-    }
-    const bool grid_order = order == PKV_ITEMS_GRID;
-    if (grid_order) start[0] = 0;
+    // the sequences in the order their items are emitted
+    std::vector<int> seqs(num_seqs);
+    for (int s = 0; s < num_seqs; ++s) seqs[s] = s;
+    if (order == PKV_ITEMS_SEQUENCES_LONGEST_FIRST)
+        std::stable_sort(seqs.begin(), seqs.end(),
+                         [&](int a, int b) { return context_lens[a] > context_lens[b]; });
+    // bucket of an item: its tiles (largest first) for longest first, one
+    // bucket otherwise
+    const bool by_tiles = order == PKV_ITEMS_LONGEST_FIRST;
+    const int nbuckets = by_tiles ? P / kTile + 1 : 1;  // tiles per item: 0 .. P / 16
+    auto bucket = [&](int tokens) { return by_tiles ? (tokens + kTile - 1) / kTile : 0; };
+    std::vector<int64_t> start(nbuckets + 1, 0);
     for (int s = 0; s < num_seqs; ++s) {
         const int L = context_lens[s];
         const int np = L > 0 ? (L + P - 1) / P : 1;
-        for (int h = 0; h < num_kv_heads; ++h) {
-            const int64_t base = ((int64_t)s * num_kv_heads + h) * NP;
-            for (int part = 0; part < np; ++part) {
-                const int tok = std::min(P, L - part * P);
-                const int b = grid_order ? 0 : (tok + kTile - 1) / kTile;
-                items[start[b]++] = (int32_t)(base + part);
-            }
+        for (int part = 0; part < np; ++part)
+            start[bucket(std::min(P, L - part * P))] += num_kv_heads;
+    }
+    int64_t at = 0;  // counts to start offsets, the largest bucket first
+    for (int b = nbuckets - 1; b >= 0; --b) {
+        const int64_t c = start[b];
+        start[b] = at;
+        at += c;
+    }
+    for (int s : seqs) {
+        const int L = context_lens[s];
+        const int np = L > 0 ? (L + P - 1) / P : 1;
+        for (int part = 0; part < np; ++part) {
+            int64_t& pos = start[bucket(std::min(P, L - part * P))];
+            for (int h = 0; h < num_kv_heads; ++h)
+                items[pos++] = (int32_t)(((int64_t)s * num_kv_heads + h) * NP + part);
         }
     }
     return PKV_OK;

@@ -1,5 +1,6 @@
-"""Decode over the longest-first work list (pkv_decode_attention_items and
-its e4m3 form) against the fp64 oracle and against the full grid.
+"""Decode over the planner's work list (pkv_decode_attention_items and its
+e4m3 form), in each of its orders, against the fp64 oracle and against the
+full grid.
 
 Each CTA computes the same (sequence, KV head, partition) whatever order
 the CTAs run in, and the merging CTA combines the partials in partition
@@ -51,8 +52,8 @@ def decode(p, scale, P, dev, items=None, fp8=False, dev_error=None, fill=float("
     return out.cpu()
 
 
-def plan(p, Hkv, P):
-    return _abi.pkv_decode_work_items(p["lens"], Hkv, int(max(p["lens"])), P)
+def plan(p, Hkv, P, order=_abi.PKV_ITEMS_LONGEST_FIRST):
+    return _abi.pkv_decode_work_items(p["lens"], Hkv, int(max(p["lens"])), P, order=order)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
@@ -63,7 +64,9 @@ def test_work_list_matches_oracle_and_full_grid(dtype, D, Hq, Hkv, bs, P, cuda_d
     seed = zlib.crc32(repr(("wl", dtype, D, Hq, Hkv, bs, P)).encode()) % 10000
     p = paged_problem(seed, Hq, Hkv, D, bs, LENS, dtype)
     scale = 1.0 / np.sqrt(D)
-    got = decode(p, scale, P, cuda_device, items=plan(p, Hkv, P))
+    order = (_abi.PKV_ITEMS_LONGEST_FIRST, _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST,
+             _abi.PKV_ITEMS_BATCH_ORDER)[seed % 3]
+    got = decode(p, scale, P, cuda_device, items=plan(p, Hkv, P, order))
     full = decode(p, scale, P, cuda_device)
     want = ref.decode_attention(p["q"], p["kc"], p["vc"], p["tables"], p["lens"], scale, dtype,
                                 Hkv, bs)
@@ -73,10 +76,12 @@ def test_work_list_matches_oracle_and_full_grid(dtype, D, Hq, Hkv, bs, P, cuda_d
 
 @pytest.mark.parametrize("Hq,Hkv,bs,P", [(8, 8, 16, 0), (16, 2, 16, 32), (32, 2, 64, 128),
                                          (8, 1, 32, 64)])
-def test_work_list_e4m3_matches_oracle_and_full_grid(Hq, Hkv, bs, P, cuda_device):
+@pytest.mark.parametrize("order", [_abi.PKV_ITEMS_LONGEST_FIRST,
+                                   _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST])
+def test_work_list_e4m3_matches_oracle_and_full_grid(Hq, Hkv, bs, P, order, cuda_device):
     p = fp8_problem(zlib.crc32(repr((Hq, Hkv, bs, P)).encode()) % 10000, Hq, Hkv, 128, bs,
                     LENS, "bf16")
-    got = decode(p, 0.09, P, cuda_device, items=plan(p, Hkv, P), fp8=True)
+    got = decode(p, 0.09, P, cuda_device, items=plan(p, Hkv, P, order), fp8=True)
     full = decode(p, 0.09, P, cuda_device, fp8=True)
     want = ref.decode_attention_fp8(p["q"], p["kc"], p["vc"], p["ks"], p["vs"], p["tables"],
                                     p["lens"], 0.09, "bf16", Hkv, bs)
@@ -119,9 +124,11 @@ def test_empty_work_list_launches_nothing(cuda_device):
     assert (got == -3.0).all()
 
 
-def test_cache_driver_runs_the_work_list(cuda_device):
+@pytest.mark.parametrize("work_list", ["auto", "longest_first", "sequences_longest_first",
+                                       "batch_order"])
+def test_cache_driver_runs_the_work_list(work_list, cuda_device):
     """PagedKVCache plans the work list on the host for each step; its steps
-    give the full grid's output bit for bit."""
+    give the full grid's output bit for bit, in every order."""
     dev = cuda_device
     g = torch.Generator().manual_seed(9)
     S, Hq, Hkv, D, bs, P = 6, 16, 4, 128, 16, 64
@@ -131,7 +138,7 @@ def test_cache_driver_runs_the_work_list(cuda_device):
     kc = torch.randn(nb, bs, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
     vc = torch.randn(nb, bs, Hkv, D, generator=g).to(torch.bfloat16).to(dev)
     outs = []
-    for wl in (True, False):
+    for wl in (work_list, False):
         c = PagedKVCache(nb, bs, Hq, Hkv, D, torch.bfloat16, dev, 32, P, free_order=order,
                          key_cache=kc.clone(), value_cache=vc.clone(), scale=0.1, work_list=wl)
         for s in range(S):
