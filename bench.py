@@ -531,9 +531,10 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     host memory.  Per step: the step's q, k and v go up in one copy from
     pinned memory (on a second stream, into one of two input buffers), the
     host pool reserves the slots and plans the work list
-    (PagedKVCache.prepare_step), the metadata goes up in one copy
-    (upload_step), the kernels run (launch_step), and the attention output
-    comes back to pinned host memory; the host waits for it.
+    (PagedKVCache.prepare_step, one native call), and one more native call
+    (PagedKVCache.run_step) uploads the metadata, runs the kernels and
+    copies the attention output back to pinned host memory; the host waits
+    for it.
 
     serial: the host waits for step i's output before it enqueues step i+1
     (the pool's work for step i+1 and its input upload still overlap step
@@ -567,14 +568,12 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
 
     def enqueue(i, prep):
         b, o = i % 2, i % nout
-        with torch.cuda.stream(stream):
-            stream.wait_event(ev_in[b])
-            cache.upload_step(prep, stream)
-            dq, dk, dv = views[b]
-            cache.launch_step(prep, dq, dk, dv, outs[o], stream=stream)
-            ev_used[b].record(stream)
-            houts[o].copy_(outs[o], non_blocking=True)
-            ev_out[o].record(stream)
+        stream.wait_event(ev_in[b])
+        dq, dk, dv = views[b]
+        # metadata upload, copies, slot write, attention and readback: one call
+        cache.run_step(prep, dq, dk, dv, outs[o], out_host=houts[o], stream=stream)
+        ev_used[b].record(stream)
+        ev_out[o].record(stream)
 
     def upload_inputs(i):
         b = i % 2
@@ -621,7 +620,7 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
             "python_gc": "collected before the timed loop, paused during it",
             "host_ms_per_step": {
                 "pool_append_tables_and_work_list": round(1e3 * host["prepare"] / steps, 4),
-                "metadata_upload_and_launches": round(1e3 * host["enqueue"] / steps, 4),
+                "step_enqueue": round(1e3 * host["enqueue"] / steps, 4),
                 "input_upload_enqueue": round(1e3 * host["input_upload_enqueue"] / steps, 4),
                 "readback_wait": round(1e3 * host["wait"] / steps, 4)}}
 

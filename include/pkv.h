@@ -64,6 +64,9 @@ typedef enum {
 
 typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 
+/* The host block pool (opaque; see "Host block pool" below). */
+typedef struct pkv_pool pkv_pool;
+
 /* Codes a kernel writes into dev_error[0]; dev_error[1] gets the index. */
 #define PKV_DEVERR_NONE 0
 #define PKV_DEVERR_CONTEXT_LEN 1 /* index: seq; len < 0, > max_context_len or > table */
@@ -275,6 +278,95 @@ PKV_API int pkv_decode_attention_items(void* out, const void* query, const void*
                                        cudaStream_t stream);
 
 /* ---------------------------------------------------------------------- */
+/* One decode step in two calls                                            */
+/* ---------------------------------------------------------------------- */
+/*
+ * The per-step sequence the pages describe ("Paged KV" wiki page, 实现原理 /
+ * 运行阶段: take a slot, write the new K/V, attend through the Block Table;
+ * "PagedAttention 动态内存分页" page, 写时复制与内存共享: copy a shared block
+ * before writing into it), as one host call and one device call.  They
+ * compose the entry points above and add no arithmetic: a caller saves the
+ * per-call overhead of driving the steps one by one.
+ */
+
+/*
+ * Host part: pkv_seq_append_batch for the n sequences (slots, cow_pairs,
+ * *num_pairs), then pkv_pool_block_tables (block_tables [n,
+ * max_blocks_per_seq] padded with -1, context_lens [n], *max_context_len),
+ * then, when a work list is wanted, pkv_decode_work_items into work_items
+ * (*num_items; -1 when none was made).  order_split is the list's order
+ * (PKV_ITEMS_*) when the step splits a sequence into partitions
+ * (0 < partition_size < *max_context_len), order_one_pass when it does not;
+ * -1 makes no list for that case.  All pointers are host memory.  Errors
+ * are those of the three calls; an error in the first leaves the sequences
+ * before the failing one appended (as pkv_seq_append_batch does).
+ */
+PKV_API int pkv_step_prepare(pkv_pool* pool, int n, const int64_t* seq_ids, int64_t* slots,
+                             int32_t* cow_pairs, int* num_pairs, int32_t* block_tables,
+                             int max_blocks_per_seq, int32_t* context_lens,
+                             int* max_context_len, int num_kv_heads, int partition_size,
+                             int order_split, int order_one_pass, int32_t* work_items,
+                             int items_capacity, int* num_items);
+
+/*
+ * Device part, enqueued on `stream` in this order:
+ *   1. meta_bytes from meta_host to meta_device (cudaMemcpyAsync; pinned
+ *      host memory keeps it asynchronous; 0 bytes: none) — typically the
+ *      step's slots, pairs, tables, lengths and work list in one buffer,
+ *      which the pointers below then point into;
+ *   2. pkv_copy_blocks (or _fp8) of the num_pairs cow_pairs (0: none);
+ *   3. pkv_write_slots (or _fp8) of the num_tokens new rows (0: none);
+ *   4. pkv_decode_attention (or _fp8), over work_items when that is not
+ *      NULL (pkv_decode_attention_items);
+ *   5. out_bytes of out to out_host (cudaMemcpyAsync; 0: none).
+ * The cache is e4m3 (the _fp8 calls, block_stride in bytes) when k_scale
+ * or v_scale is not NULL.  Every field means what the argument of the same
+ * name means in those calls; the key/value rows and queries are
+ * [num_tokens | num_seqs, heads, head_dim] in dtype.  A failing part
+ * returns its status with the parts before it already enqueued.
+ */
+typedef struct pkv_decode_step_args {
+    const void* meta_host;
+    void* meta_device;
+    size_t meta_bytes;
+    const int32_t* cow_pairs;
+    int num_pairs;
+    const void* key;
+    const void* value;
+    const int64_t* slot_mapping;
+    int num_tokens;
+    void* key_cache;
+    void* value_cache;
+    float* k_scale;
+    float* v_scale;
+    int num_blocks;
+    int block_size;
+    int num_kv_heads;
+    int head_dim;
+    int64_t block_stride;
+    void* out;
+    const void* query;
+    const int32_t* block_tables;
+    int max_blocks_per_seq;
+    const int32_t* context_lens;
+    int num_seqs;
+    int max_context_len;
+    int num_q_heads;
+    float scale;
+    int partition_size;
+    void* workspace;
+    size_t workspace_bytes;
+    const int32_t* work_items;
+    int num_items;
+    void* out_host;
+    size_t out_bytes;
+    pkv_dtype dtype;
+    int32_t* dev_error;
+} pkv_decode_step_args;
+
+PKV_API int pkv_decode_step(const pkv_decode_step_args* args, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------- */
 /* Paged prefill attention                                                 */
 /* ---------------------------------------------------------------------- */
 /*
@@ -446,9 +538,8 @@ PKV_API int pkv_decode_attention_fp8_items(void* out, const void* query, const v
  * 0, 1, ... when free_order is NULL); freed blocks are pushed in table order;
  * an operation that runs out of blocks returns PKV_ERR_OOM and changes
  * nothing.  Not thread-safe: the caller serialises calls on one pool.
- * All pointers here are host pointers.
+ * All pointers here are host pointers.  (pkv_pool is declared at the top.)
  */
-typedef struct pkv_pool pkv_pool;
 
 /* free_order: NULL or a permutation of 0..num_blocks-1 (host int32). */
 PKV_API int pkv_pool_create(int num_blocks, int block_size, const int32_t* free_order,

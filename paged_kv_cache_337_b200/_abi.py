@@ -62,6 +62,9 @@ SIGNATURES = {
     "pkv_decode_attention_fp8_items": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _p, _i, _i, _i,
                                             _i, _i, _i, _i, _i64, _f, _i, _p, _sz, _p, _i, _i,
                                             _p, _p]),
+    "pkv_step_prepare": (_i, [_p, _i, _p, _p, _p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _p, _i,
+                              _p]),
+    "pkv_decode_step": (_i, [_p, _p]),
     "pkv_pool_create": (_i, [_i, _i, _p, C.POINTER(_p)]),
     "pkv_pool_destroy": (None, [_p]),
     "pkv_seq_add": (_i, [_p, _i64, _i]),
@@ -94,6 +97,24 @@ SIGNATURES = {
 }
 
 _lib = None
+
+
+class DecodeStepArgs(C.Structure):
+    """pkv_decode_step_args (include/pkv.h): one decode step's device work."""
+
+    _fields_ = [("meta_host", _p), ("meta_device", _p), ("meta_bytes", _sz),
+                ("cow_pairs", _p), ("num_pairs", _i),
+                ("key", _p), ("value", _p), ("slot_mapping", _p), ("num_tokens", _i),
+                ("key_cache", _p), ("value_cache", _p), ("k_scale", _p), ("v_scale", _p),
+                ("num_blocks", _i), ("block_size", _i), ("num_kv_heads", _i), ("head_dim", _i),
+                ("block_stride", _i64),
+                ("out", _p), ("query", _p), ("block_tables", _p), ("max_blocks_per_seq", _i),
+                ("context_lens", _p), ("num_seqs", _i), ("max_context_len", _i),
+                ("num_q_heads", _i), ("scale", _f), ("partition_size", _i),
+                ("workspace", _p), ("workspace_bytes", _sz),
+                ("work_items", _p), ("num_items", _i),
+                ("out_host", _p), ("out_bytes", _sz),
+                ("dtype", _i), ("dev_error", _p)]
 
 
 class PkvError(RuntimeError):

@@ -29,6 +29,8 @@ the library; this module only moves arguments.
 launch waits for the upload's event, and the next upload into the same
 staging bank waits for the last launch that read it.
 """
+import ctypes as C
+
 import torch
 
 from . import _abi
@@ -125,7 +127,8 @@ class PagedKVCache:
         buffer and one device buffer holding slots | lengths | copy pairs |
         Block Tables | work items, so a step's metadata travels in one copy
         (of the used prefix) and the next step can be prepared while the
-        previous upload is in flight."""
+        previous upload is in flight.  Each bank keeps the step arguments
+        (pkv_decode_step_args) whose pointers into it do not change."""
         banks = self._staging.get(n)
         if banks is None:
             pin = torch.cuda.is_available()
@@ -144,41 +147,72 @@ class PagedKVCache:
             for _ in range(2):
                 h = torch.empty(max(words, 1), dtype=torch.int32, pin_memory=pin)
                 d = torch.empty(max(words, 1), dtype=torch.int32, device=self.device)
+                ids = torch.empty(n, dtype=torch.int64)
                 hv, dv = views(h), views(d)
-                banks.append(dict(ids=torch.empty(n, dtype=torch.int64), h=h, d=d,
-                                  h_slots=hv["slots"], h_lens=hv["lens"], h_pairs=hv["pairs"],
-                                  h_tables=hv["tables"], h_items=hv["items"],
-                                  d_slots=dv["slots"], d_lens=dv["lens"], d_pairs=dv["pairs"],
-                                  d_tables=dv["tables"], d_items=dv["items"], items_off=i0,
-                                  uploaded=None, consumed=None))
+                bank = dict(ids=ids, h=h, d=d, h_slots=hv["slots"], h_lens=hv["lens"],
+                            h_pairs=hv["pairs"], h_tables=hv["tables"], h_items=hv["items"],
+                            d_slots=dv["slots"], d_lens=dv["lens"], d_pairs=dv["pairs"],
+                            d_tables=dv["tables"], d_items=dv["items"], items_off=i0,
+                            items_cap=cap, uploaded=None, consumed=None, stream=None)
+                # host pointers of the bank for pkv_step_prepare
+                bank["prep_ptrs"] = (ids.data_ptr(), hv["slots"].data_ptr(),
+                                     hv["pairs"].data_ptr(), hv["tables"].data_ptr(),
+                                     hv["lens"].data_ptr(), hv["items"].data_ptr())
+                bank["args"] = self._step_args(bank, n)
+                banks.append(bank)
             self._staging[n] = banks = [banks, 0]
         banks[1] ^= 1
         return banks[0][banks[1]]
 
+    def _step_args(self, bank, n):
+        """pkv_decode_step_args with every field that stays fixed for a bank."""
+        a = _abi.DecodeStepArgs()
+        nb, bs, hkv, d, bstride = self._geom
+        a.meta_host, a.meta_device = bank["h"].data_ptr(), bank["d"].data_ptr()
+        a.cow_pairs, a.slot_mapping = bank["d_pairs"].data_ptr(), bank["d_slots"].data_ptr()
+        a.key_cache, a.value_cache = self.key_cache.data_ptr(), self.value_cache.data_ptr()
+        if self.fp8:
+            a.k_scale, a.v_scale = self.k_scale.data_ptr(), self.v_scale.data_ptr()
+        a.num_blocks, a.block_size, a.num_kv_heads, a.head_dim = nb, bs, hkv, d
+        a.block_stride = bstride
+        a.block_tables, a.max_blocks_per_seq = bank["d_tables"].data_ptr(), self.max_blocks_per_seq
+        a.context_lens, a.num_seqs, a.num_tokens = bank["d_lens"].data_ptr(), n, n
+        a.num_q_heads, a.scale, a.partition_size = (self.num_q_heads, float(self.scale),
+                                                    int(self.partition_size))
+        a.dtype, a.dev_error = self._dtype_code, self.dev_error.data_ptr()
+        return a
+
+    def _orders(self):
+        """(order when the step splits sequences, order when it does not) for
+        pkv_step_prepare; -1: no work list."""
+        if not self.work_list:
+            return -1, -1
+        if self._item_order is None:  # "auto"
+            return (_abi.PKV_ITEMS_LONGEST_FIRST if self.fp8 else
+                    _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST), -1
+        return self._item_order, self._item_order
+
     def prepare_step(self, seq_ids):
-        """Host part of a decode step: reserve one slot per sequence (new
-        blocks and copy-on-write pairs as needed) and gather the Block Tables
-        and lengths into pinned memory.  Returns the prepared step."""
+        """Host part of a decode step (pkv_step_prepare): reserve one slot per
+        sequence (new blocks and copy-on-write pairs as needed), gather the
+        Block Tables and lengths into pinned memory and plan the work list.
+        Returns the prepared step."""
         st = self._stage(len(seq_ids))
         if st["uploaded"] is not None:
             st["uploaded"].synchronize()  # this bank's last upload has left
         if st.get("ids_src") is not seq_ids:  # a new id list: convert it once
             st["ids"].copy_(torch.as_tensor(seq_ids, dtype=torch.int64))
             st["ids_src"] = seq_ids
-        slots, pairs = self.pool.append_batch(st["ids"], st["h_slots"], st["h_pairs"])
-        tables, lens, longest = self.pool.block_tables(
-            st["ids"], self.max_blocks_per_seq, -1, st["h_tables"], st["h_lens"], with_max=True)
-        n_items = -1  # the full grid
-        order = self._item_order
-        split = 0 < self.partition_size < longest
-        if self.work_list and order is None and split:
-            order = (_abi.PKV_ITEMS_LONGEST_FIRST if self.fp8 else
-                     _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST)
-        if self.work_list and order is not None:
-            n_items = _abi.pkv_decode_work_items(lens, self.num_kv_heads, longest,
-                                                 self.partition_size, st["h_items"],
-                                                 order).numel()
-        return dict(st=st, num_pairs=pairs.shape[0], max_len=longest, num_items=n_items)
+        ids, slots, pairs, tables, lens, items = st["prep_ptrs"]
+        npairs, longest, nitems = C.c_int(), C.c_int(), C.c_int()
+        split, one = self._orders()
+        _abi._check(_abi.lib().pkv_step_prepare(
+            self.pool._h, len(seq_ids), ids, slots, pairs, C.byref(npairs), tables,
+            self.max_blocks_per_seq, lens, C.byref(longest), self.num_kv_heads,
+            int(self.partition_size), split, one, items, st["items_cap"], C.byref(nitems)),
+            "pkv_step_prepare")
+        return dict(st=st, num_pairs=npairs.value, max_len=longest.value,
+                    num_items=nitems.value)
 
     def upload_step(self, prep, stream=None):
         """One host-to-device copy of a prepared step's metadata (the work
@@ -201,80 +235,103 @@ class PagedKVCache:
             self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
         return self._workspace if need else None
 
+    def _check_step_tensors(self, query, key, value, out, out_host):
+        """The binding's checks, once per set of shapes, dtypes and devices."""
+        sig = self._signature(query, key, value, out) + (
+            None if out_host is None else (tuple(out_host.shape), out_host.dtype,
+                                           out_host.is_pinned()),)
+        if sig in self._seen:
+            return
+        S = query.shape[0]
+        _abi._on_device("decode step", query, key, value, out)
+        if query.device != self.device:
+            raise ValueError("decode step: tensors must be on the cache's device")
+        want = {"query": (query, (S, self.num_q_heads, self.head_dim)),
+                "key": (key, (S, self.num_kv_heads, self.head_dim)),
+                "value": (value, (S, self.num_kv_heads, self.head_dim)),
+                "out": (out, (S, self.num_q_heads, self.head_dim))}
+        for name, (t, shape) in want.items():
+            if tuple(t.shape) != shape or t.dtype != self.dtype or not t.is_contiguous():
+                raise ValueError("decode step: %s must be a contiguous %s tensor of shape %s"
+                                 % (name, self.dtype, shape))
+        if out_host is not None and (out_host.device.type != "cpu" or
+                                     out_host.shape != out.shape or
+                                     out_host.dtype != out.dtype or
+                                     not out_host.is_contiguous()):
+            raise ValueError("decode step: out_host must be a host copy of out's shape")
+        self._seen.add(sig)
+
+    def run_step(self, prep, query, key, value, out, out_host=None, stream=None):
+        """Device part of a prepared decode step in one native call
+        (pkv_decode_step): the metadata upload, the copy-on-write copies, the
+        slot write, decode attention and, with out_host (pinned host memory
+        for an asynchronous copy), the output's copy to the host.  All on
+        `stream` (the current stream by default)."""
+        st = prep["st"]
+        S = len(st["ids"])
+        self._check_step_tensors(query, key, value, out, out_host)
+        s_ = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if st["consumed"] is not None and st["stream"] is not s_:
+            s_.wait_event(st["consumed"])  # a launch on another stream read this bank
+        a = st["args"]
+        items = prep.get("num_items", -1)
+        a.meta_bytes = 4 * (st["items_off"] + max(items, 0))
+        a.num_pairs = prep["num_pairs"]
+        a.key, a.value, a.query, a.out = (key.data_ptr(), value.data_ptr(), query.data_ptr(),
+                                          out.data_ptr())
+        a.max_context_len = prep["max_len"]
+        ws = self.workspace(S, prep["max_len"])
+        a.workspace, a.workspace_bytes = (ws.data_ptr(), ws.numel()) if ws is not None else (
+            None, 0)
+        a.work_items = st["d_items"].data_ptr() if items >= 0 else None
+        a.num_items = max(items, 0)
+        if out_host is not None:
+            a.out_host, a.out_bytes = out_host.data_ptr(), out.numel() * out.element_size()
+        else:
+            a.out_host, a.out_bytes = None, 0
+        _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
+                    "pkv_decode_step")
+        for ev in ("uploaded", "consumed"):
+            if st[ev] is None:
+                st[ev] = torch.cuda.Event()
+            st[ev].record(s_)
+        st["stream"] = s_
+        return out
+
     def launch_step(self, prep, query, key, value, out, max_len=None, stream=None):
         """Device part of a decode step (copy, write, attention) with the
         prepared metadata uploaded by upload_step (on this or another
         stream: the launch waits for it)."""
         st = prep["st"]
-        n = prep["num_pairs"]
-        items = prep.get("num_items", -1)
-        if max_len is not None and max_len != prep["max_len"]:
-            items = -1  # the work list was planned for the prepared bound
-        max_len = prep["max_len"] if max_len is None else max_len
         s_ = stream if stream is not None else torch.cuda.current_stream(self.device)
         if st["uploaded"] is not None:
             s_.wait_event(st["uploaded"])
-        try:
-            return self._launch(st, n, items, max_len, query, key, value, out, stream)
-        finally:
-            if st["consumed"] is None:
-                st["consumed"] = torch.cuda.Event()
-            st["consumed"].record(s_)
-
-    def _launch(self, st, n, items, max_len, query, key, value, out, stream):
-        if n:
-            self._copy(st["d_pairs"][:n], stream)
-        ws = self.workspace(len(st["ids"]), max_len)
-        wl = st["d_items"][:items] if items >= 0 else None
-        if not self._checked(query, key, value, out):
-            # first use of these tensor shapes: the binding's full checks
-            self._write(key, value, st["d_slots"], stream)
-            self._attend(out, query, st["d_tables"], st["d_lens"], max_len, ws, stream, wl)
-            self._seen.add(self._signature(query, key, value, out))
-            return out
-        # same shapes, dtypes and device as a call already checked: pass the
-        # pointers straight to the C entry points
-        L = _abi.lib()
-        sp = _abi._stream(stream, self.device)
-        kc, vc = self.key_cache, self.value_cache
-        nb, bs, hkv, d, bstride = self._geom
-        S = query.shape[0]
-        err = self.dev_error.data_ptr()
-        wsp, wsn = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
-        args = (st["d_tables"].data_ptr(), self.max_blocks_per_seq, st["d_lens"].data_ptr(), S,
-                int(max_len), self.num_q_heads, hkv, d, nb, bs, bstride, float(self.scale),
-                int(self.partition_size), wsp, wsn)
-        tail = (self._dtype_code, err, sp)
-        if wl is not None:
-            tail = (wl.data_ptr(), wl.numel()) + tail
-        if self.fp8:
-            ks, vs = self.k_scale.data_ptr(), self.v_scale.data_ptr()
-            _abi._check(L.pkv_write_slots_fp8(
-                key.data_ptr(), value.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
-                st["d_slots"].data_ptr(), S, nb, bs, hkv, d, bstride, self._dtype_code, err, sp),
-                "pkv_write_slots_fp8")
-            fn = L.pkv_decode_attention_fp8_items if wl is not None else L.pkv_decode_attention_fp8
-            _abi._check(fn(out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), ks, vs,
-                           *args, *tail), "pkv_decode_attention_fp8")
-            return out
-        _abi._check(L.pkv_write_slots(key.data_ptr(), value.data_ptr(), kc.data_ptr(),
-                                      vc.data_ptr(), st["d_slots"].data_ptr(), S, nb, bs, hkv,
-                                      d, bstride, self._dtype_code, err, sp), "pkv_write_slots")
-        fn = L.pkv_decode_attention_items if wl is not None else L.pkv_decode_attention
-        _abi._check(fn(out.data_ptr(), query.data_ptr(), kc.data_ptr(), vc.data_ptr(), *args,
-                       *tail), "pkv_decode_attention")
+        if max_len is not None and max_len != prep["max_len"]:
+            # the work list was planned for the prepared bound: the full grid
+            prep = dict(prep, max_len=max_len, num_items=-1)
+        self._check_step_tensors(query, key, value, out, None)
+        a = st["args"]
+        items = prep.get("num_items", -1)
+        a.meta_bytes = 0
+        a.num_pairs = prep["num_pairs"]
+        a.key, a.value, a.query, a.out = (key.data_ptr(), value.data_ptr(), query.data_ptr(),
+                                          out.data_ptr())
+        a.max_context_len = prep["max_len"]
+        ws = self.workspace(len(st["ids"]), prep["max_len"])
+        a.workspace, a.workspace_bytes = (ws.data_ptr(), ws.numel()) if ws is not None else (
+            None, 0)
+        a.work_items = st["d_items"].data_ptr() if items >= 0 else None
+        a.num_items = max(items, 0)
+        a.out_host, a.out_bytes = None, 0
+        _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
+                    "pkv_decode_step")
+        if st["consumed"] is None:
+            st["consumed"] = torch.cuda.Event()
+        st["consumed"].record(s_)
+        st["stream"] = s_
         return out
 
-    # -- the three device calls, for either cache type ---------------------
-    def _copy(self, pairs, stream):
-        if self.fp8:
-            _abi.pkv_copy_blocks_fp8(self.key_cache, self.value_cache, self.k_scale,
-                                     self.v_scale, pairs, dev_error=self.dev_error,
-                                     stream=stream)
-        else:
-            _abi.pkv_copy_blocks(self.key_cache, self.value_cache, pairs,
-                                 dev_error=self.dev_error, stream=stream)
-
+    # -- single device calls, for either cache type ---------------------------
     def _write(self, key, value, slots, stream):
         if self.fp8:
             _abi.pkv_write_slots_fp8(key, value, self.key_cache, self.value_cache, self.k_scale,
@@ -301,17 +358,13 @@ class PagedKVCache:
         return tuple((tuple(t.shape), t.dtype, t.device, t.is_contiguous())
                      for t in (query, key, value, out))
 
-    def _checked(self, query, key, value, out):
-        return self._signature(query, key, value, out) in self._seen
-
     def decode_step(self, seq_ids, query, key, value, out=None, stream=None):
         """One full decode step for seq_ids (query [S, Hq, D], key/value
         [S, Hkv, D] on the device).  Returns out [S, Hq, D]."""
         prep = self.prepare_step(seq_ids)
-        self.upload_step(prep, stream)
         if out is None:
             out = torch.empty_like(query)
-        return self.launch_step(prep, query, key, value, out, stream=stream)
+        return self.run_step(prep, query, key, value, out, stream=stream)
 
     # -- swapping to pinned host memory -------------------------------------
     def enable_swap(self, num_host_blocks):

@@ -155,3 +155,51 @@ def test_cache_driver_runs_the_work_list(work_list, cuda_device):
         outs.append(step)
     for a, b in zip(*outs):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_run_step_in_one_call_matches_the_separate_calls(fp8, cuda_device):
+    """PagedKVCache.run_step (pkv_decode_step: upload, copies, write, attention
+    and the output's copy to pinned host memory in one native call) gives
+    bit for bit the output of upload_step + launch_step on an identical
+    cache, through copy-on-write steps, and its host copy equals the
+    device output."""
+    dev = cuda_device
+    g = torch.Generator().manual_seed(12)
+    S, Hq, Hkv, D, bs, P = 5, 16, 4, 128, 16, 64
+    lens = [37, 70, 300, 1, 129]
+    nb = 80
+    order = torch.randperm(nb, generator=g).tolist()
+    kv = torch.uint8 if fp8 else None
+    init = (torch.randint(0, 120, (nb, bs, Hkv, D), generator=g, dtype=torch.uint8) if fp8 else
+            torch.randn(nb, bs, Hkv, D, generator=g).to(torch.bfloat16))
+    caches = []
+    for _ in range(2):
+        c = PagedKVCache(nb, bs, Hq, Hkv, D, torch.bfloat16, dev, 32, P, free_order=order,
+                         key_cache=init.clone().to(dev), value_cache=init.clone().to(dev),
+                         scale=0.1, kv_dtype=kv, kv_scale=0.02)
+        for s in range(S):
+            c.add_sequence(s, lens[s])
+        c.fork(0, 5)  # sequence 0's partial last block is shared: a copy-on-write step
+        caches.append(c)
+    ids = list(range(S + 1))
+    host = torch.empty(S + 1, Hq, D, dtype=torch.bfloat16).pin_memory()
+    gq = torch.Generator().manual_seed(13)
+    for step in range(4):
+        q = torch.randn(S + 1, Hq, D, generator=gq).to(torch.bfloat16).to(dev)
+        k = torch.randn(S + 1, Hkv, D, generator=gq).to(torch.bfloat16).to(dev)
+        v = torch.randn(S + 1, Hkv, D, generator=gq).to(torch.bfloat16).to(dev)
+        a, b = caches
+        pa, pb = a.prepare_step(ids), b.prepare_step(ids)
+        assert pa["num_pairs"] == pb["num_pairs"] == (1 if step == 0 else 0)
+        out_a = torch.empty_like(q)
+        a.run_step(pa, q, k, v, out_a, out_host=host)
+        b.upload_step(pb)
+        out_b = b.launch_step(pb, q, k, v, torch.empty_like(q))
+        torch.cuda.synchronize()
+        assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+        assert torch.equal(host.view(torch.int16), out_a.cpu().view(torch.int16))
+    for c in caches:
+        c.check_errors()
+    assert torch.equal(caches[0].key_cache, caches[1].key_cache)
+    assert torch.equal(caches[0].value_cache, caches[1].value_cache)
