@@ -56,6 +56,10 @@ PROFILE_TRAFFIC = {
     "7b_s256_h32_d128_bs16_bf16": os.path.join(ROOT, "profiles", "decode_attention_7b_s256.md"),
     "7b_s256_h32_d128_bs16_bf16_kv_e4m3": os.path.join(ROOT, "profiles",
                                                         "decode_attention_fp8_7b_s256.md"),
+    "70b_gqa_s64_hq64_hkv8_d128_bs16_bf16": os.path.join(ROOT, "profiles",
+                                                          "decode_attention_gqa_70b.md"),
+    "70b_gqa_s64_hq64_hkv8_d128_bs16_bf16_kv_e4m3": os.path.join(
+        ROOT, "profiles", "decode_attention_fp8_gqa_70b.md"),
     "prefill_s8_l2048_hq32_hkv8_d128_bs16_bf16": os.path.join(ROOT, "profiles",
                                                                "prefill_attention_s8_l2048.md"),
 }
@@ -723,6 +727,9 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
         # copy-on-write: a bytes kernel, plus a scale kernel for e4m3 caches
         return (((2 if fp8 else 1) if state["npairs"] else 0)) + 2
 
+    # inputs and caches were made on the default stream; the timed
+    # stream is not ordered after it
+    torch.cuda.synchronize(dev)
     for i in range(args.warmup):
         step(states[i % n_states])
     torch.cuda.synchronize(dev)
@@ -856,6 +863,9 @@ def run_cow_layers(args, world, rank, local):
     def timed(fn, K):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(K)]
+        # inputs and caches were made on the default stream; the timed
+        # stream is not ordered after it
+        torch.cuda.synchronize(dev)
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize(dev)
@@ -960,13 +970,15 @@ def run_swap(args, world, rank, local):
     kc, vc, hk, hv = cache.key_cache, cache.value_cache, cache.host_key_cache, cache.host_value_cache
 
     def step(ev=None):
-        pairs = torch.cat([cache.pool.swap_out(s) for s in moved]).to(dev)
+        with torch.cuda.stream(stream):  # the pairs go up on the stream that reads them
+            pairs = torch.cat([cache.pool.swap_out(s) for s in moved]).to(dev)
         if ev:
             ev[0].record(stream)
         _abi.pkv_swap_blocks(kc, vc, hk, hv, pairs, dev_error=err, stream=stream)
         if ev:
             ev[1].record(stream)
-        pairs = torch.cat([cache.pool.swap_in(s) for s in moved]).to(dev)
+        with torch.cuda.stream(stream):
+            pairs = torch.cat([cache.pool.swap_in(s) for s in moved]).to(dev)
         if ev:
             ev[2].record(stream)
         _abi.pkv_swap_blocks(hk, hv, kc, vc, pairs, dev_error=err, stream=stream)
@@ -974,6 +986,9 @@ def run_swap(args, world, rank, local):
             ev[3].record(stream)
         return 2 * pairs.shape[0] * 2 * block_bytes
 
+    # inputs and caches were made on the default stream; the timed
+    # stream is not ordered after it
+    torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -1104,6 +1119,9 @@ def run_prefill(args, world, rank, local, with_cpu=True):
         if ev:
             ev[1].record(stream)
 
+    # inputs and caches were made on the default stream; the timed
+    # stream is not ordered after it
+    torch.cuda.synchronize(dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -1254,6 +1272,9 @@ def run_shared_prefix(args, world, rank, local):
                                       stream=stream, work_items=stt["items"])
             return (1 if stt["npairs"] else 0) + 2
 
+        # inputs and caches were made on the default stream; the timed
+        # stream is not ordered after it
+        torch.cuda.synchronize(dev)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize(dev)

@@ -102,8 +102,10 @@ class PagedKVCache:
         blocks taken, in order."""
         self.pool.add(seq_id, num_tokens)
         if key is not None and num_tokens > 0:
-            slots = self.pool.slot_mapping(seq_id, 0, num_tokens).to(self.device)
-            self._write(key, value, slots, stream)
+            s = stream if stream is not None else torch.cuda.current_stream(self.device)
+            with torch.cuda.stream(s):  # the slots go up on the stream that writes them
+                slots = self.pool.slot_mapping(seq_id, 0, num_tokens).to(self.device)
+            self._write(key, value, slots, s)
 
     def fork(self, parent, child):
         self.pool.fork(parent, child)

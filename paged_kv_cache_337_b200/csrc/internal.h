@@ -28,6 +28,22 @@ class NvtxRange {
     bool on_;
 };
 
+// The partitions of a decode launch: the partition length actually used
+// and the number of partitions of the grid.  One pass (the longest context
+// rounded up to the 16-token tile) when partition_size is 0 or covers
+// max_context_len.
+inline void plan_partitions(int max_context_len, int partition_size, int* P, int* NP) {
+    constexpr int kTile = 16;
+    if (partition_size <= 0 || partition_size >= max_context_len) {
+        const int ctx = max_context_len > 0 ? max_context_len : 1;
+        *P = (ctx + kTile - 1) / kTile * kTile;
+        *NP = 1;
+    } else {
+        *P = partition_size;
+        *NP = (max_context_len + partition_size - 1) / partition_size;
+    }
+}
+
 }  // namespace pkv
 
 #define PKV_NVTX_RANGE(name) ::pkv::NvtxRange pkv_nvtx_range_(name)
