@@ -657,6 +657,14 @@ __device__ __forceinline__ void decode_cta(const CUtensorMap& kmap, const CUtens
     }
     const int t_begin = part * P;
     const int t_end = min(L, t_begin + P);
+    // Tiles of 16 tokens per block (block_size is a multiple of 16, at most
+    // 256) and a multiplier that divides a tile index by it: the high word
+    // of ti * ceil(2^32 / tpb) is floor(ti / tpb) for every ti below 2^28,
+    // and tile indexes stay below 2^27, so the loop needs no division.
+    const unsigned tpb = (unsigned)(bs / kTile);
+    const unsigned tpb_mul = tpb == 1 ? 0u : 0xFFFFFFFFu / tpb + 1u;
+    const unsigned ti0 = (unsigned)(t_begin / kTile);
+    auto block_of = [&](unsigned ti) -> unsigned { return tpb_mul ? __umulhi(ti, tpb_mul) : ti; };
     const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
     const int nlb = t_end > t_begin ? (t_end - 1) / bs - lb0 + 1 : 0;
 
@@ -675,9 +683,10 @@ __device__ __forceinline__ void decode_cta(const CUtensorMap& kmap, const CUtens
         return (int64_t)(phys >= 0 && phys < p.num_blocks ? phys : 0) * p.num_kv_heads + kvh;
     };
     auto issue = [&](int st, int tile) {
-        const int t0 = t_begin + tile * kTile;
-        const int phys = table[t0 / bs - lb0];
-        const int off = t0 % bs;
+        const unsigned ti = ti0 + (unsigned)tile;
+        const unsigned lb = block_of(ti);
+        const int phys = table[lb - (unsigned)lb0];
+        const int off = (int)(ti - lb * tpb) * kTile;
         uint8_t* kdst = my_stages + st * Pl::kStageBytes;
         uint8_t* vdst = kdst + Pl::kTileBytes;
         mbar_arrive_expect_tx(&my_bars[st], Pl::kTx);
@@ -720,7 +729,7 @@ __device__ __forceinline__ void decode_cta(const CUtensorMap& kmap, const CUtens
         const int valid = min(kTile, t_end - (t_begin + tile * kTile));
         float kscale = 1.f, vscale = 1.f;
         if constexpr (FP8) {
-            const int64_t si = scale_index(table[(t_begin + tile * kTile) / bs - lb0]) & 3;
+            const int64_t si = scale_index(table[block_of(ti0 + (unsigned)tile) - (unsigned)lb0]) & 3;
             kscale = my_scales[st * 8 + si];
             vscale = my_scales[st * 8 + 4 + si];
 
