@@ -25,11 +25,13 @@
 //     tensor cores work on one tile while the other tile's softmax runs;
 //   - eight softmax warps, four per Q tile (one tensor-memory lane quarter
 //     each, one row per thread), read S, apply the causal mask, keep the
-//     running max and sum, write P over S (a 16-bit high part and its
-//     16-bit remainder, two MMAs) and rescale O when the running max grows
-//     by more than 2^8, then write the normalised output;
+//     running max and sum, write P over S (one f16 rounding; a bf16 high
+//     part and its remainder, two MMAs, for a bf16 V group beyond f16's
+//     range) and rescale O when the running max grows by more than 2^8,
+//     then write the normalised output;
 //   - four Q warps stage each item's Q tiles once the previous item's last
-//     S has read them.
+//     S has read them, and convert each landed bf16 V tile to f16 in
+//     shared memory, so that P V runs as one f16 MMA per 16 keys.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -61,10 +63,12 @@ constexpr int kThreads = (kQWarp0 + kQWarps) * 32;
 // high | P low, 32 each, written over S once it is read) at 256 t and
 // 256 t + 64, O at 256 t + 128; key tile j uses S buffer j % 2
 constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = kKeys / 2, kTmemCols = 512;
-// kv_full/empty per stage; s_full/p_full per (Q tile, S buffer); o_done and
-// o_free per Q tile; drain, q_ready, q_free
-constexpr int kNumBars = 2 * kStages + 6 * kQTiles + 3;
-constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16;
+// kv_full/kv_empty/v_ready per stage; s_full/p_full per (Q tile, S
+// buffer); o_done and o_free per Q tile; drain, q_ready, q_free
+constexpr int kNumBars = 3 * kStages + 6 * kQTiles + 3;
+// after the barriers: the tensor-memory address (16 bytes) and, per stage,
+// one byte per 16-key group of V: 1 = converted to f16, 0 = left in bf16
+constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16 + 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;  // rescale O when the max grows by more than 2^8
 
@@ -129,6 +133,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
 struct Bars {
     uint64_t* kv_full;   // [kStages]: TMA bytes landed
     uint64_t* kv_empty;  // [kStages]: the P V MMAs reading the stage completed
+    uint64_t* v_ready;   // [kStages]: a bf16 V tile converted (the four Q warps)
     uint64_t* s_full;    // [kQTiles][2]: S of the buffer in tensor memory
     uint64_t* p_full;    // [kQTiles][2]: P of the buffer written (and O rescaled)
     uint64_t* o_done;    // [kQTiles]: the P V MMAs of the Q tile completed
@@ -264,12 +269,13 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
 // picks the ring stage (g mod kStages) and the S buffer (g mod 2).
 template <bool BF16>
 __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem, uint32_t qaddr,
-                           uint8_t* stages, bool* failed) {
+                           uint8_t* stages, const uint32_t* vflags, bool* failed) {
     // one lane issues every MMA and every commit (a commit tracks the MMAs
     // of the thread that executes it)
     const bool leader = tc::elect_one();
     constexpr uint32_t kIdS = tc::f16_idesc(BF16, false, kRows, kKeys);  // K: K-major B
     constexpr uint32_t kIdPV = tc::f16_idesc(BF16, true, kRows, kD);     // V: MN-major B
+    constexpr uint32_t kIdPVh = tc::f16_idesc(false, true, kRows, kD);   // V converted to f16
     // descriptor bases; a step's byte offset enters the start-address
     // field (16-byte units, no carry: shared addresses stay below 256 KiB)
     const uint64_t qd0 = tc::sw128_desc(qaddr, 16, 1024);
@@ -294,17 +300,23 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
     // O += P V of Q tile t for key tile g (O = P V for an item's first):
     // 8 steps of 16 keys; V's 8-key groups 1 KiB apart (SBO), its 64-dim
     // halves 16 KiB apart (LBO)
-    auto issue_pv = [&](int t, int g, bool first) {
+    // A bf16 V tile's 16-key groups are in f16 (flag byte 1: one MMA with
+    // the f16 P) or still in bf16 (two MMAs: P's high part and remainder).
+    auto issue_pv = [&](int t, int g, bool first, uint32_t flags) {
         const uint64_t vd = vd0 + (uint64_t)(((g % kStages) * kStageBytes) >> 4);
         const uint32_t cs = kTileCols * t, cp = cs + kKeys * (g & 1);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk) {
             if (leader) {
-                tc::mma_ts(tmem + cs + kColO, tmem + cp + kk * 8, vd + kk * (2048 >> 4), kIdPV,
-                           (!first || kk > 0) ? 1u : 0u);
-                if constexpr (BF16)  // the remainder of a bf16 P
-                    tc::mma_ts(tmem + cs + kColO, tmem + cp + kColPl + kk * 8,
-                               vd + kk * (2048 >> 4), kIdPV, 1u);
+                const uint64_t v = vd + kk * (2048 >> 4);
+                const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+                if (!BF16 || ((flags >> (8 * kk)) & 1u)) {
+                    tc::mma_ts(tmem + cs + kColO, tmem + cp + kk * 8, v, BF16 ? kIdPVh : kIdPV,
+                               acc);
+                } else {
+                    tc::mma_ts(tmem + cs + kColO, tmem + cp + kk * 8, v, kIdPV, acc);
+                    tc::mma_ts(tmem + cs + kColO, tmem + cp + kColPl + kk * 8, v, kIdPV, 1u);
+                }
             }
         }
         if (leader) tc::commit(smem_addr(&b.o_done[t]));
@@ -348,7 +360,11 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
             // tile A
             if (!wait(&b.p_full[buf], ph)) break;
             if (j == 0 && nk > 0 && !wait(&b.o_free[0], (nk - 1) & 1)) break;
-            issue_pv(0, g, j == 0);
+            // a bf16 V tile converted (it landed before its S)
+            if (BF16 && !wait(&b.v_ready[g % kStages], (g / kStages) & 1)) break;
+            const uint32_t vf =
+                BF16 ? *reinterpret_cast<const volatile uint32_t*>(vflags + g % kStages) : 0u;
+            issue_pv(0, g, j == 0, vf);
             if (more) {
                 if (!wait(&b.kv_full[(g + 2) % kStages], ((g + 2) / kStages) & 1)) break;
                 issue_s(0, g + 2);
@@ -356,7 +372,7 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
             // tile B
             if (!wait(&b.p_full[2 + buf], ph)) break;
             if (j == 0 && nk > 0 && !wait(&b.o_free[1], (nk - 1) & 1)) break;
-            issue_pv(1, g, j == 0);
+            issue_pv(1, g, j == 0, vf);
             if (leader) tc::commit(smem_addr(&b.kv_empty[g % kStages]));  // both P V of the stage
             if (more) {
                 issue_s(1, g + 2);
@@ -380,6 +396,58 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
     return __all_sync(0xffffffffu, ok);
 }
 
+// bf16 V tile -> f16, in place, by the four Q warps (bf16 caches only).
+// P V then runs as one f16 MMA per 16 keys: P rounded once to f16 carries
+// at most 2^-11 relative error per weight (P <= 2^8, row sum >= 1), where a
+// bf16 P alone would need a second MMA for its remainder.  The conversion
+// is exact for every bf16 value of magnitude 2^-14 .. 65504 and within
+// 2^-25 absolute below.  A 16-key group holding a value of magnitude
+// 65536 or more (or an infinity or NaN) stays in bf16 and its P V takes the
+// two-part bf16 path, so no input changes the result's accuracy.  Q warp qw
+// owns keys 16 qw .. 16 qw + 15 of the tile (2 KiB of each 64-dim half;
+// the swizzle permutes 16-byte chunks within a row, so the rows stay put);
+// rows at or past `valid` (keys past the context) are zeroed.  Returns the
+// group's flag: 1 converted, 0 left in bf16.
+__device__ __forceinline__ uint32_t convert_v_group(uint8_t* vt, int qw, int lane, int valid) {
+    constexpr int kChunks = 8;  // 16-byte chunks per lane: 4 per 64-dim half
+    uint4 v[kChunks];
+    uint32_t mx = 0;  // largest magnitude (bf16 bits) of each 16-bit lane, valid rows
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int row = 16 * qw + (lane >> 3) + 4 * (i & 3);
+        v[i] = *reinterpret_cast<const uint4*>(vt + (i >> 2) * kHalfBytes + qw * 2048 +
+                                               (lane + 32 * (i & 3)) * 16);
+        if (row < valid) {
+            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(w[e] & 0x7fff7fffu));
+        }
+    }
+    // 0x4780 is bf16 65536, the first magnitude beyond f16's 65504
+    const bool wide = __any_sync(0xffffffffu, (mx >> 16) >= 0x4780u || (mx & 0xffffu) >= 0x4780u);
+#pragma unroll
+    for (int i = 0; i < kChunks; ++i) {
+        const int row = 16 * qw + (lane >> 3) + 4 * (i & 3);
+        uint4 o = make_uint4(0, 0, 0, 0);
+        if (row < valid) {
+            if (wide) {
+                o = v[i];
+            } else {
+                uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w[e] = Storage<__half>::from_float2(__uint_as_float(w[e] << 16),
+                                                        __uint_as_float(w[e] & 0xffff0000u));
+                o = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        *reinterpret_cast<uint4*>(vt + (i >> 2) * kHalfBytes + qw * 2048 +
+                                  (lane + 32 * (i & 3)) * 16) = o;
+    }
+    return wide ? 0u : 1u;
+}
+
 // Q warps (warps 10-13): per item, once every S MMA of the previous item
 // has completed (q_free), Q rows (token r / G, head kvh * G + r % G) are
 // copied into shared memory swizzled as the MMA reads them.  Q warp w takes
@@ -387,14 +455,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 // 64 w + i / 16, + 2, ...; all copies are in flight before one wait, and
 // rows past the sequence's are zero-filled.
 template <typename T>
-__device__ void stage_q(const PrefillParams& p, const Bars& b, uint8_t* qsm, int qw, int lane,
-                        bool* failed) {
+__device__ void stage_q(const PrefillParams& p, const Bars& b, uint8_t* qsm, uint8_t* stages,
+                        uint32_t* vflags, int qw, int lane, bool* failed) {
     constexpr int kRowsPerWarp = kQTiles * kRows / kQWarps;
     const T* qbase = static_cast<const T*>(p.query);
     const int G = p.group, Hq = p.num_q_heads;
     const int ch = lane & 15;
     const uint64_t stream_once = l2_policy_evict_first();  // Q is read once
     int nk = 0;
+    int gv = 0;  // V tiles converted over all items
     for (int k = 0; !*failed; ++k) {
         const int idx = item_index(k);
         if (idx >= p.num_items) break;
@@ -425,12 +494,29 @@ __device__ void stage_q(const PrefillParams& p, const Bars& b, uint8_t* qsm, int
         __syncwarp();
         if (lane == 0) mbar_arrive_one(b.q_ready);
         ++nk;
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            // the item's V tiles, as they land
+            for (int j = 0; j < it.ntiles; ++j, ++gv) {
+                const int st = gv % kStages;
+                if (!warp_wait(&b.kv_full[st], (gv / kStages) & 1)) {
+                    *failed = true;
+                    break;
+                }
+                const uint32_t f = convert_v_group(stages + st * kStageBytes + kTileBytes, qw,
+                                                   lane, it.L - j * kKeys);
+                tc::fence_proxy_async_smem();  // the tensor cores read V through the async proxy
+                if (lane == 0) reinterpret_cast<uint8_t*>(vflags + st)[qw] = (uint8_t)f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive_one(&b.v_ready[st]);
+            }
+        }
     }
 }
 
 template <typename T>
 __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tmem,
-                             uint8_t* stages, int warp, int lane, bool* failed) {
+                             uint8_t* stages, const uint32_t* vflags, int warp, int lane,
+                             bool* failed) {
     const int t = (warp - kSoftmaxWarp0) >> 2;  // Q tile of this warp
     const int quarter = warp & 3;              // tensor-memory lanes 32 * quarter .. + 31
     const uint32_t trow = tmem + ((uint32_t)(32 * quarter) << 16) + kTileCols * t;
@@ -502,37 +588,60 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
                 }
             }
             // P = 2^(s - m) on key pairs (packed fp32 FMA, add and subtract);
-            // the row sum in four independent packed partial sums.  A bf16 P
-            // is written as a 16-bit high part and the 16-bit remainder (two
-            // MMAs): one bf16 value carries up to 2^-9 relative error per
-            // weight.  An f16 P (2^-11, P <= 2^8, row sum >= 1) is one part.
-            constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
+            // the row sum in four independent packed partial sums.  P enters
+            // P V as one f16 rounding (2^-11 relative error per weight, P <=
+            // 2^8, row sum >= 1): f16 caches, and bf16 caches whose V group
+            // the Q warps converted to f16.  A bf16 group left in bf16 takes
+            // P as a bf16 high part and its bf16 remainder (two MMAs): one
+            // bf16 rounding alone carries up to 2^-9 per weight.
+            constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+            uint32_t fl = 0x01010101u;  // one byte per 16-key group: 1 = f16
+            if constexpr (kBf16) {
+                const int st = g % kStages;
+                if (!warp_wait(&b.v_ready[st], (g / kStages) & 1)) break;
+                fl = *reinterpret_cast<const volatile uint32_t*>(vflags + st);
+            }
             const float2 sl2 = make_float2(sl, sl), nmu2 = make_float2(-mu, -mu);
             float2 ls[4] = {};
 #pragma unroll
             for (int c = 0; c < kKeys / 32; ++c) {
-                uint32_t hi[16], lo[16];
+                float2 w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float2 x =
                         ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), sl2, nmu2);
-                    const float2 w = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    ls[e & 3] = fadd2(ls[e & 3], w);
-                    hi[e] = Storage<T>::from_float2(w.x, w.y);
-                    if constexpr (kSplit) {
-                        const float2 rem = fsub2(w, Storage<T>::to_float2(hi[e]));
-                        lo[e] = Storage<T>::from_float2(rem.x, rem.y);
-                    }
+                    w[e] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    ls[e & 3] = fadd2(ls[e & 3], w[e]);
                 }
-                tc::st16(srow + 16 * c, hi);  // over S, already read
-                if constexpr (kSplit) tc::st16(srow + kColPl + 16 * c, lo);
+                uint32_t hi[16], lo[16];
+                const uint32_t pair = (fl >> (16 * c)) & 0x0101u;  // groups 2c, 2c + 1
+                if (pair == 0x0101u) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) hi[e] = Storage<__half>::from_float2(w[e].x, w[e].y);
+                    tc::st16(srow + 16 * c, hi);  // over S, already read
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        if ((pair >> (8 * (e >> 3))) & 1u) {
+                            hi[e] = Storage<__half>::from_float2(w[e].x, w[e].y);
+                            lo[e] = 0u;
+                        } else {
+                            hi[e] = Storage<T>::from_float2(w[e].x, w[e].y);
+                            const float2 rem = fsub2(w[e], Storage<T>::to_float2(hi[e]));
+                            lo[e] = Storage<T>::from_float2(rem.x, rem.y);
+                        }
+                    }
+                    tc::st16(srow + 16 * c, hi);
+                    tc::st16(srow + kColPl + 16 * c, lo);
+                }
             }
             ls[0] = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
             l += ls[0].x + ls[0].y;
             // keys past the context in the item's last tile: zero their V
-            // rows (NaN bit patterns there must not meet their zero weights)
+            // rows (NaN bit patterns there must not meet their zero weights);
+            // the Q warps do it for bf16 caches while converting
             const int key0 = j * kKeys;
-            if (t == 0 && key0 + kKeys > it.L) {
+            if (!kBf16 && t == 0 && key0 + kKeys > it.L) {
                 const int st = g % kStages;
                 if (!warp_wait(&b.kv_full[st], (g / kStages) & 1)) break;
                 uint8_t* vt = stages + st * kStageBytes + kTileBytes;
@@ -607,13 +716,16 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     uint8_t* stages = smem + kQBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
-    uint64_t* tail = bars + 2 * kStages + 6 * kQTiles;
+    uint32_t* vflags = tmem_slot + 4;  // [kStages]: four group bytes each
+    uint64_t* sp = bars + 3 * kStages;
+    uint64_t* tail = sp + 6 * kQTiles;
     Bars b{bars,
            bars + kStages,
            bars + 2 * kStages,
-           bars + 2 * kStages + 2 * kQTiles,
-           bars + 2 * kStages + 4 * kQTiles,
-           bars + 2 * kStages + 5 * kQTiles,
+           sp,
+           sp + 2 * kQTiles,
+           sp + 4 * kQTiles,
+           sp + 5 * kQTiles,
            tail,
            tail + 1,
            tail + 2};
@@ -627,6 +739,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&b.kv_full[i], 1);
             mbar_init(&b.kv_empty[i], 1);
+            mbar_init(&b.v_ready[i], kQWarps);
         }
         for (int t = 0; t < kQTiles; ++t) {
             for (int u = 0; u < 2; ++u) {
@@ -653,11 +766,11 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         produce(kmap, vmap, p, stages, b, lane, &failed);
     else if (warp == kMmaWarp)
         issue_mmas<std::is_same<T, __nv_bfloat16>::value>(p, b, tmem, smem_addr(qsm), stages,
-                                                          &failed);
+                                                          vflags, &failed);
     else if (warp >= kQWarp0)
-        stage_q<T>(p, b, qsm, warp - kQWarp0, lane, &failed);
+        stage_q<T>(p, b, qsm, stages, vflags, warp - kQWarp0, lane, &failed);
     else
-        softmax_rows<T>(p, b, tmem, stages, warp, lane, &failed);
+        softmax_rows<T>(p, b, tmem, stages, vflags, warp, lane, &failed);
     if (failed) report_error(p.dev_error, PKV_DEVERR_TIMEOUT, 0);
     tc::fence_before_sync();
     __syncthreads();

@@ -76,6 +76,70 @@ def test_prefill_large_scores_stay_finite(cuda_device):
     assert tolerance_violation(got, want, ATOL, RTOL) <= 0
 
 
+def test_prefill_bf16_values_beyond_f16_range(cuda_device):
+    """A bf16 cache's P V runs in f16 where its values allow (the V tile
+    converted in shared memory); a 16-key group holding a value of
+    magnitude 65536 or more keeps bf16 and the two-part P.  Such values sit
+    in a few late groups (the middle of tile 3, the last partial tile, a
+    group of the second sequence), beside plain groups of the same tiles.
+    Rows that cannot see them are held to the usual bound.  The rows that
+    do see them get 2^-15 max|V| w_big more, w_big being the weight those
+    tokens carry in the row (the oracle's output over an indicator V): the
+    two-part P holds a weight to about 2^-17 of itself, and that rounding
+    times a 1e5 value can exceed 2e-3 on its own, in any 16-bit P."""
+    p, q, qs = case(11, 8, 2, 16, [300, 70], [300, 70], "bf16")
+    g = torch.Generator().manual_seed(12)
+    vc = p["vc"].float()
+    big = ((0, 243), (0, 250), (0, 299), (1, 66))
+    for s, tok in big:
+        blk = int(p["tables"][s][tok // 16])
+        vc[blk, tok % 16] = torch.randn(vc.shape[2:], generator=g) * 1e5
+    p["vc"] = vc.to(torch.bfloat16)
+    vmax = float(p["vc"].float().abs().max())
+    assert vmax > 65536
+    scale = 1.0 / np.sqrt(128)
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    got = run_prefill(p, q, qs, scale, cuda_device, err)
+    want = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                 2, 16)
+    assert err.tolist() == [0, 0]
+    assert torch.isfinite(got).all()
+    # a row sees a big token when its position is at or past it
+    sees = np.zeros(int(qs[-1]), bool)
+    for s, tok in big:
+        L, n = int(p["lens"][s]), int(qs[s + 1] - qs[s])
+        pos = L - n + np.arange(n)
+        sees[qs[s]:qs[s + 1]] |= pos >= tok
+    assert (~sees).sum() > 300 and sees.sum() > 50
+    assert tolerance_violation(got[~sees], want[~sees], ATOL, RTOL) <= 0
+    ind = torch.zeros(p["vc"].shape)
+    for s, tok in big:
+        ind[int(p["tables"][s][tok // 16]), tok % 16] = 1.0
+    w_big = ref.prefill_attention(q, p["kc"], ind.to(torch.bfloat16), p["tables"], p["lens"], qs,
+                                  scale, "bf16", 2, 16)[..., :1]
+    excess = (np.abs(got.double().numpy() - want)
+              - (ATOL + vmax * 2.0 ** -15 * w_big + RTOL * np.abs(want)))
+    assert excess[sees].max() <= 0
+
+
+def test_prefill_bf16_all_values_beyond_f16_range(cuda_device):
+    """Every V group of a bf16 cache beyond f16's range: the whole P V takes
+    the two-part bf16 path.  V scaled by 2^17 scales the exact output by
+    2^17 and changes no weight, so got / 2^17 must meet the usual bound
+    against the oracle of the unscaled cache."""
+    p, q, qs = case(13, 8, 2, 16, [300, 70], [300, 70], "bf16")
+    scale = 1.0 / np.sqrt(128)
+    want = ref.prefill_attention(q, p["kc"], p["vc"], p["tables"], p["lens"], qs, scale, "bf16",
+                                 2, 16)
+    big = dict(p)
+    big["vc"] = (p["vc"].float() * 2.0 ** 17).to(torch.bfloat16)  # exact: a power of two
+    err = torch.zeros(2, dtype=torch.int32, device=cuda_device)
+    got = run_prefill(big, q, qs, scale, cuda_device, err)
+    assert err.tolist() == [0, 0]
+    assert torch.isfinite(got).all()
+    assert tolerance_violation(got.double() / 2.0 ** 17, want, ATOL, RTOL) <= 0
+
+
 def test_prefill_bad_lengths_are_reported(cuda_device):
     p, q, qs = case(6, 4, 4, 16, [10, 20], [10, 20], "f16")
     lens = torch.tensor([10, 5], dtype=torch.int32)  # sequence 1: 20 rows but 5 tokens
