@@ -537,7 +537,8 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     host pool reserves the slots and plans the work list
     (PagedKVCache.prepare_step, one native call), and one more native call
     (PagedKVCache.run_step) uploads the metadata, runs the kernels and
-    copies the attention output back to pinned host memory; the host waits
+    copies the attention output back to pinned host memory on a readback
+    stream, where the copy overlaps the next step's kernels; the host waits
     for it.
 
     serial: the host waits for step i's output before it enqueues step i+1
@@ -558,6 +559,7 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     outs = [torch.empty((S, Hq, D), dtype=dt, device=dev) for _ in range(nout)]
     houts = [torch.empty((S, Hq, D), dtype=dt).pin_memory() for _ in range(nout)]
     copy_stream = torch.cuda.Stream(dev)
+    readback_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
     ev_used = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b done
     ev_out = [torch.cuda.Event() for _ in range(nout)]  # a step's result on the host
@@ -573,11 +575,14 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     def enqueue(i, prep):
         b, o = i % 2, i % nout
         stream.wait_event(ev_in[b])
+        if i >= nout:
+            stream.wait_event(ev_out[o])  # step i - nout's readback has read outs[o]
         dq, dk, dv = views[b]
         # metadata upload, copies, slot write, attention and readback: one call
-        cache.run_step(prep, dq, dk, dv, outs[o], out_host=houts[o], stream=stream)
+        cache.run_step(prep, dq, dk, dv, outs[o], out_host=houts[o], stream=stream,
+                       readback_stream=readback_stream)
         ev_used[b].record(stream)
-        ev_out[o].record(stream)
+        ev_out[o].record(readback_stream)
 
     def upload_inputs(i):
         b = i % 2
@@ -638,7 +643,7 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     _abi.lib()
-    P = spec.partition_size if args.partition_size < 0 else args.partition_size
+    P = spec.partition_for(fp8) if args.partition_size < 0 else args.partition_size
 
     # seeded shapes on the CPU; cache values drawn on the device (per rank)
     gen = torch.Generator("cpu").manual_seed(spec.seed)

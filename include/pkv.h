@@ -318,7 +318,14 @@ PKV_API int pkv_step_prepare(pkv_pool* pool, int n, const int64_t* seq_ids, int6
  *   3. pkv_write_slots (or _fp8) of the num_tokens new rows (0: none);
  *   4. pkv_decode_attention (or _fp8), over work_items when that is not
  *      NULL (pkv_decode_attention_items);
- *   5. out_bytes of out to out_host (cudaMemcpyAsync; 0: none).
+ *   5. out_bytes of out to out_host (cudaMemcpyAsync; 0: none).  With
+ *      out_stream not NULL the copy goes on out_stream instead: the call
+ *      records out_event on `stream` after step 4 and makes out_stream
+ *      wait for it, so that the copy overlaps whatever the caller enqueues
+ *      next on `stream`.  Both handles are the caller's (out_event an
+ *      event it created; PKV_ERR_INVALID when it is NULL); the caller must
+ *      not overwrite `out` before the copy has run (wait on an event it
+ *      records on out_stream).
  * The cache is e4m3 (the _fp8 calls, block_stride in bytes) when k_scale
  * or v_scale is not NULL.  Every field means what the argument of the same
  * name means in those calls; the key/value rows and queries are
@@ -362,6 +369,8 @@ typedef struct pkv_decode_step_args {
     size_t out_bytes;
     pkv_dtype dtype;
     int32_t* dev_error;
+    cudaStream_t out_stream; /* NULL: the readback goes on `stream` */
+    cudaEvent_t out_event;   /* used with out_stream */
 } pkv_decode_step_args;
 
 PKV_API int pkv_decode_step(const pkv_decode_step_args* args, cudaStream_t stream);

@@ -263,12 +263,17 @@ class PagedKVCache:
             raise ValueError("decode step: out_host must be a host copy of out's shape")
         self._seen.add(sig)
 
-    def run_step(self, prep, query, key, value, out, out_host=None, stream=None):
+    def run_step(self, prep, query, key, value, out, out_host=None, stream=None,
+                 readback_stream=None):
         """Device part of a prepared decode step in one native call
         (pkv_decode_step): the metadata upload, the copy-on-write copies, the
         slot write, decode attention and, with out_host (pinned host memory
         for an asynchronous copy), the output's copy to the host.  All on
-        `stream` (the current stream by default)."""
+        `stream` (the current stream by default), except the output's copy
+        when readback_stream is given: it then runs there once the attention
+        is done, overlapping what comes next on `stream`.  The caller reads
+        out_host, and writes `out` again, only after that copy (an event
+        recorded on readback_stream after this call)."""
         st = prep["st"]
         S = len(st["ids"])
         self._check_step_tensors(query, key, value, out, out_host)
@@ -291,6 +296,13 @@ class PagedKVCache:
             a.out_host, a.out_bytes = out_host.data_ptr(), out.numel() * out.element_size()
         else:
             a.out_host, a.out_bytes = None, 0
+        a.out_stream, a.out_event = None, None
+        if out_host is not None and readback_stream is not None:
+            if st.get("attended") is None:
+                st["attended"] = torch.cuda.Event()
+                st["attended"].record(s_)  # the handle exists once recorded
+            a.out_stream = readback_stream.cuda_stream
+            a.out_event = st["attended"].cuda_event
         _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
                     "pkv_decode_step")
         for ev in ("uploaded", "consumed"):

@@ -107,7 +107,18 @@ extern "C" int pkv_decode_step(const pkv_decode_step_args* a, cudaStream_t strea
     if (st != PKV_OK) return st;
     if (a->out_bytes > 0) {
         PKV_REQUIRE(a->out_host && a->out, PKV_ERR_INVALID, "pkv_decode_step: NULL output");
-        e = cudaMemcpyAsync(a->out_host, a->out, a->out_bytes, cudaMemcpyDeviceToHost, stream);
+        cudaStream_t rs = stream;
+        if (a->out_stream != nullptr) {
+            PKV_REQUIRE(a->out_event != nullptr, PKV_ERR_INVALID,
+                        "pkv_decode_step: out_stream without out_event");
+            e = cudaEventRecord(a->out_event, stream);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(a->out_stream, a->out_event, 0);
+            if (e != cudaSuccess)
+                return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: readback stream: %s",
+                                 cudaGetErrorString(e));
+            rs = a->out_stream;
+        }
+        e = cudaMemcpyAsync(a->out_host, a->out, a->out_bytes, cudaMemcpyDeviceToHost, rs);
         if (e != cudaSuccess)
             return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: output readback: %s",
                              cudaGetErrorString(e));

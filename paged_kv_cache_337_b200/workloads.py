@@ -42,6 +42,7 @@ class DecodeSpec:
     pool_blocks: int = 0  # 0: ceil(pool_factor * blocks the sequences need)
     pool_factor: float = 1.1
     partition_size: int = 0  # 0: single pass
+    partition_size_e4m3: int = -1  # over an e4m3 cache (-1: partition_size)
     shared_prefix: bool = False
 
     @property
@@ -56,17 +57,26 @@ class DecodeSpec:
     def max_blocks_per_seq(self):
         return -(-self.len_hi // self.block_size)
 
+    def partition_for(self, fp8):
+        """Tokens per split-K partition over a 16-bit (fp8 False) or an e4m3
+        cache."""
+        if fp8 and self.partition_size_e4m3 >= 0:
+            return self.partition_size_e4m3
+        return self.partition_size
+
 
 # The five workloads (sizes as the benchmark configurations state them).
 TINY = DecodeSpec("tiny_s4_h8_d64_bs16_f16", 1001, 4, 8, 8, 64, 16, 1, 128, "f16",
                   pool_blocks=64)
 DECODE_7B = DecodeSpec("7b_s256_h32_d128_bs16_bf16", 1002, 256, 32, 32, 128, 16,
                        128, 2048, "bf16")
-# The GQA configuration fixes no partition size: 2048 tokens (about three
-# waves of CTAs for this batch on 148 SMs) measured fastest for both cache
-# types among 512-4096; the long-context configuration fixes 512.
+# The GQA configuration fixes no partition size.  Over a 16-bit cache 2048
+# tokens (about three waves of CTAs for this batch on 148 SMs) measured
+# fastest among 512-4096; an e4m3 token is half the bytes, and 4096 tokens
+# measured fastest there (2048: 4892 GB/s, 3072: 4943, 4096: 5277 on B200).
+# The long-context configuration fixes 512.
 GQA_70B = DecodeSpec("70b_gqa_s64_hq64_hkv8_d128_bs16_bf16", 1003, 64, 64, 8, 128,
-                     16, 512, 8192, "bf16", partition_size=2048)
+                     16, 512, 8192, "bf16", partition_size=2048, partition_size_e4m3=4096)
 LONG_BS32 = DecodeSpec("long_s8_l32768_hq32_hkv8_d128_bs32_bf16", 1004, 8, 32, 8,
                        128, 32, 32768, 32768, "bf16", partition_size=512)
 LONG_BS64 = DecodeSpec("long_s8_l32768_hq32_hkv8_d128_bs64_bf16", 1004, 8, 32, 8,

@@ -215,3 +215,37 @@ def test_fp8_argument_errors_raise(cuda_device):
     with pytest.raises(ValueError):
         _abi.pkv_decode_attention_fp8(q.clone(), q, kc.to(torch.bfloat16), kc, good, good,
                                       tables, lens, 1, 0.1)
+
+
+@pytest.mark.parametrize("work_list", [False, True], ids=["grid", "work_list"])
+def test_decode_fp8_gqa_shape_at_its_partition_size(work_list, cuda_device):
+    """The 70B-shaped GQA layout (64 query / 8 KV heads, block size 16) over
+    an e4m3 cache at the partition size that workload uses for e4m3 caches
+    (4096 tokens), lengths on and around the partition boundaries, on the
+    full grid and on the work list (items longest first)."""
+    from paged_kv_cache_337_b200 import workloads as W
+    P = W.GQA_70B.partition_for(True)
+    assert P == 4096
+    lens = [512, 4095, 4096, 4097, 8192, 6000, 1, 8191, 17, 4200]
+    p = fp8_problem(2024, 64, 8, 128, 16, lens, "bf16")
+    scale = 1.0 / np.sqrt(128)
+    dev = cuda_device
+    q = p["q"].to(dev)
+    kc, vc = p["kc"].to(dev), p["vc"].to(dev)
+    ks, vs = padded_scales(p["ks"], dev), padded_scales(p["vs"], dev)
+    tables = torch.as_tensor(p["tables"]).to(dev)
+    tl = torch.as_tensor(p["lens"]).to(dev)
+    max_len = int(max(lens))
+    out = torch.full_like(q, float("nan"))
+    ws = torch.empty(_abi.pkv_decode_workspace_bytes(len(lens), 64, max_len, P, 128),
+                     dtype=torch.uint8, device=dev)
+    err = torch.zeros(2, dtype=torch.int32, device=dev)
+    items = None
+    if work_list:
+        items = _abi.pkv_decode_work_items(lens, 8, max_len, P).to(dev)
+    _abi.pkv_decode_attention_fp8(out, q, kc, vc, ks, vs, tables, tl, max_len, scale, P, ws,
+                                  dev_error=err, work_items=items)
+    torch.cuda.synchronize()
+    want = oracle_decode_fp8(p, 8, 16, scale, "bf16")
+    assert err.tolist() == [0, 0]
+    assert tolerance_violation(out.cpu(), want, ATOL, RTOL) <= 0

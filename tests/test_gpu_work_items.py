@@ -157,13 +157,15 @@ def test_cache_driver_runs_the_work_list(work_list, cuda_device):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-@pytest.mark.parametrize("fp8", [False, True])
-def test_run_step_in_one_call_matches_the_separate_calls(fp8, cuda_device):
+@pytest.mark.parametrize("fp8,readback", [(False, False), (True, False), (False, True)],
+                         ids=["bf16", "e4m3", "bf16_readback_stream"])
+def test_run_step_in_one_call_matches_the_separate_calls(fp8, readback, cuda_device):
     """PagedKVCache.run_step (pkv_decode_step: upload, copies, write, attention
     and the output's copy to pinned host memory in one native call) gives
     bit for bit the output of upload_step + launch_step on an identical
     cache, through copy-on-write steps, and its host copy equals the
-    device output."""
+    device output, also when that copy runs on a readback stream (waited
+    for through an event recorded there)."""
     dev = cuda_device
     g = torch.Generator().manual_seed(12)
     S, Hq, Hkv, D, bs, P = 5, 16, 4, 128, 16, 64
@@ -193,7 +195,15 @@ def test_run_step_in_one_call_matches_the_separate_calls(fp8, cuda_device):
         pa, pb = a.prepare_step(ids), b.prepare_step(ids)
         assert pa["num_pairs"] == pb["num_pairs"] == (1 if step == 0 else 0)
         out_a = torch.empty_like(q)
-        a.run_step(pa, q, k, v, out_a, out_host=host)
+        host.fill_(float("nan"))
+        if readback:
+            rs = torch.cuda.Stream(dev)
+            a.run_step(pa, q, k, v, out_a, out_host=host, readback_stream=rs)
+            done = torch.cuda.Event()
+            done.record(rs)
+            done.synchronize()
+        else:
+            a.run_step(pa, q, k, v, out_a, out_host=host)
         b.upload_step(pb)
         out_b = b.launch_step(pb, q, k, v, torch.empty_like(q))
         torch.cuda.synchronize()
