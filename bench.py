@@ -634,6 +634,28 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
                 "readback_wait": round(1e3 * host["wait"] / steps, 4)}}
 
 
+def pool_memory(pool, ids, block_size, num_blocks, max_len):
+    """KV memory of the host pool ("PagedAttention 动态内存分页" page, 性能监控要点:
+    GPU memory utilisation): blocks handed out, the token slots they hold,
+    the tokens the sequences have written (logical: a shared block counts
+    once per sequence, so utilisation passes 1 with sharing), the slots of a
+    sequence's last block that hold none (at most block_size - 1), and the
+    slots a contiguous reservation of max_len tokens per sequence would
+    hold ("一文读懂vLLM..." page: what paging replaces)."""
+    free = pool.num_free()
+    used_blocks = num_blocks - free
+    tokens = sum(pool.num_tokens(s) for s in ids)
+    slots = used_blocks * block_size
+    waste = [(-pool.num_tokens(s)) % block_size for s in ids]
+    contiguous = len(ids) * max_len
+    return {"blocks_in_use": used_blocks, "blocks_free": free, "slots_in_use": slots,
+            "tokens": tokens, "utilization": round(tokens / slots, 4) if slots else None,
+            "empty_slots_per_sequence_max": max(waste) if waste else 0,
+            "empty_slots_per_sequence_mean": round(sum(waste) / len(waste), 2) if waste else 0,
+            "contiguous_prealloc_slots": contiguous,
+            "contiguous_prealloc_utilization": round(tokens / contiguous, 4) if contiguous else None}
+
+
 def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc=True):
     """One decode workload: returns its JSON line (rank 0) or None."""
     from paged_kv_cache_337_b200 import _abi
@@ -790,6 +812,7 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
                "sample": "first %d of %d sequences (all %d query heads), decode step "
                          "repeated %d times, %.1f s" % (n, S, Hq, reps, secs)}
     alloc = allocator_latency(spec, lens0, order.tolist(), rank) if with_alloc else None
+    memory = pool_memory(cache.pool, ids, bs, nb, spec.len_hi)
 
     if rank != 0:
         return None
@@ -822,6 +845,7 @@ def run_pkv(args, spec, world, rank, local, fp8=False, with_cpu=True, with_alloc
                      "traffic": traffic, "kernel": "paged_decode_kernel",
                      "peak_source": peak_kind},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clock_info,
+        "memory": memory,
     }
     if alloc is not None:
         line["allocator"] = alloc
@@ -1313,6 +1337,8 @@ def run_shared_prefix(args, world, rank, local):
             cache.pool.append(s)
     steady = snapshot()
     steady_res, _ = time_state(steady)
+    memory = pool_memory(cache.pool, ids, bs, inp.num_blocks,
+                         int(inp.prompt_lens.max()) + int(inp.diverge.max()) + 1)
     clock_info = clocks.stop() if clocks else None
     peak, peak_kind = measured_peak()
     if rank == 0:
@@ -1328,7 +1354,7 @@ def run_shared_prefix(args, world, rank, local):
             "fork_step": fork_res, "steady_step": steady_res,
             "decode_tok_s": round(world * S / (fork_res["ms_per_step"] * 1e-3), 1),
             "peak_gbs": peak, "peak_source": peak_kind, "gpu_launches": launches,
-            "clocks": clock_info,
+            "clocks": clock_info, "memory": memory,
         }
         return line
     return None
