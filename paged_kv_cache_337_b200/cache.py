@@ -337,6 +337,7 @@ class PagedKVCache:
         a.work_items = st["d_items"].data_ptr() if items >= 0 else None
         a.num_items = max(items, 0)
         a.out_host, a.out_bytes = None, 0
+        a.out_stream, a.out_event = None, None
         _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
                     "pkv_decode_step")
         if st["consumed"] is None:
