@@ -536,10 +536,10 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     pinned memory (on a second stream, into one of two input buffers), the
     host pool reserves the slots and plans the work list
     (PagedKVCache.prepare_step, one native call), and one more native call
-    (PagedKVCache.run_step) uploads the metadata, runs the kernels and
-    copies the attention output back to pinned host memory on a readback
-    stream, where the copy overlaps the next step's kernels; the host waits
-    for it.
+    (PagedKVCache.run_step) uploads the metadata on the input-upload
+    stream, runs the kernels and copies the attention output back to pinned
+    host memory on a readback stream, where the copy overlaps the next
+    step's kernels; the host waits for it.
 
     serial: the host waits for step i's output before it enqueues step i+1
     (the pool's work for step i+1 and its input upload still overlap step
@@ -580,7 +580,7 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
         dq, dk, dv = views[b]
         # metadata upload, copies, slot write, attention and readback: one call
         cache.run_step(prep, dq, dk, dv, outs[o], out_host=houts[o], stream=stream,
-                       readback_stream=readback_stream)
+                       readback_stream=readback_stream, upload_stream=copy_stream)
         ev_used[b].record(stream)
         ev_out[o].record(readback_stream)
 

@@ -313,7 +313,14 @@ PKV_API int pkv_step_prepare(pkv_pool* pool, int n, const int64_t* seq_ids, int6
  *   1. meta_bytes from meta_host to meta_device (cudaMemcpyAsync; pinned
  *      host memory keeps it asynchronous; 0 bytes: none) — typically the
  *      step's slots, pairs, tables, lengths and work list in one buffer,
- *      which the pointers below then point into;
+ *      which the pointers below then point into.  With meta_stream not
+ *      NULL the copy goes on meta_stream instead, after meta_stream waits
+ *      for meta_after (when not NULL: an event the caller recorded after
+ *      the last launch that read meta_device), and `stream` waits for
+ *      meta_event, which the call records on meta_stream after the copy.
+ *      A copy on the compute stream waits, in the copy engine, behind the
+ *      previous step's output copy; on a stream of its own it is done
+ *      while the previous step computes;
  *   2. pkv_copy_blocks (or _fp8) of the num_pairs cow_pairs (0: none);
  *   3. pkv_write_slots (or _fp8) of the num_tokens new rows (0: none);
  *   4. pkv_decode_attention (or _fp8), over work_items when that is not
@@ -371,6 +378,9 @@ typedef struct pkv_decode_step_args {
     int32_t* dev_error;
     cudaStream_t out_stream; /* NULL: the readback goes on `stream` */
     cudaEvent_t out_event;   /* used with out_stream */
+    cudaStream_t meta_stream; /* NULL: the metadata upload goes on `stream` */
+    cudaEvent_t meta_event;   /* used with meta_stream (PKV_ERR_INVALID when NULL) */
+    cudaEvent_t meta_after;   /* optional, with meta_stream */
 } pkv_decode_step_args;
 
 PKV_API int pkv_decode_step(const pkv_decode_step_args* args, cudaStream_t stream);

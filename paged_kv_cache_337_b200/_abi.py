@@ -114,7 +114,8 @@ class DecodeStepArgs(C.Structure):
                 ("workspace", _p), ("workspace_bytes", _sz),
                 ("work_items", _p), ("num_items", _i),
                 ("out_host", _p), ("out_bytes", _sz),
-                ("dtype", _i), ("dev_error", _p), ("out_stream", _p), ("out_event", _p)]
+                ("dtype", _i), ("dev_error", _p), ("out_stream", _p), ("out_event", _p),
+                ("meta_stream", _p), ("meta_event", _p), ("meta_after", _p)]
 
 
 class PkvError(RuntimeError):

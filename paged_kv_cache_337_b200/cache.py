@@ -264,7 +264,7 @@ class PagedKVCache:
         self._seen.add(sig)
 
     def run_step(self, prep, query, key, value, out, out_host=None, stream=None,
-                 readback_stream=None):
+                 readback_stream=None, upload_stream=None):
         """Device part of a prepared decode step in one native call
         (pkv_decode_step): the metadata upload, the copy-on-write copies, the
         slot write, decode attention and, with out_host (pinned host memory
@@ -273,7 +273,11 @@ class PagedKVCache:
         when readback_stream is given: it then runs there once the attention
         is done, overlapping what comes next on `stream`.  The caller reads
         out_host, and writes `out` again, only after that copy (an event
-        recorded on readback_stream after this call)."""
+        recorded on readback_stream after this call).  With upload_stream,
+        the metadata upload goes there (after the last launch that read this
+        staging bank) and `stream` waits for it: on the compute stream it
+        would wait in the copy engine behind the previous step's readback,
+        on a stream of its own it lands while the previous step computes."""
         st = prep["st"]
         S = len(st["ids"])
         self._check_step_tensors(query, key, value, out, out_host)
@@ -297,6 +301,15 @@ class PagedKVCache:
         else:
             a.out_host, a.out_bytes = None, 0
         a.out_stream, a.out_event = None, None
+        a.meta_stream, a.meta_event, a.meta_after = None, None, None
+        if upload_stream is not None and a.meta_bytes > 0:
+            if st.get("meta_up") is None:
+                st["meta_up"] = torch.cuda.Event()
+                st["meta_up"].record(upload_stream)  # the handle exists once recorded
+            a.meta_stream = upload_stream.cuda_stream
+            a.meta_event = st["meta_up"].cuda_event
+            if st["consumed"] is not None:
+                a.meta_after = st["consumed"].cuda_event
         if out_host is not None and readback_stream is not None:
             if st.get("attended") is None:
                 st["attended"] = torch.cuda.Event()
@@ -338,6 +351,7 @@ class PagedKVCache:
         a.num_items = max(items, 0)
         a.out_host, a.out_bytes = None, 0
         a.out_stream, a.out_event = None, None
+        a.meta_stream, a.meta_event, a.meta_after = None, None, None
         _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
                     "pkv_decode_step")
         if st["consumed"] is None:

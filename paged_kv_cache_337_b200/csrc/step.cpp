@@ -45,8 +45,22 @@ extern "C" int pkv_decode_step(const pkv_decode_step_args* a, cudaStream_t strea
     if (a->meta_bytes > 0) {
         PKV_REQUIRE(a->meta_host && a->meta_device, PKV_ERR_INVALID,
                     "pkv_decode_step: NULL metadata buffer");
+        cudaStream_t ms = stream;
+        if (a->meta_stream != nullptr) {
+            PKV_REQUIRE(a->meta_event != nullptr, PKV_ERR_INVALID,
+                        "pkv_decode_step: meta_stream without meta_event");
+            ms = a->meta_stream;
+            e = a->meta_after != nullptr ? cudaStreamWaitEvent(ms, a->meta_after, 0) : cudaSuccess;
+            if (e != cudaSuccess)
+                return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: metadata stream: %s",
+                                 cudaGetErrorString(e));
+        }
         e = cudaMemcpyAsync(a->meta_device, a->meta_host, a->meta_bytes, cudaMemcpyHostToDevice,
-                            stream);
+                            ms);
+        if (e == cudaSuccess && a->meta_stream != nullptr) {
+            e = cudaEventRecord(a->meta_event, ms);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, a->meta_event, 0);
+        }
         if (e != cudaSuccess)
             return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: metadata upload: %s",
                              cudaGetErrorString(e));

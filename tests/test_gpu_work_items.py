@@ -158,14 +158,15 @@ def test_cache_driver_runs_the_work_list(work_list, cuda_device):
 
 
 @pytest.mark.parametrize("fp8,readback", [(False, False), (True, False), (False, True)],
-                         ids=["bf16", "e4m3", "bf16_readback_stream"])
+                         ids=["bf16", "e4m3", "bf16_readback_and_upload_streams"])
 def test_run_step_in_one_call_matches_the_separate_calls(fp8, readback, cuda_device):
     """PagedKVCache.run_step (pkv_decode_step: upload, copies, write, attention
     and the output's copy to pinned host memory in one native call) gives
     bit for bit the output of upload_step + launch_step on an identical
     cache, through copy-on-write steps, and its host copy equals the
     device output, also when that copy runs on a readback stream (waited
-    for through an event recorded there)."""
+    for through an event recorded there) and the metadata upload on an
+    upload stream."""
     dev = cuda_device
     g = torch.Generator().manual_seed(12)
     S, Hq, Hkv, D, bs, P = 5, 16, 4, 128, 16, 64
@@ -197,8 +198,8 @@ def test_run_step_in_one_call_matches_the_separate_calls(fp8, readback, cuda_dev
         out_a = torch.empty_like(q)
         host.fill_(float("nan"))
         if readback:
-            rs = torch.cuda.Stream(dev)
-            a.run_step(pa, q, k, v, out_a, out_host=host, readback_stream=rs)
+            rs, us = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+            a.run_step(pa, q, k, v, out_a, out_host=host, readback_stream=rs, upload_stream=us)
             done = torch.cuda.Event()
             done.record(rs)
             done.synchronize()
