@@ -533,13 +533,15 @@ def allocator_latency(spec, lens, order, rank):
 def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     """The decode step end to end through the public step API, from pinned
     host memory.  Per step: the step's q, k and v go up in one copy from
-    pinned memory (on a second stream, into one of two input buffers), the
-    host pool reserves the slots and plans the work list
-    (PagedKVCache.prepare_step, one native call), and one more native call
-    (PagedKVCache.run_step) uploads the metadata on the input-upload
-    stream, runs the kernels and copies the attention output back to pinned
-    host memory on a readback stream, where the copy overlaps the next
-    step's kernels; the host waits for it.
+    pinned memory (on an upload stream, into one of two input buffers,
+    issued while the previous step computes), the host pool reserves the
+    slots and plans the work list (PagedKVCache.prepare_step, one native
+    call), and one more native call (PagedKVCache.run_step) uploads the
+    metadata on the upload stream, runs the kernels and copies the
+    attention output back to pinned host memory on a readback stream,
+    where the copy overlaps the next step's kernels; the host waits for it.
+    (run_step can take the q/k/v copy too, `inputs=`; issued with the step
+    rather than a step ahead, it measured slower on the shortest steps.)
 
     serial: the host waits for step i's output before it enqueues step i+1
     (the pool's work for step i+1 and its input upload still overlap step
@@ -558,7 +560,7 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
     nout = 2 if pipelined else 1
     outs = [torch.empty((S, Hq, D), dtype=dt, device=dev) for _ in range(nout)]
     houts = [torch.empty((S, Hq, D), dtype=dt).pin_memory() for _ in range(nout)]
-    copy_stream = torch.cuda.Stream(dev)
+    upload_stream = torch.cuda.Stream(dev)
     readback_stream = torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
     ev_used = [torch.cuda.Event() for _ in range(2)]  # the step using buffer b done
@@ -580,17 +582,17 @@ def run_e2e(args, spec, cache, ids, steps, stream, P, fp8, world, dev):
         dq, dk, dv = views[b]
         # metadata upload, copies, slot write, attention and readback: one call
         cache.run_step(prep, dq, dk, dv, outs[o], out_host=houts[o], stream=stream,
-                       readback_stream=readback_stream, upload_stream=copy_stream)
+                       readback_stream=readback_stream, upload_stream=upload_stream)
         ev_used[b].record(stream)
         ev_out[o].record(readback_stream)
 
     def upload_inputs(i):
         b = i % 2
-        with torch.cuda.stream(copy_stream):
+        with torch.cuda.stream(upload_stream):
             if i >= 2:
-                copy_stream.wait_event(ev_used[b])  # step i - 2 done with the buffer
+                upload_stream.wait_event(ev_used[b])  # step i - 2 done with the buffer
             d_in[b].copy_(h_in[i % 2], non_blocking=True)
-            ev_in[b].record(copy_stream)
+            ev_in[b].record(upload_stream)
 
     barrier(world)
     torch.cuda.synchronize(dev)

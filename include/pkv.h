@@ -310,6 +310,10 @@ PKV_API int pkv_step_prepare(pkv_pool* pool, int n, const int64_t* seq_ids, int6
 
 /*
  * Device part, enqueued on `stream` in this order:
+ *   0. in_bytes from in_host to in_device (cudaMemcpyAsync; 0 bytes:
+ *      none) — typically the step's queries and new key/value rows, which
+ *      query, key and value then point into; on meta_stream when that is
+ *      set, like step 1;
  *   1. meta_bytes from meta_host to meta_device (cudaMemcpyAsync; pinned
  *      host memory keeps it asynchronous; 0 bytes: none) — typically the
  *      step's slots, pairs, tables, lengths and work list in one buffer,
@@ -378,9 +382,12 @@ typedef struct pkv_decode_step_args {
     int32_t* dev_error;
     cudaStream_t out_stream; /* NULL: the readback goes on `stream` */
     cudaEvent_t out_event;   /* used with out_stream */
-    cudaStream_t meta_stream; /* NULL: the metadata upload goes on `stream` */
+    cudaStream_t meta_stream; /* NULL: the uploads go on `stream` */
     cudaEvent_t meta_event;   /* used with meta_stream (PKV_ERR_INVALID when NULL) */
     cudaEvent_t meta_after;   /* optional, with meta_stream */
+    const void* in_host;      /* step 0: pinned host source */
+    void* in_device;          /* step 0: device destination */
+    size_t in_bytes;          /* 0: no input upload */
 } pkv_decode_step_args;
 
 PKV_API int pkv_decode_step(const pkv_decode_step_args* args, cudaStream_t stream);

@@ -115,7 +115,8 @@ class DecodeStepArgs(C.Structure):
                 ("work_items", _p), ("num_items", _i),
                 ("out_host", _p), ("out_bytes", _sz),
                 ("dtype", _i), ("dev_error", _p), ("out_stream", _p), ("out_event", _p),
-                ("meta_stream", _p), ("meta_event", _p), ("meta_after", _p)]
+                ("meta_stream", _p), ("meta_event", _p), ("meta_after", _p),
+                ("in_host", _p), ("in_device", _p), ("in_bytes", _sz)]
 
 
 class PkvError(RuntimeError):

@@ -264,7 +264,7 @@ class PagedKVCache:
         self._seen.add(sig)
 
     def run_step(self, prep, query, key, value, out, out_host=None, stream=None,
-                 readback_stream=None, upload_stream=None):
+                 readback_stream=None, upload_stream=None, inputs=None):
         """Device part of a prepared decode step in one native call
         (pkv_decode_step): the metadata upload, the copy-on-write copies, the
         slot write, decode attention and, with out_host (pinned host memory
@@ -277,7 +277,13 @@ class PagedKVCache:
         the metadata upload goes there (after the last launch that read this
         staging bank) and `stream` waits for it: on the compute stream it
         would wait in the copy engine behind the previous step's readback,
-        on a stream of its own it lands while the previous step computes."""
+        on a stream of its own it lands while the previous step computes.
+        inputs=(host, device): a pinned host tensor copied into a device
+        tensor of the same size first (on upload_stream when given), e.g.
+        the step's query, key and value rows, which query, key and value
+        then view; the copy waits, like the metadata's, for the last launch
+        that read this staging bank, so the caller alternates its input
+        buffers as the banks alternate (one per step, two of them)."""
         st = prep["st"]
         S = len(st["ids"])
         self._check_step_tensors(query, key, value, out, out_host)
@@ -302,7 +308,20 @@ class PagedKVCache:
             a.out_host, a.out_bytes = None, 0
         a.out_stream, a.out_event = None, None
         a.meta_stream, a.meta_event, a.meta_after = None, None, None
-        if upload_stream is not None and a.meta_bytes > 0:
+        a.in_host, a.in_device, a.in_bytes = None, None, 0
+        if inputs is not None:
+            h, d = inputs
+            nbytes = d.numel() * d.element_size()
+            key_ = ("inputs", h.data_ptr(), d.data_ptr(), nbytes)
+            if key_ not in self._seen:  # checked once per pair of buffers
+                if (h.device.type != "cpu" or not h.is_pinned() or not h.is_contiguous() or
+                        d.device != self.device or not d.is_contiguous() or
+                        h.numel() * h.element_size() != nbytes):
+                    raise ValueError("decode step: inputs must be a pinned host tensor and a "
+                                     "contiguous device tensor of the same size")
+                self._seen.add(key_)
+            a.in_host, a.in_device, a.in_bytes = h.data_ptr(), d.data_ptr(), nbytes
+        if upload_stream is not None and (a.meta_bytes > 0 or a.in_bytes > 0):
             if st.get("meta_up") is None:
                 st["meta_up"] = torch.cuda.Event()
                 st["meta_up"].record(upload_stream)  # the handle exists once recorded
@@ -352,6 +371,7 @@ class PagedKVCache:
         a.out_host, a.out_bytes = None, 0
         a.out_stream, a.out_event = None, None
         a.meta_stream, a.meta_event, a.meta_after = None, None, None
+        a.in_host, a.in_device, a.in_bytes = None, None, 0
         _abi._check(_abi.lib().pkv_decode_step(C.byref(a), C.c_void_p(s_.cuda_stream)),
                     "pkv_decode_step")
         if st["consumed"] is None:

@@ -42,27 +42,40 @@ extern "C" int pkv_decode_step(const pkv_decode_step_args* a, cudaStream_t strea
     PKV_REQUIRE(a != nullptr, PKV_ERR_INVALID, "pkv_decode_step: NULL arguments");
     const bool fp8 = a->k_scale != nullptr || a->v_scale != nullptr;
     cudaError_t e;
+    // steps 0 and 1: the uploads, on meta_stream when the caller gives one
+    const bool uploads = a->in_bytes > 0 || a->meta_bytes > 0;
+    cudaStream_t us = stream;
+    if (uploads && a->meta_stream != nullptr) {
+        PKV_REQUIRE(a->meta_event != nullptr, PKV_ERR_INVALID,
+                    "pkv_decode_step: meta_stream without meta_event");
+        us = a->meta_stream;
+        e = a->meta_after != nullptr ? cudaStreamWaitEvent(us, a->meta_after, 0) : cudaSuccess;
+        if (e != cudaSuccess)
+            return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: upload stream: %s",
+                             cudaGetErrorString(e));
+    }
+    if (a->in_bytes > 0) {
+        PKV_REQUIRE(a->in_host && a->in_device, PKV_ERR_INVALID,
+                    "pkv_decode_step: NULL input buffer");
+        e = cudaMemcpyAsync(a->in_device, a->in_host, a->in_bytes, cudaMemcpyHostToDevice, us);
+        if (e != cudaSuccess)
+            return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: input upload: %s",
+                             cudaGetErrorString(e));
+    }
     if (a->meta_bytes > 0) {
         PKV_REQUIRE(a->meta_host && a->meta_device, PKV_ERR_INVALID,
                     "pkv_decode_step: NULL metadata buffer");
-        cudaStream_t ms = stream;
-        if (a->meta_stream != nullptr) {
-            PKV_REQUIRE(a->meta_event != nullptr, PKV_ERR_INVALID,
-                        "pkv_decode_step: meta_stream without meta_event");
-            ms = a->meta_stream;
-            e = a->meta_after != nullptr ? cudaStreamWaitEvent(ms, a->meta_after, 0) : cudaSuccess;
-            if (e != cudaSuccess)
-                return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: metadata stream: %s",
-                                 cudaGetErrorString(e));
-        }
         e = cudaMemcpyAsync(a->meta_device, a->meta_host, a->meta_bytes, cudaMemcpyHostToDevice,
-                            ms);
-        if (e == cudaSuccess && a->meta_stream != nullptr) {
-            e = cudaEventRecord(a->meta_event, ms);
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, a->meta_event, 0);
-        }
+                            us);
         if (e != cudaSuccess)
             return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: metadata upload: %s",
+                             cudaGetErrorString(e));
+    }
+    if (uploads && a->meta_stream != nullptr) {
+        e = cudaEventRecord(a->meta_event, us);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, a->meta_event, 0);
+        if (e != cudaSuccess)
+            return pkv::fail(PKV_ERR_CUDA, "pkv_decode_step: upload event: %s",
                              cudaGetErrorString(e));
     }
     int st = PKV_OK;

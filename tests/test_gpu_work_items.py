@@ -165,8 +165,8 @@ def test_run_step_in_one_call_matches_the_separate_calls(fp8, readback, cuda_dev
     bit for bit the output of upload_step + launch_step on an identical
     cache, through copy-on-write steps, and its host copy equals the
     device output, also when that copy runs on a readback stream (waited
-    for through an event recorded there) and the metadata upload on an
-    upload stream."""
+    for through an event recorded there) and the step's inputs and metadata
+    go up on an upload stream inside the call."""
     dev = cuda_device
     g = torch.Generator().manual_seed(12)
     S, Hq, Hkv, D, bs, P = 5, 16, 4, 128, 16, 64
@@ -198,8 +198,15 @@ def test_run_step_in_one_call_matches_the_separate_calls(fp8, readback, cuda_dev
         out_a = torch.empty_like(q)
         host.fill_(float("nan"))
         if readback:
+            # q, k and v go up from one pinned buffer inside the call
             rs, us = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-            a.run_step(pa, q, k, v, out_a, out_host=host, readback_stream=rs, upload_stream=us)
+            h_in = torch.cat([q.flatten(), k.flatten(), v.flatten()]).cpu().pin_memory()
+            d_in = torch.empty_like(h_in, device=dev)
+            nq, nk = q.numel(), k.numel()
+            dq, dk = d_in[:nq].view(q.shape), d_in[nq:nq + nk].view(k.shape)
+            dv = d_in[nq + nk:].view(v.shape)
+            a.run_step(pa, dq, dk, dv, out_a, out_host=host, readback_stream=rs,
+                       upload_stream=us, inputs=(h_in, d_in))
             done = torch.cuda.Event()
             done.record(rs)
             done.synchronize()
