@@ -38,6 +38,12 @@ def test_default_decode_line(cuda_device):
     assert e["value"] > 0 and e["unit"] == "GB/s"
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert d["gpu_launches"] >= 2 * d["steps"]  # slot write + attention per step
+    m = d["memory"]  # the host pool's KV memory after the steps
+    assert 0 < m["blocks_in_use"] <= d["config"]["pool_blocks"]
+    assert m["slots_in_use"] == 16 * m["blocks_in_use"]
+    assert 0.9 < m["utilization"] <= 1.0  # no sharing: at most 15 empty slots a sequence
+    assert m["empty_slots_per_sequence_max"] <= 15
+    assert m["contiguous_prealloc_utilization"] < m["utilization"]
     c = d["clocks"]
     assert c is None or (c["sm_max_mhz"] > 0 and isinstance(c["reasons"], list))
 
