@@ -105,3 +105,18 @@ def test_step_args_layout_matches_the_header():
     got = dict(zip(out[0::2], map(int, out[1::2])))
     assert got.pop("size") == C.sizeof(_abi.DecodeStepArgs)
     assert got == {f: getattr(_abi.DecodeStepArgs, f).offset for f in fields}
+
+
+def test_decode_step_rejects_an_upload_stream_without_its_event():
+    """pkv_decode_step returns PKV_ERR_INVALID before any device work when
+    the uploads go on meta_stream but no meta_event is given, or when an
+    input upload has no buffers.  (The stream value is never used: the
+    check comes first.)"""
+    a = _abi.DecodeStepArgs()
+    host = (C.c_uint8 * 64)()
+    a.meta_host, a.meta_device, a.meta_bytes = C.addressof(host), C.addressof(host), 64
+    a.meta_stream, a.meta_event = 0x1, None
+    assert _abi.lib().pkv_decode_step(C.byref(a), None) == _abi.PKV_ERR_INVALID
+    b = _abi.DecodeStepArgs()
+    b.in_bytes, b.in_host, b.in_device = 64, None, None
+    assert _abi.lib().pkv_decode_step(C.byref(b), None) == _abi.PKV_ERR_INVALID
