@@ -16,8 +16,9 @@
 // tiles and output.
 // The work runs on the 5th-generation tensor cores with the accumulators in
 // tensor memory:
-//   - a producer warp brings 64-key K and V tiles through a 4-stage ring
-//     (one TMA box per 16 slots of a block and per 64-dim half);
+//   - two producer warps, one for K and one for V, bring 64-key tiles
+//     through a 4-stage ring (one TMA box per 16 slots of a block and per
+//     64-dim half);
 //   - an MMA warp issues, per key tile, S = Q K^T for both Q tiles (M 128,
 //     N 64, K 16 steps; Q and K from shared memory) into tensor memory,
 //     then O += P V for each tile as its P is ready (P read from tensor
@@ -58,7 +59,8 @@ constexpr int kQBytes = kQTiles * kQTileBytes;
 constexpr int kBoxKeys = 16;                        // slots per TMA box
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4 * kQTiles;
 constexpr int kQWarp0 = kSoftmaxWarp0 + kSoftmaxWarps, kQWarps = 4;
-constexpr int kThreads = (kQWarp0 + kQWarps) * 32;
+constexpr int kVProducerWarp = kQWarp0 + kQWarps;
+constexpr int kThreads = (kVProducerWarp + 1) * 32;
 // tensor-memory columns per Q tile t: two S buffers (64 columns each; P
 // high | P low, 32 each, written over S once it is read) at 256 t and
 // 256 t + 64, O at 256 t + 128; key tile j uses S buffer j % 2
@@ -188,15 +190,19 @@ __device__ Item decode_item(const PrefillParams& p, int idx, bool report) {
     return it;
 }
 
-// Producer: warp 0.  A box past the context still loads a block (the last
-// one) so that every stage receives its full byte count; those rows are
-// masked (K) or zeroed (V) downstream.  The block ids come from the Block
-// Table one warp-wide load per eight key tiles (lane i: the id of box i of
-// the window), handed to lane 0, which issues the TMA loads, by shuffles.
-// The ring position runs on across items, so the next item's tiles load
-// while the current one finishes.
+// Producers: warp 0 loads the K tiles, the last warp the V tiles, into the
+// same ring stages (each stage's full barrier takes one arrival per
+// producer with its byte count).  A box past the context still loads a
+// block (the last one) so that every stage receives its full byte count;
+// those rows are masked (K) or zeroed (V) downstream.  The block ids come
+// from the Block Table one warp-wide load per eight key tiles (lane i: the
+// id of box i of the window), handed by shuffles to the lanes that issue
+// the loads: eight lanes, one box each (a TMA box costs its issuing lane
+// less when several lanes of the warp issue one each).  The ring position
+// runs on across items, so the next item's tiles load while the current
+// one finishes.
 __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const PrefillParams& p,
-                        uint8_t* stages, const Bars& b, int lane, bool* failed) {
+                        uint8_t* stages, const Bars& b, int lane, bool is_v, bool* failed) {
     constexpr int kBoxes = kKeys / kBoxKeys;       // TMA boxes per key tile and 64-dim half
     constexpr int kWindowTiles = 32 / kBoxes;      // key tiles per warp-wide block-id load
     const int bs = p.block_size;
@@ -224,35 +230,23 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
                 *failed = true;
                 break;
             }
-            int phys[kBoxes];
-#pragma unroll
-            for (int bx = 0; bx < kBoxes; ++bx)
-                phys[bx] = __shfl_sync(0xffffffffu, phys_lane, (j % kWindowTiles) * kBoxes + bx);
-            if (lane == 0) {
-                uint8_t* kdst = stages + st * kStageBytes;
-                uint8_t* vdst = kdst + kTileBytes;
-                mbar_arrive_expect_tx(&b.kv_full[st], kStageBytes);
-#pragma unroll
-                for (int bx = 0; bx < kBoxes; ++bx) {
-                    const int key0 = j * kKeys + bx * kBoxKeys;
-                    const int off = key0 < it.L ? key0 % bs : 0;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if constexpr (kL2Hints) {
-                            tma_load_5d_hint(kdst + h * kHalfBytes + bx * kBoxKeys * 128,
-                                             &kmap, &b.kv_full[st], 0, it.kvh, off, h, phys[bx],
-                                             keep);
-                            tma_load_5d_hint(vdst + h * kHalfBytes + bx * kBoxKeys * 128,
-                                             &vmap, &b.kv_full[st], 0, it.kvh, off, h, phys[bx],
-                                             keep);
-                        } else {
-                            tma_load_5d(kdst + h * kHalfBytes + bx * kBoxKeys * 128, &kmap,
-                                        &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
-                            tma_load_5d(vdst + h * kHalfBytes + bx * kBoxKeys * 128, &vmap,
-                                        &b.kv_full[st], 0, it.kvh, off, h, phys[bx]);
-                        }
-                    }
-                }
+            const int phys_box =
+                __shfl_sync(0xffffffffu, phys_lane, (j % kWindowTiles) * kBoxes + ((lane >> 1) & 3));
+            // one lane per box of this warp's operand (box lane / 2 of the
+            // tile, 64-dim half lane % 2)
+            if (lane == 0) mbar_arrive_expect_tx(&b.kv_full[st], kTileBytes);
+            __syncwarp();
+            if (lane < 2 * kBoxes) {
+                const int bx = lane >> 1, h = lane & 1;
+                const int key0 = j * kKeys + bx * kBoxKeys;
+                const int off = key0 < it.L ? key0 % bs : 0;
+                uint8_t* dst = stages + st * kStageBytes + (is_v ? kTileBytes : 0) +
+                               h * kHalfBytes + bx * kBoxKeys * 128;
+                const CUtensorMap* map = is_v ? &vmap : &kmap;
+                if constexpr (kL2Hints)
+                    tma_load_5d_hint(dst, map, &b.kv_full[st], 0, it.kvh, off, h, phys_box, keep);
+                else
+                    tma_load_5d(dst, map, &b.kv_full[st], 0, it.kvh, off, h, phys_box);
             }
             __syncwarp();
             ++gk;
@@ -737,7 +731,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     if (threadIdx.x == 32 * kMmaWarp) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&b.kv_full[i], 1);
+            mbar_init(&b.kv_full[i], 2);  // the K and the V producer
             mbar_init(&b.kv_empty[i], 1);
             mbar_init(&b.v_ready[i], kQWarps);
         }
@@ -762,12 +756,12 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     const uint32_t tmem = *tmem_slot;
 
     bool failed = false;
-    if (warp == kProducerWarp)
-        produce(kmap, vmap, p, stages, b, lane, &failed);
+    if (warp == kProducerWarp || warp == kVProducerWarp)
+        produce(kmap, vmap, p, stages, b, lane, warp == kVProducerWarp, &failed);
     else if (warp == kMmaWarp)
         issue_mmas<std::is_same<T, __nv_bfloat16>::value>(p, b, tmem, smem_addr(qsm), stages,
                                                           vflags, &failed);
-    else if (warp >= kQWarp0)
+    else if (warp >= kQWarp0 && warp < kQWarp0 + kQWarps)
         stage_q<T>(p, b, qsm, stages, vflags, warp - kQWarp0, lane, &failed);
     else
         softmax_rows<T>(p, b, tmem, stages, vflags, warp, lane, &failed);
