@@ -19,11 +19,12 @@
 //   - two producer warps, one for K and one for V, bring 64-key tiles
 //     through a 4-stage ring (one TMA box per 16 slots of a block and per
 //     64-dim half);
-//   - an MMA warp issues, per key tile, S = Q K^T for both Q tiles (M 128,
+//   - two MMA warps, one per Q tile, issue per key tile S = Q K^T (M 128,
 //     N 64, K 16 steps; Q and K from shared memory) into tensor memory,
-//     then O += P V for each tile as its P is ready (P read from tensor
-//     memory, V from shared memory as an MN-major B operand), so that the
-//     tensor cores work on one tile while the other tile's softmax runs;
+//     then O += P V as the tile's P is ready (P read from tensor memory, V
+//     from shared memory as an MN-major B operand), so that the tensor
+//     cores work on one tile while the other tile's softmax runs, and
+//     neither tile's issue waits behind the other's P;
 //   - eight softmax warps, four per Q tile (one tensor-memory lane quarter
 //     each, one row per thread), read S, apply the causal mask, keep the
 //     running max and sum, write P over S (one f16 rounding; a bf16 high
@@ -59,8 +60,8 @@ constexpr int kQBytes = kQTiles * kQTileBytes;
 constexpr int kBoxKeys = 16;                        // slots per TMA box
 constexpr int kProducerWarp = 0, kMmaWarp = 1, kSoftmaxWarp0 = 2, kSoftmaxWarps = 4 * kQTiles;
 constexpr int kQWarp0 = kSoftmaxWarp0 + kSoftmaxWarps, kQWarps = 4;
-constexpr int kVProducerWarp = kQWarp0 + kQWarps;
-constexpr int kThreads = (kVProducerWarp + 1) * 32;
+constexpr int kVProducerWarp = kQWarp0 + kQWarps, kMmaWarpB = kVProducerWarp + 1;
+constexpr int kThreads = (kMmaWarpB + 1) * 32;
 // tensor-memory columns per Q tile t: two S buffers (64 columns each; P
 // high | P low, 32 each, written over S once it is read) at 256 t and
 // 256 t + 64, O at 256 t + 128; key tile j uses S buffer j % 2
@@ -258,12 +259,15 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
             mbar_wait_bounded(&b.kv_full[q % kStages], (q / kStages) & 1);
 }
 
-// MMA issuer: warp 1, in step; one elected lane issues each MMA and commit,
-// the descriptors stay warp-uniform.  g counts key tiles over all items: it
+// MMA issuers: warp 1 for Q tile 0 and the last warp for Q tile 1, each in
+// step; one elected lane issues each MMA and commit, the descriptors stay
+// warp-uniform.  A commit tracks the MMAs of the thread that executes it,
+// so the barriers both tiles release (a stage's kv_empty, q_free, drain)
+// take one commit from each warp.  g counts key tiles over all items: it
 // picks the ring stage (g mod kStages) and the S buffer (g mod 2).
 template <bool BF16>
 __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem, uint32_t qaddr,
-                           uint8_t* stages, const uint32_t* vflags, bool* failed) {
+                           uint8_t* stages, const uint32_t* vflags, int t, bool* failed) {
     // one lane issues every MMA and every commit (a commit tracks the MMAs
     // of the thread that executes it)
     const bool leader = tc::elect_one();
@@ -323,11 +327,11 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
         tc::fence_after_sync();
         return true;
     };
-    // Per item, S runs two key tiles ahead of P V, so that a tile's softmax
-    // finds its next S ready, and the tensor cores take one tile's P V and
-    // S while the other tile's softmax runs:
-    //   S_A(0) S_B(0) S_A(1) S_B(1) | P_A(j): PV_A(j) S_A(j+2) | P_B(j): PV_B(j) S_B(j+2)
-    // After the item's last S, q_free lets the Q warp stage the next item;
+    // Per item, S runs two key tiles ahead of P V, so that the tile's
+    // softmax finds its next S ready, and the tensor cores take this tile's
+    // P V and S while the other tile's softmax runs:
+    //   S(0) S(1) | P(j): PV(j) S(j+2)
+    // After both tiles' last S, q_free lets the Q warps stage the next item;
     // before an item's first P V overwrites O, o_free says the previous
     // item's output has been read.
     int g0 = 0;  // first key tile of the item, counted over all items
@@ -342,35 +346,24 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
         for (int j = 0; j < min(nt, 2); ++j) {
             const int g = g0 + j;
             if (!wait(&b.kv_full[g % kStages], (g / kStages) & 1)) break;
-            issue_s(0, g);
-            issue_s(1, g);
+            issue_s(t, g);
         }
         if (*failed) break;
-        if (nt <= 2 && leader) tc::commit(smem_addr(b.q_free));  // the item's last S issued
+        if (nt <= 2 && leader) tc::commit(smem_addr(b.q_free));  // the tile's last S issued
         for (int j = 0; j < nt; ++j) {
             const int g = g0 + j, buf = g & 1;
-            const uint32_t ph = (g >> 1) & 1;
-            const bool more = j + 2 < nt;
-            // tile A
-            if (!wait(&b.p_full[buf], ph)) break;
-            if (j == 0 && nk > 0 && !wait(&b.o_free[0], (nk - 1) & 1)) break;
+            if (!wait(&b.p_full[2 * t + buf], (g >> 1) & 1)) break;
+            if (j == 0 && nk > 0 && !wait(&b.o_free[t], (nk - 1) & 1)) break;
             // a bf16 V tile converted (it landed before its S)
             if (BF16 && !wait(&b.v_ready[g % kStages], (g / kStages) & 1)) break;
             const uint32_t vf =
                 BF16 ? *reinterpret_cast<const volatile uint32_t*>(vflags + g % kStages) : 0u;
-            issue_pv(0, g, j == 0, vf);
-            if (more) {
+            issue_pv(t, g, j == 0, vf);
+            if (leader) tc::commit(smem_addr(&b.kv_empty[g % kStages]));  // this tile's P V
+            if (j + 2 < nt) {
                 if (!wait(&b.kv_full[(g + 2) % kStages], ((g + 2) / kStages) & 1)) break;
-                issue_s(0, g + 2);
-            }
-            // tile B
-            if (!wait(&b.p_full[2 + buf], ph)) break;
-            if (j == 0 && nk > 0 && !wait(&b.o_free[1], (nk - 1) & 1)) break;
-            issue_pv(1, g, j == 0, vf);
-            if (leader) tc::commit(smem_addr(&b.kv_empty[g % kStages]));  // both P V of the stage
-            if (more) {
-                issue_s(1, g + 2);
-                if (j + 3 == nt && leader) tc::commit(smem_addr(b.q_free));  // the item's last S
+                issue_s(t, g + 2);
+                if (j + 3 == nt && leader) tc::commit(smem_addr(b.q_free));  // the tile's last S
             }
         }
         g0 += nt;
@@ -732,7 +725,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     if (threadIdx.x == 32 * kMmaWarp) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&b.kv_full[i], 2);  // the K and the V producer
-            mbar_init(&b.kv_empty[i], 1);
+            mbar_init(&b.kv_empty[i], 2);  // the P V of each Q tile
             mbar_init(&b.v_ready[i], kQWarps);
         }
         for (int t = 0; t < kQTiles; ++t) {
@@ -743,9 +736,9 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&b.o_done[t], 1);
             mbar_init(&b.o_free[t], 4);  // the tile's four softmax warps
         }
-        mbar_init(b.drain, 1);
+        mbar_init(b.drain, 2);     // both MMA warps
         mbar_init(b.q_ready, kQWarps);  // the Q warps
-        mbar_init(b.q_free, 1);   // a commit after the item's last S
+        mbar_init(b.q_free, 2);   // a commit after each Q tile's last S
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
@@ -758,9 +751,9 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     bool failed = false;
     if (warp == kProducerWarp || warp == kVProducerWarp)
         produce(kmap, vmap, p, stages, b, lane, warp == kVProducerWarp, &failed);
-    else if (warp == kMmaWarp)
+    else if (warp == kMmaWarp || warp == kMmaWarpB)
         issue_mmas<std::is_same<T, __nv_bfloat16>::value>(p, b, tmem, smem_addr(qsm), stages,
-                                                          vflags, &failed);
+                                                          vflags, warp == kMmaWarpB, &failed);
     else if (warp >= kQWarp0 && warp < kQWarp0 + kQWarps)
         stage_q<T>(p, b, qsm, stages, vflags, warp - kQWarp0, lane, &failed);
     else
