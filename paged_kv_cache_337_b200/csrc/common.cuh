@@ -116,14 +116,18 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 // Waits for the phase with the given parity to complete, for at most
-// limit_ns nanoseconds.  Returns false when the limit ran out.
+// limit_ns nanoseconds.  Returns false when the limit ran out.  The elapsed
+// time is a signed difference, so a global timer that steps back does not
+// end the wait (it lengthens it by the step).  The loop is kept this short
+// on purpose: waiting warps poll it, and every instruction it adds takes an
+// issue slot from the warps that work.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > limit_ns) return false;
+        if ((int64_t)(global_timer_ns() - t0) > (int64_t)limit_ns) return false;
     }
 }
 

@@ -582,39 +582,41 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
             // P as a bf16 high part and its bf16 remainder (two MMAs): one
             // bf16 rounding alone carries up to 2^-9 per weight.
             constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+            const float2 sl2 = make_float2(sl, sl), nmu2 = make_float2(-mu, -mu);
+            float2 ls[4] = {};
+            float2 w[kKeys / 2];
+#pragma unroll
+            for (int e = 0; e < kKeys / 2; ++e) {
+                const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nmu2);
+                w[e] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                ls[e & 3] = fadd2(ls[e & 3], w[e]);
+            }
+            // the V groups' format, once the exponentials are done
             uint32_t fl = 0x01010101u;  // one byte per 16-key group: 1 = f16
             if constexpr (kBf16) {
                 const int st = g % kStages;
                 if (!warp_wait(&b.v_ready[st], (g / kStages) & 1)) break;
                 fl = *reinterpret_cast<const volatile uint32_t*>(vflags + st);
             }
-            const float2 sl2 = make_float2(sl, sl), nmu2 = make_float2(-mu, -mu);
-            float2 ls[4] = {};
 #pragma unroll
             for (int c = 0; c < kKeys / 32; ++c) {
-                float2 w[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 x =
-                        ffma2(make_float2(sv[32 * c + 2 * e], sv[32 * c + 2 * e + 1]), sl2, nmu2);
-                    w[e] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    ls[e & 3] = fadd2(ls[e & 3], w[e]);
-                }
                 uint32_t hi[16], lo[16];
                 const uint32_t pair = (fl >> (16 * c)) & 0x0101u;  // groups 2c, 2c + 1
                 if (pair == 0x0101u) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) hi[e] = Storage<__half>::from_float2(w[e].x, w[e].y);
+                    for (int e = 0; e < 16; ++e)
+                        hi[e] = Storage<__half>::from_float2(w[16 * c + e].x, w[16 * c + e].y);
                     tc::st16(srow + 16 * c, hi);  // over S, already read
                 } else {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
+                        const float2 we = w[16 * c + e];
                         if ((pair >> (8 * (e >> 3))) & 1u) {
-                            hi[e] = Storage<__half>::from_float2(w[e].x, w[e].y);
+                            hi[e] = Storage<__half>::from_float2(we.x, we.y);
                             lo[e] = 0u;
                         } else {
-                            hi[e] = Storage<T>::from_float2(w[e].x, w[e].y);
-                            const float2 rem = fsub2(w[e], Storage<T>::to_float2(hi[e]));
+                            hi[e] = Storage<T>::from_float2(we.x, we.y);
+                            const float2 rem = fsub2(we, Storage<T>::to_float2(hi[e]));
                             lo[e] = Storage<T>::from_float2(rem.x, rem.y);
                         }
                     }
