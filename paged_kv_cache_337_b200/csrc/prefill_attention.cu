@@ -191,7 +191,7 @@ __device__ Item decode_item(const PrefillParams& p, int idx, bool report) {
     return it;
 }
 
-// Producers: warp 0 loads the K tiles, the last warp the V tiles, into the
+// Producers: warp 0 loads the K tiles, warp 14 the V tiles, into the
 // same ring stages (each stage's full barrier takes one arrival per
 // producer with its byte count).  A box past the context still loads a
 // block (the last one) so that every stage receives its full byte count;
@@ -259,7 +259,7 @@ __device__ void produce(const CUtensorMap& kmap, const CUtensorMap& vmap, const 
             mbar_wait_bounded(&b.kv_full[q % kStages], (q / kStages) & 1);
 }
 
-// MMA issuers: warp 1 for Q tile 0 and the last warp for Q tile 1, each in
+// MMA issuers: warp 1 for Q tile 0 and warp 15 for Q tile 1, each in
 // step; one elected lane issues each MMA and commit, the descriptors stay
 // warp-uniform.  A commit tracks the MMAs of the thread that executes it,
 // so the barriers both tiles release (a stage's kv_empty, q_free, drain)
