@@ -483,7 +483,7 @@ def grid_label(args, P, max_len, fp8):
     if wl == "auto":
         if not 0 < P < max_len:
             return "full grid (one pass per sequence)"
-        wl = "longest_first" if fp8 else "sequences_longest_first"
+        wl = "sequences_longest_first"
     if wl == "none":
         return "full grid"
     return "work list of the (sequence, KV head, partition) items holding tokens, " + {

@@ -49,9 +49,9 @@ class PagedKVCache:
 
         work_list: the decode grid.  "auto" (or True): the full grid when
         every sequence fits one partition, else the library's work list,
-        items longest first for an e4m3 cache and sequences longest first
-        for a 16-bit cache (the orders measured fastest on B200 for the
-        GQA and long-context batches); "longest_first",
+        sequences longest first (the order measured fastest on B200 for the
+        GQA batches, 16-bit and e4m3, and level with the others on the
+        long-context batches); "longest_first",
         "sequences_longest_first", "batch_order": the work list in that
         order on every step; False or "none": the full grid."""
         self.num_blocks = num_blocks
@@ -190,8 +190,7 @@ class PagedKVCache:
         if not self.work_list:
             return -1, -1
         if self._item_order is None:  # "auto"
-            return (_abi.PKV_ITEMS_LONGEST_FIRST if self.fp8 else
-                    _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST), -1
+            return _abi.PKV_ITEMS_SEQUENCES_LONGEST_FIRST, -1
         return self._item_order, self._item_order
 
     def prepare_step(self, seq_ids):

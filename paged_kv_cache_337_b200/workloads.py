@@ -72,11 +72,13 @@ DECODE_7B = DecodeSpec("7b_s256_h32_d128_bs16_bf16", 1002, 256, 32, 32, 128, 16,
                        128, 2048, "bf16")
 # The GQA configuration fixes no partition size.  Over a 16-bit cache 2048
 # tokens (about three waves of CTAs for this batch on 148 SMs) measured
-# fastest among 512-4096; an e4m3 token is half the bytes, and 4096 tokens
-# measured fastest there (2048: 4892 GB/s, 3072: 4943, 4096: 5277 on B200).
+# fastest among 512-4096; an e4m3 token is half the bytes, and 3584 tokens
+# with sequences longest first measured fastest there (2048: 4892 GB/s,
+# 3072: 4943, 4096: 5277 with items longest first; 3584: 5358-5368 with
+# sequences longest first, against 5271-5277 for 4096 in the same runs).
 # The long-context configuration fixes 512.
 GQA_70B = DecodeSpec("70b_gqa_s64_hq64_hkv8_d128_bs16_bf16", 1003, 64, 64, 8, 128,
-                     16, 512, 8192, "bf16", partition_size=2048, partition_size_e4m3=4096)
+                     16, 512, 8192, "bf16", partition_size=2048, partition_size_e4m3=3584)
 LONG_BS32 = DecodeSpec("long_s8_l32768_hq32_hkv8_d128_bs32_bf16", 1004, 8, 32, 8,
                        128, 32, 32768, 32768, "bf16", partition_size=512)
 LONG_BS64 = DecodeSpec("long_s8_l32768_hq32_hkv8_d128_bs64_bf16", 1004, 8, 32, 8,

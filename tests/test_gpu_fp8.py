@@ -221,12 +221,12 @@ def test_fp8_argument_errors_raise(cuda_device):
 def test_decode_fp8_gqa_shape_at_its_partition_size(work_list, cuda_device):
     """The 70B-shaped GQA layout (64 query / 8 KV heads, block size 16) over
     an e4m3 cache at the partition size that workload uses for e4m3 caches
-    (4096 tokens), lengths on and around the partition boundaries, on the
+    (3584 tokens), lengths on and around the partition boundaries, on the
     full grid and on the work list (items longest first)."""
     from paged_kv_cache_337_b200 import workloads as W
     P = W.GQA_70B.partition_for(True)
-    assert P == 4096
-    lens = [512, 4095, 4096, 4097, 8192, 6000, 1, 8191, 17, 4200]
+    assert P == 3584
+    lens = [512, 3583, 3584, 3585, 7168, 6000, 1, 7167, 17, 4200, 8192, 7169]
     p = fp8_problem(2024, 64, 8, 128, 16, lens, "bf16")
     scale = 1.0 / np.sqrt(128)
     dev = cuda_device
