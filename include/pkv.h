@@ -727,6 +727,14 @@ PKV_API int64_t pkv_block_bytes(int block_size, int num_kv_heads, int head_dim,
  * affected. */
 PKV_API int pkv_selftest_bounded_wait(int32_t* dev_error, int limit_us, cudaStream_t stream);
 
+/* Self-test of the 2^x that the prefill softmax takes from the FMA pipe for
+ * part of its exponentials (its own arithmetic; the pages give no
+ * exponential): y[i] = 2^x[i] for n fp32 values, x and y device arrays of n
+ * floats (0 <= n <= 2^28), launched on stream.  Within 3.0e-6 relative for
+ * x in [-126, 8]; +0 for x <= -127, -inf and NaN; subnormal below 2^-126
+ * for x in (-127, -126). */
+PKV_API int pkv_selftest_ex2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 PKV_API const char* pkv_status_string(int status);
 /* Message of the calling thread's last failed call ("" if none). */
 PKV_API const char* pkv_last_error(void);

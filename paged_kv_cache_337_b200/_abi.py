@@ -91,6 +91,7 @@ SIGNATURES = {
     "pkv_swap_blocks": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i64, _i64, _i64, _p, _p]),
     "pkv_block_bytes": (_i64, [_i, _i, _i, _i, _i]),
     "pkv_selftest_bounded_wait": (_i, [_p, _i, _p]),
+    "pkv_selftest_ex2_poly": (_i, [_p, _p, _i, _p]),
     "pkv_status_string": (C.c_char_p, [_i]),
     "pkv_last_error": (C.c_char_p, []),
     "pkv_version": (_i, []),
@@ -528,6 +529,18 @@ def pkv_selftest_bounded_wait(dev_error, limit_us, stream=None):
     _check(lib().pkv_selftest_bounded_wait(_ptr(dev_error), int(limit_us),
                                            _stream(stream, dev_error.device)),
            "pkv_selftest_bounded_wait")
+
+
+def pkv_selftest_ex2_poly(x, y, stream=None):
+    """y = 2^x elementwise by the prefill softmax's FMA-pipe exponential
+    (float32 device tensors of one size)."""
+    _on_device("pkv_selftest_ex2_poly", x, y)
+    _need(x, torch.float32, "x")
+    _need(y, torch.float32, "y")
+    if x.numel() != y.numel():
+        raise ValueError("x and y differ in size")
+    _check(lib().pkv_selftest_ex2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream, x.device)),
+           "pkv_selftest_ex2_poly")
 
 
 def pkv_block_bytes(block_size, num_kv_heads, head_dim, num_layers, dtype_bytes):

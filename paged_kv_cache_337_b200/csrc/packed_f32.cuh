@@ -1,6 +1,7 @@
 // packed_f32.cuh — fp32 arithmetic on sm_100a that takes a pair of floats
-// per instruction (fma/add/sub .f32x2), the three-input maximum, and the
-// hardware 2^x approximation.
+// per instruction (fma/add/sub .f32x2), the three-input maximum, the
+// hardware 2^x approximation and a 2^x on a pair from FMA-pipe arithmetic
+// alone.
 #pragma once
 
 namespace pkv {
@@ -66,6 +67,46 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// a + b on a pair, rounded toward minus infinity
+__device__ __forceinline__ float2 fadd2_rm(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// 2^x on a pair without the exponential unit: FMA-pipe arithmetic only, so
+// that a softmax can split its exponentials between the two pipes (as
+// FlashAttention-4 does on Blackwell).  For x <= 2^22:
+//   - x is clamped to -127 below (-inf and NaN included);
+//   - adding 1.5 * 2^23 rounded down leaves floor(x) = j as an integer in
+//     the low mantissa bits of the sum t, and f = x - j in [0, 1) is exact;
+//   - 2^f comes from a degree-4 polynomial with constant term 1, its other
+//     coefficients fitted here by linear programming to the least maximum
+//     relative error over [0, 1] (3.0e-6, evaluated in fp32);
+//   - 2^j is added into the exponent field: t's bits shifted left by 23
+//     are j << 23 modulo 2^32.
+// So x = -127 gives exactly +0 (the polynomial's 1.0 carries exponent 127)
+// and x in (-127, -126) a subnormal below 2^-126; from -126 up the result
+// is 2^x within the fit's error.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -127.f);
+    x.y = fmaxf(x.y, -127.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+    const float2 t = fadd2_rm(x, magic);
+    const float2 f = fsub2(x, fsub2(t, magic));
+    float2 q = ffma2(make_float2(0x1.b7ea5cp-7f, 0x1.b7ea5cp-7f), f,
+                     make_float2(0x1.abfe7ep-5f, 0x1.abfe7ep-5f));
+    q = ffma2(q, f, make_float2(0x1.ee2374p-3f, 0x1.ee2374p-3f));
+    q = ffma2(q, f, make_float2(0x1.62d6d0p-1f, 0x1.62d6d0p-1f));
+    q = ffma2(q, f, make_float2(1.f, 1.f));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 }  // namespace pkv

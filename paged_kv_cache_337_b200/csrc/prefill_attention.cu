@@ -27,7 +27,9 @@
 //     neither tile's issue waits behind the other's P;
 //   - eight softmax warps, four per Q tile (one tensor-memory lane quarter
 //     each, one row per thread), read S, apply the causal mask, keep the
-//     running max and sum, write P over S (one f16 rounding; a bf16 high
+//     running max and sum, take a quarter of the exponentials from an
+//     FMA-pipe polynomial and the rest from the exponential unit, write P
+//     over S (one f16 rounding; a bf16 high
 //     part and its remainder, two MMAs, for a bf16 V group beyond f16's
 //     range) and rescale O when the running max grows by more than 2^8,
 //     then write the normalised output;
@@ -67,8 +69,9 @@ constexpr int kThreads = (kMmaWarpB + 1) * 32;
 // 256 t + 64, O at 256 t + 128; key tile j uses S buffer j % 2
 constexpr uint32_t kTileCols = 256, kColO = 128, kColPl = kKeys / 2, kTmemCols = 512;
 // kv_full/kv_empty/v_ready per stage; s_full/p_full per (Q tile, S
-// buffer); o_done and o_free per Q tile; drain, q_ready, q_free
-constexpr int kNumBars = 3 * kStages + 6 * kQTiles + 3;
+// buffer); o_done and o_free per Q tile; drain, q_ready, q_free; item_done
+// per Q tile
+constexpr int kNumBars = 3 * kStages + 7 * kQTiles + 3;
 // after the barriers: the tensor-memory address (16 bytes) and, per stage,
 // one byte per 16-key group of V: 1 = converted to f16, 0 = left in bf16
 constexpr size_t kSmemBytes = 1024 + kQBytes + kStages * kStageBytes + kNumBars * 8 + 16 + 16;
@@ -113,6 +116,16 @@ __device__ __forceinline__ void mbar_arrive_one(uint64_t* bar) {
 #endif
 constexpr bool kL2Hints = PKV_PREFILL_L2_HINTS != 0;
 
+// Of every eight key pairs of a softmax pass, how many take 2^x from the
+// FMA-pipe polynomial (ex2_poly2) instead of the exponential unit.  The
+// softmax is bound by instruction issue more than by the exponential unit:
+// two of eight measured fastest, each pair moved beyond that slower.
+#ifndef PKV_PREFILL_POLY_EXP
+#define PKV_PREFILL_POLY_EXP 2
+#endif
+constexpr int kPolyPairsPer8 = PKV_PREFILL_POLY_EXP;
+static_assert(kPolyPairsPer8 >= 0 && kPolyPairsPer8 <= 8, "pairs of eight");
+
 // 16-byte copy global -> shared that does not wait (cp.async, L2 only);
 // when copy is false, the destination is zero-filled and nothing is read
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src, bool copy,
@@ -144,6 +157,7 @@ struct Bars {
     uint64_t* drain;     // every MMA issued completed (exit)
     uint64_t* q_ready;   // the Q tiles of the next item are staged
     uint64_t* q_free;    // every S MMA of the item completed: Q may be restaged
+    uint64_t* item_done; // [kQTiles]: the item's last P V of the Q tile completed
 };
 
 // One work item: 256 rows of one (sequence, KV head).
@@ -366,6 +380,9 @@ __device__ void issue_mmas(const PrefillParams& p, const Bars& b, uint32_t tmem,
                 if (j + 3 == nt && leader) tc::commit(smem_addr(b.q_free));  // the tile's last S
             }
         }
+        // one phase per item: every MMA of this tile so far, its last P V
+        // included, completed
+        if (!*failed && leader) tc::commit(smem_addr(&b.item_done[t]));
         g0 += nt;
         ++nk;
     }
@@ -510,6 +527,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
     const int r = 32 * quarter + lane;
     const float sl = p.scale_log2;
     int g0 = 0;  // first key tile of the item, counted over all items
+    int ni = 0;  // items run so far (the phase of item_done)
     for (int k = 0; !*failed; ++k) {
         const int idx = item_index(k);
         if (idx >= p.num_items) break;
@@ -588,7 +606,10 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
 #pragma unroll
             for (int e = 0; e < kKeys / 2; ++e) {
                 const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), sl2, nmu2);
-                w[e] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                if ((e & 7) < kPolyPairsPer8)
+                    w[e] = ex2_poly2(x);
+                else
+                    w[e] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                 ls[e & 3] = fadd2(ls[e & 3], w[e]);
             }
             // the V groups' format, once the exponentials are done
@@ -648,11 +669,13 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
             __syncwarp();
             if (lane == 0) mbar_arrive_one(&b.p_full[2 * t + buf]);
         }
-        // the item's last two P V (phases ge - 2 and ge - 1 of o_done), in
-        // order; the previous item's were waited for at its end
+        // The item's last P V, through item_done (phase ni, one per item;
+        // the next needs this item's o_free, so the wait cannot alias).  A
+        // parity wait is sound only while its barrier is at most one phase
+        // past the phase waited for; o_done, one phase per key tile, can
+        // here be one or two phases past P V ge - 2.
         const int ge = g0 + it.ntiles;
-        if (j < it.ntiles || (it.ntiles >= 2 && !warp_wait(&b.o_done[t], (ge - 2) & 1)) ||
-            !warp_wait(&b.o_done[t], (ge - 1) & 1)) {
+        if (j < it.ntiles || !warp_wait(&b.item_done[t], ni & 1)) {
             *failed = true;
             break;
         }
@@ -692,6 +715,7 @@ __device__ void softmax_rows(const PrefillParams& p, const Bars& b, uint32_t tme
         __syncwarp();
         if (lane == 0) mbar_arrive_one(&b.o_free[t]);
         g0 = ge;
+        ++ni;
     }
 }
 
@@ -717,7 +741,8 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
            sp + 5 * kQTiles,
            tail,
            tail + 1,
-           tail + 2};
+           tail + 2,
+           tail + 3};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (warp == kProducerWarp) {
@@ -737,6 +762,7 @@ paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             mbar_init(&b.o_done[t], 1);
             mbar_init(&b.o_free[t], 4);  // the tile's four softmax warps
+            mbar_init(&b.item_done[t], 1);
         }
         mbar_init(b.drain, 2);     // both MMA warps
         mbar_init(b.q_ready, kQWarps);  // the Q warps

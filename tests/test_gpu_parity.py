@@ -332,3 +332,38 @@ def test_bounded_wait_expires_and_reports(cuda_device):
     got = gpu_decode(p, 2, 16, 0.125, 0, cuda_device)
     want = oracle_decode(p, 2, 16, 0.125, "bf16")
     assert tolerance_violation(got, want, ATOL, RTOL) <= 0
+
+
+def test_fma_pipe_exp2_within_its_bound(cuda_device):
+    """The 2^x the prefill softmax takes from the FMA pipe for part of its
+    exponentials, held to the exact power of two: within 3.0e-6 relative on
+    [-126, 8] (the softmax's range is (-inf, 8]), exact at integers, +0 at
+    and below -127 (masked scores, -inf, NaN), and between 0 and 2^-126 in
+    (-127, -126)."""
+    rng = np.random.default_rng(5)
+    dense = np.linspace(-126.0, 8.0, 1_000_003, dtype=np.float32)
+    near = (np.arange(-126, 8)[:, None] + np.float32(1) - rng.random((134, 64)) * 1e-5)
+    x = np.concatenate([dense, near.astype(np.float32).ravel(),
+                        rng.uniform(-126, 8, 200_000).astype(np.float32)])
+    xt = torch.from_numpy(x).to(cuda_device)
+    y = torch.empty_like(xt)
+    _abi.pkv_selftest_ex2_poly(xt, y)
+    got = y.cpu().double().numpy()
+    rel = np.abs(got / np.exp2(x.astype(np.float64)) - 1.0)
+    assert rel.max() <= 3.0e-6, rel.max()
+    ints = np.arange(-126, 9, dtype=np.float32)
+    edges = np.array([-127.0, -128.0, -1e30, -np.inf, np.nan], np.float32)
+    sub = np.array([-126.999, -126.5, -126.001], np.float32)
+    xt = torch.from_numpy(np.concatenate([ints, edges, sub])).to(cuda_device)
+    y = torch.full_like(xt, 7.0)
+    _abi.pkv_selftest_ex2_poly(xt, y)
+    got = y.cpu().double().numpy()
+    assert (got[:len(ints)] == np.exp2(ints.astype(np.float64))).all()
+    assert (got[len(ints):len(ints) + len(edges)] == 0.0).all()
+    tail = got[len(ints) + len(edges):]
+    assert ((tail >= 0.0) & (tail <= 2.0 ** -126)).all()
+    # an odd count: the last element has no partner
+    xt = torch.tensor([1.5, -0.25, 3.0], device=cuda_device)
+    y = torch.zeros_like(xt)
+    _abi.pkv_selftest_ex2_poly(xt, y)
+    assert np.allclose(y.cpu().double().numpy(), np.exp2([1.5, -0.25, 3.0]), rtol=3.0e-6, atol=0)
