@@ -60,6 +60,10 @@ PROFILE_TRAFFIC = {
                                                           "decode_attention_gqa_70b.md"),
     "70b_gqa_s64_hq64_hkv8_d128_bs16_bf16_kv_e4m3": os.path.join(
         ROOT, "profiles", "decode_attention_fp8_gqa_70b.md"),
+    "long_s8_l32768_hq32_hkv8_d128_bs32_bf16": os.path.join(ROOT, "profiles",
+                                                             "decode_attention_long_bs32.md"),
+    "long_s8_l32768_hq32_hkv8_d128_bs64_bf16": os.path.join(ROOT, "profiles",
+                                                             "decode_attention_long_bs64.md"),
     "prefill_s8_l2048_hq32_hkv8_d128_bs16_bf16": os.path.join(ROOT, "profiles",
                                                                "prefill_attention_s8_l2048.md"),
 }

@@ -45,7 +45,7 @@ def test_traffic_only_with_the_recorded_digest(bench):
 
 def test_no_traffic_for_a_workload_without_a_summary(bench):
     digest = bench.kernel_source_digest()
-    assert bench.profiled_traffic(digest, "long_s8_l32768_hq32_hkv8_d128_bs32_bf16") is None
+    assert bench.profiled_traffic(digest, "shared_prefix_p16x8_pre1024_h32_d128_bs16_bf16") is None
     assert bench.profiled_traffic(digest, "no_such_workload") is None
 
 
