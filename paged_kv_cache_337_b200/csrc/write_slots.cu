@@ -7,6 +7,10 @@
 // the source and, inside its block, in the cache, so the kernel is a gather
 // of 16-byte vectors: one thread per vector, K and V in one launch, slots
 // read once per vector from L1.  Bound: HBM (read + write of the rows).
+// The two divisions per vector (vector -> token, slot -> block) run in
+// 32-bit arithmetic whenever the launch's vector and slot counts allow: a
+// 64-bit division is a long instruction sequence, and with two per 16-byte
+// vector it made a prompt-sized write issue-bound.
 #include "common.cuh"
 
 namespace pkv {
@@ -14,31 +18,36 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// I: the type of the vector, token and slot indexes (uint32_t when every
+// one of them, and the grid stride past the last, fits; else int64_t).
+// Addresses are formed in 64 bits either way.
+template <typename I>
 __global__ void __launch_bounds__(kThreads)
 write_slots_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
                    uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
                    const int64_t* __restrict__ slot_mapping, int num_tokens,
-                   int64_t num_slots, int block_size, int64_t row_vecs,
+                   int64_t num_slots, int block_size, I row_vecs,
                    int64_t block_stride_vecs, int32_t* __restrict__ dev_error) {
     // work item i: token i / (2 * row_vecs), K (first half) or V, vector
-    const int64_t per_token = 2 * row_vecs;
-    const int64_t total = (int64_t)num_tokens * per_token;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = i / per_token;
-        const int64_t r = i - t * per_token;
+    const I per_token = 2 * row_vecs;
+    const I total = (I)num_tokens * per_token;
+    const I bs = (I)block_size;
+    for (I i = (I)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (I)gridDim.x * blockDim.x) {
+        const I t = i / per_token;
+        const I r = i - t * per_token;
         const int64_t slot = __ldg(slot_mapping + t);
         if (slot < 0) continue;  // padding token
         if (slot >= num_slots) {
             if (r == 0) report_error(dev_error, PKV_DEVERR_SLOT, (int)t);
             continue;
         }
-        const int64_t blk = slot / block_size;
-        const int64_t off = slot - blk * block_size;
+        const I blk = (I)slot / bs;
+        const I off = (I)slot - blk * bs;
         const bool is_v = r >= row_vecs;
-        const int64_t v = is_v ? r - row_vecs : r;
-        const int64_t dst = blk * block_stride_vecs + off * row_vecs + v;
-        const int64_t src = t * row_vecs + v;
+        const I v = is_v ? r - row_vecs : r;
+        const int64_t dst = (int64_t)blk * block_stride_vecs + (int64_t)off * row_vecs + v;
+        const int64_t src = (int64_t)t * row_vecs + v;
         if (is_v)
             value_cache[dst] = __ldg(value + src);
         else
@@ -75,13 +84,23 @@ extern "C" int pkv_write_slots(const void* key, const void* value, void* key_cac
     DeviceGuard guard(stream, key_cache);
     const int64_t row_vecs = row / 8;
     const int64_t total = (int64_t)num_tokens * 2 * row_vecs;
+    const int64_t num_slots = (int64_t)num_blocks * block_size;
     int64_t grid = (total + kThreads - 1) / kThreads;
     if (grid > 148 * 64) grid = 148 * 64;  // grid-stride beyond 64 CTAs per SM
-    write_slots_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
-        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), slot_mapping,
-        num_tokens, (int64_t)num_blocks * block_size, block_size, row_vecs, block_stride / 8,
-        dev_error);
+    const auto* k = static_cast<const uint4*>(key);
+    const auto* v = static_cast<const uint4*>(value);
+    auto* kc = static_cast<uint4*>(key_cache);
+    auto* vc = static_cast<uint4*>(value_cache);
+    // 32-bit indexes: the vectors, the slots and the grid stride past the
+    // last vector all below 2^31
+    if (total + grid * kThreads < (int64_t(1) << 31) && num_slots < (int64_t(1) << 31))
+        write_slots_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+            k, v, kc, vc, slot_mapping, num_tokens, num_slots, block_size, (uint32_t)row_vecs,
+            block_stride / 8, dev_error);
+    else
+        write_slots_kernel<int64_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+            k, v, kc, vc, slot_mapping, num_tokens, num_slots, block_size, row_vecs,
+            block_stride / 8, dev_error);
     return launch_status("pkv_write_slots");
 }
 
