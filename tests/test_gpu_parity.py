@@ -129,6 +129,39 @@ def test_split_k_agrees_with_single_pass(cuda_device):
         assert tolerance_violation(outs[P], outs[0].double().numpy(), ATOL, RTOL) <= 0
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 4)])
+def test_split_k_repeated_launches_agree_bit_for_bit(Hq, Hkv, cuda_device):
+    """The split-K merge over 200 back-to-back launches on one workspace:
+    the partition counters start from zero each time (cleared before the
+    launch and reset by the merging CTA), no device error is recorded, and
+    every launch gives the first one's output bit for bit (the partials are
+    merged in partition order, whichever CTA arrives last)."""
+    p = paged_problem(12, Hq, Hkv, 128, 16, [1500, 3, 700, 2048, 64, 1025], "bf16")
+    dev = cuda_device
+    q, kc, vc = p["q"].to(dev), p["kc"].to(dev), p["vc"].to(dev)
+    tables, lens = to_dev(p["tables"], dev), to_dev(p["lens"], dev)
+    max_len, P, scale = int(max(p["lens"])), 256, 1.0 / np.sqrt(128)
+    ws = torch.empty(_abi.pkv_decode_workspace_bytes(q.shape[0], Hq, max_len, P, 128),
+                     dtype=torch.uint8, device=dev)
+    err = torch.zeros(2, dtype=torch.int32, device=dev)
+    first = torch.full_like(q, float("nan"))
+    _abi.pkv_decode_attention(first, q, kc, vc, tables, lens, max_len, scale, P, ws,
+                              dev_error=err)
+    out = torch.empty_like(first)
+    mismatches = torch.zeros((), dtype=torch.int64, device=dev)
+    for _ in range(200):
+        out.fill_(float("nan"))
+        _abi.pkv_decode_attention(out, q, kc, vc, tables, lens, max_len, scale, P, ws,
+                                  dev_error=err)
+        mismatches += (out.view(torch.int16) != first.view(torch.int16)).sum()
+    torch.cuda.synchronize()
+    assert err.tolist() == [0, 0]
+    assert int(mismatches) == 0
+    assert torch.isfinite(first).all()
+    want = oracle_decode(p, Hkv, 16, scale, "bf16")
+    assert tolerance_violation(first.cpu(), want, ATOL, RTOL) <= 0
+
+
 def test_combined_kv_layout_via_block_stride(cuda_device):
     """One [NB, 2, bs, Hkv, D] tensor: K and V views with block stride
     2 * bs * Hkv * D."""
