@@ -81,3 +81,12 @@ def test_prefill_rejects_a_non_positive_scale_before_any_device_work():
                                  8, 16, 16 * 4 * 128, 0.0, _abi.PKV_BF16, None, None)
     assert st == _abi.PKV_ERR_INVALID
     assert b"scale" in L.pkv_last_error()
+
+
+def test_ex2_selftest_checks_its_count_before_any_device_work(lib):
+    # a count outside 0 .. 2^28 is refused, and a count of zero is a no-op,
+    # both before any pointer or device access
+    for n in (-1, (1 << 28) + 1):
+        assert lib.pkv_selftest_ex2_poly(None, None, n, None) == _abi.PKV_ERR_INVALID
+        assert b"pkv_selftest_ex2_poly" in lib.pkv_last_error()
+    assert lib.pkv_selftest_ex2_poly(None, None, 0, None) == _abi.PKV_OK
